@@ -1,0 +1,154 @@
+"""CPU oracle for the ARL2 hybrid-attention hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the package's ``smoke()`` check and the benchmark's CPU
+baseline may import this module.  The CUDA path never calls it, and it shares
+no code with the CUDA path: it is the plain definition of what one hybrid
+layer computes, in numpy float64, with no blocking, fusion or reordering.
+
+Sources.  "ARL2 summary" below is the technical summary on the page
+"Attend Locally, Remember Linearly: Linear Attention as Cross-Frame Memory for
+Autoregressive Video Diffusion" (gist.science, German; the Italian, Japanese
+and Korean pages of the same site carry the same text).  "ARL2 abstract" is
+the authors' English abstract of arXiv 2605.16579v2 as shown on the
+fugumt.com paper_check page.
+
+Layouts (those of the C ABI): Q, K, V, O are [B, L, H, d] (token-major);
+phi_* are [H, d, d] with Q' = Q @ phi_q; S is [B, H, d_k, d_v]; alpha is
+[B, H] (one gate per stream and head for the frame); beta is [B, H, L].
+
+Readings of the pages that this file fixes (each is listed with its reason
+in the design notes of the repository):
+
+* the update's lost transposes: the delta term is K'^T diag(beta)(V' - K'S);
+* K' is L2-normalised per token, max(||k||, 1e-12) in the denominator; Q'
+  and V' are not normalised; the phi maps are plain d x d matrices;
+* alpha is one scalar per (stream, head, frame); beta one value per token;
+* O = O_intra + O_inter, with no gate or normalisation between them;
+* the delta correction carries an explicit coefficient c (``corr_scale``);
+  c = 1 is the literal formula, c = 1/L the mean over the frame's tokens.
+
+Parity status: the intra branch, the read-out and the update are each pinned
+by brute force on tiny inputs, closed forms and invariants (tests marked
+"not gpu").  The values of a full frame at the benchmark shapes are pinned
+only through those same definitions: the pages print no worked numbers.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "feature_maps", "intra_softmax", "inter_readout", "frame_query",
+    "frame_commit", "kv_attention", "stream_reference",
+]
+
+EPS_NORM = 1e-12
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def _heads_first(x: np.ndarray) -> np.ndarray:
+    """[B, L, H, d] -> [B, H, L, d]."""
+    return np.ascontiguousarray(x.transpose(0, 2, 1, 3))
+
+
+def _tokens_first(x: np.ndarray) -> np.ndarray:
+    """[B, H, L, d] -> [B, L, H, d]."""
+    return np.ascontiguousarray(x.transpose(0, 2, 1, 3))
+
+
+def feature_maps(Q, K, V, phi_q, phi_k, phi_v):
+    """Per-head grouped 1x1 feature maps (ARL2 summary, §2.1, "Anpassung"):
+    Q' = Q phi_q, K' = rownorm_2(K phi_k), V' = V phi_v, each [B, H, L, d]."""
+    Qh, Kh, Vh = (_heads_first(_f64(t)) for t in (Q, K, V))
+    Qp = Qh @ _f64(phi_q)[None]
+    Kt = Kh @ _f64(phi_k)[None]
+    Vp = Vh @ _f64(phi_v)[None]
+    norm = np.sqrt(np.sum(Kt * Kt, axis=-1, keepdims=True))
+    Kp = Kt / np.maximum(norm, EPS_NORM)
+    return Qp, Kp, Vp
+
+
+def intra_softmax(Q, K, V, scale=None):
+    """Intra-frame branch (ARL2 summary, §2.1, "Intra-Frame-Zweig"): the
+    original bidirectional softmax attention over the tokens of one frame,
+    on the unmapped Q, K, V; no mask.  Q may hold any subset of the frame's
+    query tokens.  Returns [B, Lq, H, d]."""
+    Qh, Kh, Vh = (_heads_first(_f64(t)) for t in (Q, K, V))
+    d = Qh.shape[-1]
+    scale = d ** -0.5 if scale is None else float(scale)
+    s = (Qh @ np.swapaxes(Kh, -1, -2)) * scale
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    O = (p @ Vh) / p.sum(axis=-1, keepdims=True)
+    return _tokens_first(O)
+
+
+def inter_readout(Qp, S):
+    """Inter-frame read-out (ARL2 summary, §2.1, "Ausgabe"): O_inter = Q' S,
+    with Q' [B, H, L, d_k] and S [B, H, d_k, d_v].  Returns [B, L, H, d_v]."""
+    return _tokens_first(_f64(Qp) @ _f64(S))
+
+
+def frame_query(S, Q, K, V, phi, scale=None):
+    """One denoising step: O = O_intra + Q' S_{N-1}.  The state is only read
+    (ARL2 summary, §2.2, "Clean-Pass-Aktualisierungen"); every token reads the
+    same S_{N-1} (§2.2, "Frame-Level-Zugriff")."""
+    phi_q, phi_k, phi_v = phi
+    Qp = _heads_first(_f64(Q)) @ _f64(phi_q)[None]
+    return intra_softmax(Q, K, V, scale) + inter_readout(Qp, S)
+
+
+def frame_commit(S, Q, K, V, phi, alpha, beta, corr_scale=1.0, scale=None):
+    """The clean pass of frame N: the output from S_{N-1}, then the single
+    state write of the frame (ARL2 summary, §2.1 "Zustandsaktualisierung" and
+    §2.2; ARL2 abstract: update only after the denoised pass, all tokens
+    share the pre-update state):
+
+        S_N = alpha_N S_{N-1} + c K'^T diag(beta) (V' - K' S_{N-1}).
+
+    Returns (O [B, L, H, d], S_N [B, H, d, d])."""
+    S = _f64(S)
+    O = frame_query(S, Q, K, V, phi, scale)
+    _, Kp, Vp = feature_maps(Q, K, V, *phi)
+    R = _f64(beta)[..., None] * (Vp - Kp @ S)
+    delta = np.swapaxes(Kp, -1, -2) @ R
+    S_new = _f64(alpha)[..., None, None] * S + float(corr_scale) * delta
+    return O, S_new
+
+
+def kv_attention(Q, K_ctx, V_ctx, scale=None):
+    """A softmax layer kept from the teacher, over a growing key-value cache
+    (ARL2 summary, §1, KV-cache growth): the queries of frame n attend to the
+    clean keys and values of frames 0..n-1 followed by the current pass's own
+    keys and values, with no mask.  K_ctx and V_ctx are that concatenation,
+    [B, Lk, H, d]."""
+    return intra_softmax(Q, K_ctx, V_ctx, scale)
+
+
+def stream_reference(inputs, frames, queries, corr_scale, phi, S0=None, scale=None,
+                     keep_outputs=True):
+    """Run a hybrid layer over a stream: for each frame, ``queries`` query
+    passes and one commit.  ``inputs(frame, pas)`` returns (Q, K, V) and
+    ``gates(frame)`` the pair (alpha, beta); both are supplied by the caller
+    as ``inputs = (qkv_fn, gates_fn)``.  Returns the list of per-frame output
+    lists and the list of states S_1..S_F."""
+    qkv_fn, gates_fn = inputs
+    Q0, _, _ = qkv_fn(0, 0)
+    B, L, H, d = Q0.shape
+    S = np.zeros((B, H, d, d)) if S0 is None else _f64(S0)
+    outs, states = [], []
+    for n in range(frames):
+        frame_out = []
+        for p in range(queries):
+            Q, K, V = qkv_fn(n, p)
+            O = frame_query(S, Q, K, V, phi, scale)
+            frame_out.append(O if keep_outputs else None)
+        Q, K, V = qkv_fn(n, queries)
+        alpha, beta = gates_fn(n)
+        O, S = frame_commit(S, Q, K, V, phi, alpha, beta, corr_scale, scale)
+        frame_out.append(O if keep_outputs else None)
+        outs.append(frame_out)
+        states.append(S)
+    return outs, states
