@@ -1,0 +1,458 @@
+#!/usr/bin/env python3
+"""Throughput of the ARL2 hybrid-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl arl2|reference]
+                    [--config 1|2|4] [--no-graphs]
+
+One step = one frame of one hybrid layer: 4 query-only denoising passes and
+one clean commit (intra softmax + inter read-out on every pass, the state
+write on the commit), 1560 tokens per frame, 12 heads x 128.  The default
+workload is the single-layer bf16 stream (batch 1); its inputs cycle through a
+pool of 20 (Q, K, V) triples, 288 MB, larger than the 126 MB L2, with a reuse
+distance of 20 passes.  Rank 0 prints one JSON line.
+
+Under torchrun each rank runs independent streams of its own (weak scaling,
+replicas only: the path has no exchange step); the job's value is the frames
+of all ranks divided by the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hybrid_linear_attention_arl2_b200 import workloads as W  # noqa: E402
+
+TOKENS_PER_STEP = None  # set from the config
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="arl2", choices=["arl2", "reference"])
+    ap.add_argument("--config", type=int, default=1, choices=[1, 2, 4])
+    ap.add_argument("--no-graphs", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-small", action="store_true",
+                    help="a few steps, no extras: for ncu captures of the kernels")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ flop / byte accounting
+def frame_flops(cfg: W.Config) -> dict:
+    """Algorithmic flops of one frame of one hybrid layer (all streams)."""
+    B, H, d, L, P = cfg.batch, cfg.heads, cfg.head_dim, cfg.tokens, cfg.passes
+    intra = 4.0 * L * L * d * H * B            # QK^T and PV, per pass
+    readout = 2.0 * L * d * d * H * B          # Q (phi_q S), per pass
+    maps = 2 * 2.0 * L * d * d * H * B         # K phi_k and V phi_v, commit
+    ks = 2.0 * L * d * d * H * B               # K' S, commit
+    delta = 2.0 * L * d * d * H * B            # K'^T R, commit
+    prep = 2.0 * d * d * d * H * B             # phi_q S_N, commit
+    return {"attn_per_pass": intra + readout, "frame": P * (intra + readout) + maps + ks + delta + prep}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# ------------------------------------------------------------------ device workload
+class DeviceStream:
+    """Device-resident inputs of one stream set (pool of triples, gates, phi)."""
+
+    def __init__(self, cfg: W.Config, seed_offset: int, device):
+        import torch
+        self.cfg = cfg
+        wl = W.Workload(cfg, seed=cfg.seed + 100 * seed_offset)
+        self.wl = wl
+        to = lambda x: torch.from_numpy(x).to(torch.bfloat16).to(device)
+        self.phi = tuple(to(p) for p in wl.phi(0))
+        self.pool = []
+        for i in range(cfg.pool):
+            per = [wl.pool_entry(b, i) for b in range(cfg.batch)]
+            self.pool.append(tuple(to(np.stack([t[j] for t in per])) for j in range(3)))
+        self.device = device
+
+    def gates(self, frame: int):
+        return self.wl.alpha(0, frame), self.wl.beta(0, frame)
+
+    def triple(self, frame: int, pas: int):
+        return self.pool[self.wl.pool_index(0, frame, pas)]
+
+
+def run_arl2(args, rank: int, world: int):
+    import torch
+    from hybrid_linear_attention_arl2_b200 import arl2
+
+    cfg = W.CONFIGS[args.config]
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    arl2.load_library()
+    ds = DeviceStream(cfg, rank, device)
+    stream = torch.cuda.Stream(device)
+    B, H, L, d = cfg.batch, cfg.heads, cfg.tokens, cfg.head_dim
+    flops = frame_flops(cfg)
+
+    with torch.cuda.stream(stream):
+        layer = arl2.HybridLayer(B, H, d, L, arl2.ARL2_BF16, *ds.phi, corr_scale=cfg.corr_scale, stream=stream)
+        O = torch.empty((B, L, H, d), dtype=torch.bfloat16, device=device)
+        period = 4  # frames per graph: pool phase (20 passes) and state ping-pong both repeat
+        gate_a = [torch.empty((B, H), dtype=torch.float32, device=device) for _ in range(period)]
+        gate_b = [torch.empty((B, H, L), dtype=torch.float32, device=device) for _ in range(period)]
+        # every frame's gates staged on the device before any timing: the timed
+        # loop only copies them into the per-slot buffers the graph reads
+        n_frames = args.warmup + args.steps + 2 * period
+        ga_all = torch.empty((n_frames, B, H), dtype=torch.float32, device=device)
+        gb_all = torch.empty((n_frames, B, H, L), dtype=torch.float32, device=device)
+        for f in range(n_frames):
+            a, b = ds.gates(f)
+            ga_all[f].copy_(torch.from_numpy(a))
+            gb_all[f].copy_(torch.from_numpy(b))
+
+        def load_gates(frame):
+            slot = frame % period
+            gate_a[slot].copy_(ga_all[frame], non_blocking=True)
+            gate_b[slot].copy_(gb_all[frame], non_blocking=True)
+
+        def frame_calls(frame, ev=None):
+            for p in range(cfg.passes):
+                q, k, v = ds.triple(frame, p)
+                if p < cfg.queries:
+                    if ev is not None:
+                        ev[p][0].record(stream)
+                    arl2.arl2_frame_query(layer.handle, q, k, v, O, stream)
+                    if ev is not None:
+                        ev[p][1].record(stream)
+                else:
+                    slot = frame % period
+                    arl2.arl2_frame_commit(layer.handle, q, k, v, gate_a[slot], gate_b[slot], O, stream)
+
+        # warm-up (eager): also exercises every kernel once before any capture
+        for f in range(args.warmup):
+            load_gates(f)
+            frame_calls(f)
+        stream.synchronize()
+        err = layer.last_error()
+        if err:
+            raise RuntimeError(f"device error during warm-up: {arl2.STATUS.get(err)}")
+
+        use_graphs = not args.no_graphs
+        graphs = None
+        if use_graphs:
+            # One graph = `period` frames; the handle's ping-pong parity and the
+            # pool phase both return to their start after it.
+            start = args.warmup
+            graph = torch.cuda.CUDAGraph()
+            for f in range(start, start + period):
+                load_gates(f)
+            stream.synchronize()
+            # external events become event-record nodes of the graph: they time
+            # every query launch of each replay on the launching stream
+            graph_ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                         torch.cuda.Event(enable_timing=True, external=True))
+                        for _ in range(period * cfg.queries)]
+            with torch.cuda.graph(graph, stream=stream):
+                for i, f in enumerate(range(start, start + period)):
+                    frame_calls(f, graph_ev[i * cfg.queries:(i + 1) * cfg.queries])
+            graphs = graph
+            stream.synchronize()
+
+        clocks = ClockSampler(local)
+        if dist is not None:
+            dist.barrier()
+        stream.synchronize()
+        torch.cuda.synchronize()
+        clocks.start()
+        time.sleep(0.3)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        attn_ev = []
+        f = args.warmup
+        if use_graphs:
+            # kernel timing: attention-only events around one captured query per graph replay
+            t0.record(stream)
+            steps_done = 0
+            while steps_done < args.steps:
+                for j in range(period):
+                    load_gates(f + j)
+                graphs.replay()
+                f += period
+                steps_done += period
+            t1.record(stream)
+        else:
+            t0.record(stream)
+            for s in range(args.steps):
+                load_gates(f)
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(cfg.queries)]
+                frame_calls(f, ev)
+                attn_ev.extend(ev)
+                f += 1
+            t1.record(stream)
+            steps_done = args.steps
+        t1.synchronize()
+        clk = clocks.stop()
+        ms = t0.elapsed_time(t1)
+        err = layer.last_error()
+        if err:
+            raise RuntimeError(f"device error in the timed region: {arl2.STATUS.get(err)}")
+
+        # dominant-kernel duration: the query launches of the last graph replay
+        if use_graphs:
+            attn_ev = graph_ev
+        attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
+        attn_avg_ms = float(np.mean(attn_ms))
+
+    # max over ranks
+    ms_max = ms
+    if dist is not None:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    frames_total = steps_done * world
+    value = frames_total / (ms_max / 1e3)
+    ms_per_step = ms_max / steps_done
+
+    result = {
+        "value": value, "ms_per_step": ms_per_step, "steps": steps_done, "clocks": clk,
+        "attn_avg_ms": attn_avg_ms, "flops": flops, "launches_per_step": cfg.queries + 1 + 3,
+    }
+    # end-to-end through the public API with host buffers
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, cfg, ds, layer, device, stream, dist, world)
+    layer.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(args, cfg, ds, layer, device, stream, dist, world):
+    """Same metric through the C-ABI calls with host buffers: every step copies its
+    five passes' Q, K, V and its gates from pinned host memory and reads the five
+    outputs back."""
+    import torch
+    from hybrid_linear_attention_arl2_b200 import arl2
+    B, H, L, d = cfg.batch, cfg.heads, cfg.tokens, cfg.head_dim
+    steps = max(4, min(args.steps // 4, 40))
+    host_pool = [tuple(t.cpu().pin_memory() for t in trip) for trip in ds.pool]
+    outs_host = [torch.empty((B, L, H, d), dtype=torch.bfloat16).pin_memory() for _ in range(cfg.passes)]
+    dq = [torch.empty((B, L, H, d), dtype=torch.bfloat16, device=device) for _ in range(3)]
+    O = [torch.empty((B, L, H, d), dtype=torch.bfloat16, device=device) for _ in range(cfg.passes)]
+    ga = torch.empty((B, H), dtype=torch.float32, device=device)
+    gb = torch.empty((B, H, L), dtype=torch.float32, device=device)
+    gates = {}
+    h2d = d2h = 0
+    with torch.cuda.stream(stream):
+        f0 = 1000
+        for f in range(f0, f0 + steps):
+            a, b = ds.gates(f)
+            gates[f] = (torch.from_numpy(a).pin_memory(), torch.from_numpy(b).pin_memory())
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for f in range(f0, f0 + steps):
+            for p in range(cfg.passes):
+                trip = host_pool[ds.wl.pool_index(0, f, p)]
+                for dst, src in zip(dq, trip):
+                    dst.copy_(src, non_blocking=True)
+                    h2d += src.numel() * 2
+                if p < cfg.queries:
+                    arl2.arl2_frame_query(layer.handle, dq[0], dq[1], dq[2], O[p], stream)
+                else:
+                    a, b = gates[f]
+                    ga.copy_(a, non_blocking=True)
+                    gb.copy_(b, non_blocking=True)
+                    h2d += a.numel() * 4 + b.numel() * 4
+                    arl2.arl2_frame_commit(layer.handle, dq[0], dq[1], dq[2], ga, gb, O[p], stream)
+                outs_host[p].copy_(O[p], non_blocking=True)
+                d2h += O[p].numel() * 2
+        e1.record(stream)
+        e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": steps * world / (ms / 1e3), "unit": "frames/s",
+            "h2d_bytes_per_step": h2d // steps, "d2h_bytes_per_step": d2h // steps}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def cpu_oracle_rate(cfg: W.Config, budget_s: float = 12.0, sample_note=True):
+    """The oracle as it stands, timed on this host's cores: frames/s of one
+    hybrid layer on a bounded sample (whole frames, 4 queries + 1 commit)."""
+    from oracle import arl2_oracle as o
+    wl = W.Workload(cfg)
+    phi = wl.phi(0)
+    S = np.zeros((cfg.batch, cfg.heads, cfg.head_dim, cfg.head_dim))
+    frames = 0
+    t0 = time.perf_counter()
+    while True:
+        for p in range(cfg.passes):
+            Q, K, V = wl.qkv(0, frames, p)
+            if p < cfg.queries:
+                o.frame_query(S, Q, K, V, phi)
+            else:
+                _, S = o.frame_commit(S, Q, K, V, phi, wl.alpha(0, frames), wl.beta(0, frames), cfg.c)
+        frames += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return {"value": frames / dt, "unit": "frames/s", "cores": cores, "kind": "oracle",
+            "sample": f"{frames} whole frames (4 query passes + 1 commit each) of one {cfg.name} layer, "
+                      f"numpy float64, {dt:.1f} s"}
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        return None
+
+
+def main():
+    args = _args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    cfg = W.CONFIGS[args.config]
+    if args.profile_small:
+        args.steps, args.warmup = 4, 3
+        args.no_e2e = args.no_cpu_baseline = True
+    metric = "frames/s per hybrid layer (1560-token frames, 4 query passes + 1 commit)"
+    config = {"workload": cfg.name, "batch": cfg.batch, "heads": cfg.heads, "head_dim": cfg.head_dim,
+              "tokens_per_frame": cfg.tokens, "passes_per_frame": cfg.passes,
+              "corr_scale": "1/L" if cfg.corr_scale < 0 else cfg.corr_scale,
+              "l2": f"inputs cycle through a {cfg.pool}-triple pool "
+                    f"({cfg.pool * 3 * cfg.tokens * cfg.heads * cfg.head_dim * 2 * cfg.batch / 1e6:.0f} MB > 126 MB L2)",
+              "parallelism": f"replicas x{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        budget = 3.0
+        steps = []
+        cb = None
+        for s in range(args.warmup + args.steps):
+            cb = cpu_oracle_rate(cfg, budget_s=budget / max(1, args.steps))
+            steps.append(cb["value"])
+        value = float(np.mean(steps[args.warmup:])) if args.steps else float(np.mean(steps))
+        line = {"impl": "reference", "metric": metric, "value": value, "unit": "frames/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cb["cores"], "kind": "oracle",
+                                 "sample": cb["sample"]},
+                "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    res = run_arl2(args, rank, world)
+    if rank != 0:
+        return
+    pk = peaks()
+    fl = res["flops"]
+    frame_tflops = fl["frame"] * res["value"] / max(1, world) / 1e12  # per GPU
+    attn_tflops = fl["attn_per_pass"] / (res["attn_avg_ms"] / 1e3) / 1e12
+    if pk:
+        peak_sus, peak_burst, src = pk["bf16_tflops_sustained"], pk["bf16_tflops"], "of measured"
+    else:
+        peak_sus, peak_burst, src = 1400.0, 1590.0, "of fallback"
+    line = {
+        "metric": metric, "value": res["value"], "unit": "frames/s", "n_gpus": world, "steps": res["steps"],
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+        "tokens_per_s": res["value"] * cfg.tokens * cfg.batch,
+        "pct_bf16_peak": {"value": 100.0 * frame_tflops / peak_sus, "basis": f"sustained bf16 {src}",
+                          "burst_basis": 100.0 * frame_tflops / peak_burst},
+        "roofline": {"bound": "tensor", "kernel": "attn_bf16_kernel", "achieved": attn_tflops, "peak": peak_sus,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak_sus, "traffic": None,
+                     "peak_basis": f"bf16_tflops_sustained {src}"},
+        "clocks": res["clocks"],
+        "gpu_launches": res["launches_per_step"] * res["steps"],
+    }
+    if "e2e" in res:
+        line["e2e"] = res["e2e"]
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_oracle_rate(cfg, budget_s=12.0)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

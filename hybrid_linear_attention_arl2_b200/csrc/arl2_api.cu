@@ -1,0 +1,646 @@
+// C ABI of libarl2.so (declared in include/arl2.h): handles, argument
+// validation, device allocations, TMA descriptors and kernel dispatch.
+// Every step of the hot path runs in this library's kernels; the host code
+// here only checks arguments, encodes descriptors and enqueues launches.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <set>
+
+#include "../../include/arl2.h"
+
+#include "params.h"
+
+using namespace arl2;
+
+namespace {
+
+constexpr uint64_t kStateMagic = 0x41524c3253544154ull;  // "ARL2STAT"
+constexpr uint64_t kKvMagic = 0x41524c324b564341ull;     // "ARL2KVCA"
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;
+
+std::mutex g_mu;
+std::set<const void*> g_live;  // live handles, to reject destroyed or foreign pointers
+
+// Allocation failure injection for the out-of-memory tests: ARL2_FAIL_ALLOC_AT=n
+// makes the n-th device allocation of the process (1-based) fail.
+std::atomic<long> g_alloc_count{0};
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  const long n = ++g_alloc_count;
+  const char* s = std::getenv("ARL2_FAIL_ALLOC_AT");
+  if (s && *s && std::atol(s) == n) {
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  return cudaMalloc(p, bytes);
+}
+
+bool log_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* s = std::getenv("ARL2_LOG");
+    v = (s && *s && *s != '0') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 map, 128-byte swizzle, box {64, rows, 1}; out-of-range elements read as 0.
+bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1,
+              uint64_t stride2, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1, stride2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Token-major activations [B, tokens, H, 128] as a map over (H*128, tokens, B).
+bool make_act_map(CUtensorMap* m, const void* base, int B, int64_t tokens, int H) {
+  const uint64_t row = uint64_t(H) * 128 * 2;
+  return make_map(m, base, uint64_t(H) * 128, uint64_t(tokens), uint64_t(B), row, row * uint64_t(tokens), 128);
+}
+
+// Stacked 128 x 128 bf16 matrices [slabs, 128, 128] as a map over (128, 128, slabs).
+bool make_mat_map(CUtensorMap* m, const void* base, int slabs) {
+  return make_map(m, base, 128, 128, uint64_t(slabs), 256, 256 * 128, 128);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+arl2_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return ARL2_OK;
+  if (e == cudaErrorMemoryAllocation) return ARL2_ERR_OUT_OF_MEMORY;
+  if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver) return ARL2_ERR_NO_DEVICE;
+  return ARL2_ERR_CUDA;
+}
+
+arl2_status check_config(const arl2_config* c) {
+  if (!c) return ARL2_ERR_INVALID_ARGUMENT;
+  if (c->batch < 1 || c->heads < 1 || c->head_dim < 1 || c->tokens_per_frame < 1) return ARL2_ERR_INVALID_ARGUMENT;
+  if (c->dtype != ARL2_F32 && c->dtype != ARL2_BF16) return ARL2_ERR_UNSUPPORTED;
+  if (c->flags & ~(ARL2_INTRA_ONLY | ARL2_INTER_ONLY)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (c->flags == (ARL2_INTRA_ONLY | ARL2_INTER_ONLY)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (!(std::isfinite(c->softmax_scale)) || c->softmax_scale < 0.f) return ARL2_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(c->corr_scale)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (c->dtype == ARL2_BF16) {
+    if (c->head_dim != 128) return ARL2_ERR_UNSUPPORTED;
+    if (c->tokens_per_frame > (1 << 24)) return ARL2_ERR_UNSUPPORTED;
+    if (int64_t(c->batch) * c->heads > 65535) return ARL2_ERR_UNSUPPORTED;
+  } else {
+    if (c->head_dim > 128 || c->tokens_per_frame > 4096) return ARL2_ERR_UNSUPPORTED;
+    if (int64_t(c->batch) * c->heads > 65535) return ARL2_ERR_UNSUPPORTED;
+  }
+  return ARL2_OK;
+}
+
+float softmax_scale(const arl2_config& c) {
+  return c.softmax_scale > 0.f ? c.softmax_scale : 1.f / std::sqrt(float(c.head_dim));
+}
+
+}  // namespace
+
+struct arl2_state {
+  uint64_t magic;
+  arl2_config cfg;
+  int device;
+  float scale;
+  float corr;
+  uint64_t wait_ns;
+  // f32: phi as given [H,d,d]; bf16: phi_q [H][i][k] as given, phi_k^T and phi_v^T [H][j][i]
+  void* phi[3];
+  float* S[2];
+  int cur;
+  __nv_bfloat16* S_bf;   // bf16 copy of S[cur] (bf16 path)
+  __nv_bfloat16* mqt;    // (phi_q S[cur])^T (bf16 path)
+  float* partial;        // per-chunk state-write partials (bf16 path)
+  int n_chunks;
+  uint32_t* err;
+  int64_t frame;
+  int64_t bytes;
+  cudaStream_t last_stream;
+  CUtensorMap tm_phiq, tm_phik_t, tm_phiv_t, tm_s_bf, tm_mqt;
+};
+
+struct arl2_kv {
+  uint64_t magic;
+  arl2_config cfg;
+  int device;
+  float scale;
+  uint64_t wait_ns;
+  int32_t max_frames;
+  int64_t frames;
+  void* kc;  // [B, max_frames*L, H, d]
+  void* vc;
+  uint32_t* err;
+  int64_t bytes;
+  cudaStream_t last_stream;
+};
+
+namespace {
+
+template <class T>
+bool live(const T* h, uint64_t magic) {
+  if (!h) return false;
+  std::lock_guard<std::mutex> g(g_mu);
+  return g_live.count(h) && h->magic == magic;
+}
+
+void free_state(arl2_state* h) {
+  for (void* p : {h->phi[0], h->phi[1], h->phi[2], (void*)h->S[0], (void*)h->S[1], (void*)h->S_bf, (void*)h->mqt,
+                  (void*)h->partial, (void*)h->err})
+    if (p) cudaFree(p);
+  h->magic = 0;
+  delete h;
+}
+
+void free_kv(arl2_kv* h) {
+  for (void* p : {h->kc, h->vc, (void*)h->err})
+    if (p) cudaFree(p);
+  h->magic = 0;
+  delete h;
+}
+
+#define ARL2_TRY(expr)                          \
+  do {                                          \
+    cudaError_t e_ = (expr);                    \
+    if (e_ != cudaSuccess) return from_cuda(e_); \
+  } while (0)
+
+arl2_status prepare_readout(arl2_state* h, cudaStream_t st) {
+  // MqT = (phi_q S[cur])^T from the bf16 copy of S[cur].
+  StateParams sp{};
+  sp.mqt = h->mqt;
+  sp.heads = h->cfg.heads;
+  sp.err = h->err;
+  sp.wait_limit_ns = h->wait_ns;
+  ARL2_TRY(launch_readout_prep(h->tm_s_bf, h->tm_phiq, sp, h->cfg.batch, st));
+  return ARL2_OK;
+}
+
+arl2_status run_attention(arl2_state* h, const void* q, const void* k, const void* v, void* o, cudaStream_t st) {
+  const arl2_config& c = h->cfg;
+  if (c.dtype == ARL2_F32) {
+    F32AttnParams p{};
+    p.q = static_cast<const float*>(q);
+    p.k = static_cast<const float*>(k);
+    p.v = static_cast<const float*>(v);
+    p.o = static_cast<float*>(o);
+    p.phi_q = static_cast<const float*>(h->phi[0]);
+    p.S = h->S[h->cur];
+    p.q_len = p.kv_len = p.kv_stride = c.tokens_per_frame;
+    p.heads = c.heads;
+    p.d = c.head_dim;
+    p.scale = h->scale;
+    p.flags = c.flags;
+    ARL2_TRY(launch_f32_attn(p, c.batch, st));
+    return ARL2_OK;
+  }
+  CUtensorMap tq, tk, tv;
+  if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads) ||
+      !make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads) ||
+      !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads))
+    return ARL2_ERR_CUDA;
+  AttnParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.q_len = p.kv_len = c.tokens_per_frame;
+  p.heads = c.heads;
+  p.scale_log2 = h->scale * 1.4426950408889634f;
+  p.flags = c.flags;
+  p.has_inter = 1;
+  p.err = h->err;
+  p.wait_limit_ns = h->wait_ns;
+  ARL2_TRY(launch_attn_bf16(tq, tk, tv, h->tm_mqt, p, c.batch, st));
+  return ARL2_OK;
+}
+
+bool overlaps(const void* a, const void* b, size_t n) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + n && y < x + n;
+}
+
+arl2_status check_io(const arl2_config& c, const void* q, const void* k, const void* v, const void* o) {
+  if (!q || !k || !v || !o) return ARL2_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ARL2_ERR_INVALID_ARGUMENT;
+  const size_t n = size_t(c.batch) * c.tokens_per_frame * c.heads * c.head_dim * (c.dtype == ARL2_F32 ? 4 : 2);
+  if (overlaps(o, q, n) || overlaps(o, k, n) || overlaps(o, v, n)) return ARL2_ERR_INVALID_ARGUMENT;
+  return ARL2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* arl2_status_string(arl2_status s) {
+  switch (s) {
+    case ARL2_OK: return "ok";
+    case ARL2_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case ARL2_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case ARL2_ERR_OUT_OF_MEMORY: return "out of device memory";
+    case ARL2_ERR_CUDA: return "CUDA error";
+    case ARL2_ERR_TIMEOUT: return "device-side wait timed out";
+    case ARL2_ERR_NO_DEVICE: return "no CUDA device";
+  }
+  return "unknown status";
+}
+
+int32_t arl2_abi_version(void) { return 1; }
+
+arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const void* phi_k, const void* phi_v,
+                            void* stream, arl2_state_t* out) {
+  if (!out) return ARL2_ERR_INVALID_ARGUMENT;
+  *out = nullptr;
+  arl2_status s = check_config(cfg);
+  if (s != ARL2_OK) return s;
+  if (!phi_q || !phi_k || !phi_v || !aligned16(phi_q) || !aligned16(phi_k) || !aligned16(phi_v))
+    return ARL2_ERR_INVALID_ARGUMENT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ARL2_ERR_NO_DEVICE;
+  if (cfg->dtype == ARL2_BF16 && !encode_fn()) return ARL2_ERR_NO_DEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  arl2_state* h = new (std::nothrow) arl2_state();
+  if (!h) return ARL2_ERR_OUT_OF_MEMORY;
+  h->cfg = *cfg;
+  h->device = dev;
+  h->scale = softmax_scale(*cfg);
+  h->corr = cfg->corr_scale < 0.f ? 1.f / float(cfg->tokens_per_frame) : cfg->corr_scale;
+  h->wait_ns = kDefaultWaitNs;
+  h->last_stream = st;
+  const int B = cfg->batch, H = cfg->heads, d = cfg->head_dim;
+  const size_t esz = cfg->dtype == ARL2_F32 ? 4 : 2;
+  const size_t phi_bytes = size_t(H) * d * d * esz;
+  const size_t s_bytes = size_t(B) * H * d * d * sizeof(float);
+  h->n_chunks = (cfg->tokens_per_frame + 127) / 128;
+  cudaError_t e = cudaSuccess;
+  auto alloc = [&](void** p, size_t n) {
+    if (e == cudaSuccess) {
+      e = dev_alloc(p, n);
+      if (e == cudaSuccess) h->bytes += int64_t(n);
+    }
+  };
+  for (int i = 0; i < 3; ++i) alloc(&h->phi[i], phi_bytes);
+  alloc(reinterpret_cast<void**>(&h->S[0]), s_bytes);
+  alloc(reinterpret_cast<void**>(&h->S[1]), s_bytes);
+  alloc(reinterpret_cast<void**>(&h->err), 256);
+  if (cfg->dtype == ARL2_BF16) {
+    alloc(reinterpret_cast<void**>(&h->S_bf), size_t(B) * H * d * d * 2);
+    alloc(reinterpret_cast<void**>(&h->mqt), size_t(B) * H * d * d * 2);
+    alloc(reinterpret_cast<void**>(&h->partial), size_t(B) * H * h->n_chunks * d * d * sizeof(float));
+  }
+  if (e != cudaSuccess) {
+    free_state(h);
+    return from_cuda(e);
+  }
+  const void* src[3] = {phi_q, phi_k, phi_v};
+  if (cfg->dtype == ARL2_F32) {
+    for (int i = 0; i < 3 && e == cudaSuccess; ++i)
+      e = cudaMemcpyAsync(h->phi[i], src[i], phi_bytes, cudaMemcpyDeviceToDevice, st);
+  } else {
+    e = cudaMemcpyAsync(h->phi[0], phi_q, phi_bytes, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = launch_transpose_bf16(static_cast<const __nv_bfloat16*>(phi_k), static_cast<__nv_bfloat16*>(h->phi[1]), H,
+                                st);
+    if (e == cudaSuccess)
+      e = launch_transpose_bf16(static_cast<const __nv_bfloat16*>(phi_v), static_cast<__nv_bfloat16*>(h->phi[2]), H,
+                                st);
+  }
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->S[0], 0, s_bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->S[1], 0, s_bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 256, st);
+  if (cfg->dtype == ARL2_BF16) {
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->S_bf, 0, size_t(B) * H * d * d * 2, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->mqt, 0, size_t(B) * H * d * d * 2, st);
+    if (e == cudaSuccess &&
+        !(make_mat_map(&h->tm_phiq, h->phi[0], H) && make_mat_map(&h->tm_phik_t, h->phi[1], H) &&
+          make_mat_map(&h->tm_phiv_t, h->phi[2], H) && make_mat_map(&h->tm_s_bf, h->S_bf, B * H) &&
+          make_mat_map(&h->tm_mqt, h->mqt, B * H)))
+      e = cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) {
+    free_state(h);
+    return from_cuda(e);
+  }
+  h->magic = kStateMagic;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    g_live.insert(h);
+  }
+  if (log_enabled())
+    std::fprintf(stderr, "[arl2] state_init B=%d H=%d d=%d L=%d dtype=%d bytes=%lld\n", B, H, d,
+                 cfg->tokens_per_frame, cfg->dtype, (long long)h->bytes);
+  *out = h;
+  return ARL2_OK;
+}
+
+arl2_status arl2_frame_query(arl2_state_t h, const void* q, const void* k, const void* v, void* o, void* stream) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  arl2_status s = check_io(h->cfg, q, k, v, o);
+  if (s != ARL2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  return run_attention(h, q, k, v, o, st);
+}
+
+arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, const void* v, const float* alpha,
+                              const float* beta, void* o, void* stream) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  arl2_status s = check_io(h->cfg, q, k, v, o);
+  if (s != ARL2_OK) return s;
+  if (!alpha || !beta || !aligned16(alpha) || !aligned16(beta)) return ARL2_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  s = run_attention(h, q, k, v, o, st);  // the output reads S_{N-1}
+  if (s != ARL2_OK) return s;
+  const arl2_config& c = h->cfg;
+  const int nxt = h->cur ^ 1;
+  if (c.dtype == ARL2_F32) {
+    F32CommitParams p{};
+    p.k = static_cast<const float*>(k);
+    p.v = static_cast<const float*>(v);
+    p.phi_k = static_cast<const float*>(h->phi[1]);
+    p.phi_v = static_cast<const float*>(h->phi[2]);
+    p.S_prev = h->S[h->cur];
+    p.S_next = h->S[nxt];
+    p.alpha = alpha;
+    p.beta = beta;
+    p.L = c.tokens_per_frame;
+    p.heads = c.heads;
+    p.d = c.head_dim;
+    p.corr = h->corr;
+    ARL2_TRY(launch_f32_commit(p, c.batch, st));
+  } else {
+    CUtensorMap tk, tv;
+    if (!make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads) ||
+        !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads))
+      return ARL2_ERR_CUDA;
+    StateParams sp{};
+    sp.S_prev = h->S[h->cur];
+    sp.alpha = alpha;
+    sp.beta = beta;
+    sp.partial = h->partial;
+    sp.S_next = h->S[nxt];
+    sp.S_next_bf = h->S_bf;
+    sp.mqt = h->mqt;
+    sp.L = c.tokens_per_frame;
+    sp.heads = c.heads;
+    sp.n_chunks = h->n_chunks;
+    sp.corr = h->corr;
+    sp.err = h->err;
+    sp.wait_limit_ns = h->wait_ns;
+    ARL2_TRY(launch_state_partial(tk, tv, h->tm_phik_t, h->tm_phiv_t, h->tm_s_bf, sp, c.batch, st));
+    ARL2_TRY(launch_state_finalize(sp, c.batch, st));
+    ARL2_TRY(launch_readout_prep(h->tm_s_bf, h->tm_phiq, sp, c.batch, st));
+  }
+  h->cur = nxt;
+  h->frame += 1;
+  return ARL2_OK;
+}
+
+arl2_status arl2_state_get(arl2_state_t h, float* dst, int64_t* frame, void* stream) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (frame) *frame = h->frame;
+  if (!dst) return frame ? ARL2_OK : ARL2_ERR_INVALID_ARGUMENT;
+  const arl2_config& c = h->cfg;
+  const size_t n = size_t(c.batch) * c.heads * c.head_dim * c.head_dim * sizeof(float);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  ARL2_TRY(cudaMemcpyAsync(dst, h->S[h->cur], n, cudaMemcpyDeviceToDevice, st));
+  return ARL2_OK;
+}
+
+arl2_status arl2_state_set(arl2_state_t h, const float* src, int64_t frame, void* stream) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (!src || frame < 0 || !aligned16(src)) return ARL2_ERR_INVALID_ARGUMENT;
+  const arl2_config& c = h->cfg;
+  const size_t cnt = size_t(c.batch) * c.heads * c.head_dim * c.head_dim;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  ARL2_TRY(cudaMemcpyAsync(h->S[h->cur], src, cnt * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  if (c.dtype == ARL2_BF16) {
+    ARL2_TRY(launch_to_bf16(h->S[h->cur], h->S_bf, cnt, st));
+    arl2_status s = prepare_readout(h, st);
+    if (s != ARL2_OK) return s;
+  }
+  h->frame = frame;
+  return ARL2_OK;
+}
+
+arl2_status arl2_last_error(arl2_state_t h) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  ARL2_TRY(cudaStreamSynchronize(h->last_stream));
+  uint32_t w = 0;
+  ARL2_TRY(cudaMemcpy(&w, h->err, sizeof(w), cudaMemcpyDeviceToHost));
+  if (w) ARL2_TRY(cudaMemset(h->err, 0, sizeof(w)));
+  return static_cast<arl2_status>(w);
+}
+
+int64_t arl2_state_device_bytes(arl2_state_t h) { return live(h, kStateMagic) ? h->bytes : -1; }
+
+arl2_status arl2_state_set_wait_limit(arl2_state_t h, uint64_t limit_ns) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  h->wait_ns = limit_ns ? limit_ns : kDefaultWaitNs;
+  return ARL2_OK;
+}
+
+arl2_status arl2_state_destroy(arl2_state_t h) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    g_live.erase(h);
+  }
+  cudaStreamSynchronize(h->last_stream);
+  free_state(h);
+  return ARL2_OK;
+}
+
+// ---------------------------------------------------------------- KV-cache layers
+arl2_status arl2_kv_init(const arl2_config* cfg, int32_t max_frames, void* stream, arl2_kv_t* out) {
+  if (!out) return ARL2_ERR_INVALID_ARGUMENT;
+  *out = nullptr;
+  arl2_status s = check_config(cfg);
+  if (s != ARL2_OK) return s;
+  if (max_frames < 1) return ARL2_ERR_INVALID_ARGUMENT;
+  const int64_t tokens = int64_t(max_frames) * cfg->tokens_per_frame;
+  if (cfg->dtype == ARL2_BF16 && tokens > (int64_t(1) << 31)) return ARL2_ERR_UNSUPPORTED;
+  if (cfg->dtype == ARL2_F32 && tokens > (int64_t(1) << 31)) return ARL2_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ARL2_ERR_NO_DEVICE;
+  if (cfg->dtype == ARL2_BF16 && !encode_fn()) return ARL2_ERR_NO_DEVICE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  arl2_kv* h = new (std::nothrow) arl2_kv();
+  if (!h) return ARL2_ERR_OUT_OF_MEMORY;
+  h->cfg = *cfg;
+  h->device = dev;
+  h->scale = softmax_scale(*cfg);
+  h->wait_ns = kDefaultWaitNs;
+  h->max_frames = max_frames;
+  h->last_stream = st;
+  const size_t esz = cfg->dtype == ARL2_F32 ? 4 : 2;
+  const size_t bytes = size_t(cfg->batch) * size_t(tokens) * cfg->heads * cfg->head_dim * esz;
+  cudaError_t e = dev_alloc(&h->kc, bytes);
+  if (e == cudaSuccess) e = dev_alloc(&h->vc, bytes);
+  if (e == cudaSuccess) e = dev_alloc(reinterpret_cast<void**>(&h->err), 256);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->kc, 0, bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->vc, 0, bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 256, st);
+  if (e != cudaSuccess) {
+    free_kv(h);
+    return from_cuda(e);
+  }
+  h->bytes = int64_t(2 * bytes + 256);
+  h->magic = kKvMagic;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    g_live.insert(h);
+  }
+  *out = h;
+  return ARL2_OK;
+}
+
+namespace {
+
+// Copy this pass's K and V into cache slot `frames` (the slot after the
+// committed frames), then attend over frames 0..frames of the cache.
+arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, void* o, cudaStream_t st) {
+  const arl2_config& c = h->cfg;
+  if (h->frames >= h->max_frames) return ARL2_ERR_INVALID_ARGUMENT;
+  const size_t esz = c.dtype == ARL2_F32 ? 4 : 2;
+  const size_t frame_bytes = size_t(c.tokens_per_frame) * c.heads * c.head_dim * esz;
+  const size_t stream_bytes = frame_bytes * size_t(h->max_frames);
+  char* kc = static_cast<char*>(h->kc);
+  char* vc = static_cast<char*>(h->vc);
+  ARL2_TRY(cudaMemcpy2DAsync(kc + frame_bytes * h->frames, stream_bytes, k, frame_bytes, frame_bytes, c.batch,
+                             cudaMemcpyDeviceToDevice, st));
+  ARL2_TRY(cudaMemcpy2DAsync(vc + frame_bytes * h->frames, stream_bytes, v, frame_bytes, frame_bytes, c.batch,
+                             cudaMemcpyDeviceToDevice, st));
+  const int64_t kv_tokens = int64_t(h->frames + 1) * c.tokens_per_frame;
+  const int64_t stride_tokens = int64_t(h->max_frames) * c.tokens_per_frame;
+  if (c.dtype == ARL2_F32) {
+    F32AttnParams p{};
+    p.q = static_cast<const float*>(q);
+    p.k = static_cast<const float*>(h->kc);
+    p.v = static_cast<const float*>(h->vc);
+    p.o = static_cast<float*>(o);
+    p.phi_q = nullptr;
+    p.S = nullptr;
+    p.q_len = c.tokens_per_frame;
+    p.kv_len = int(kv_tokens);
+    p.kv_stride = int(stride_tokens);
+    p.heads = c.heads;
+    p.d = c.head_dim;
+    p.scale = h->scale;
+    p.flags = 0;
+    ARL2_TRY(launch_f32_attn(p, c.batch, st));
+    return ARL2_OK;
+  }
+  CUtensorMap tq, tk, tv;
+  if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads) ||
+      !make_act_map(&tk, h->kc, c.batch, stride_tokens, c.heads) ||
+      !make_act_map(&tv, h->vc, c.batch, stride_tokens, c.heads))
+    return ARL2_ERR_CUDA;
+  AttnParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.q_len = c.tokens_per_frame;
+  p.kv_len = int(kv_tokens);
+  p.heads = c.heads;
+  p.scale_log2 = h->scale * 1.4426950408889634f;
+  p.flags = 0;
+  p.has_inter = 0;
+  p.err = h->err;
+  p.wait_limit_ns = h->wait_ns;
+  ARL2_TRY(launch_attn_bf16(tq, tk, tv, tq, p, c.batch, st));
+  return ARL2_OK;
+}
+
+}  // namespace
+
+arl2_status arl2_kv_query(arl2_kv_t h, const void* q, const void* k, const void* v, void* o, void* stream) {
+  if (!live(h, kKvMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  arl2_status s = check_io(h->cfg, q, k, v, o);
+  if (s != ARL2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  return kv_pass(h, q, k, v, o, st);
+}
+
+arl2_status arl2_kv_commit(arl2_kv_t h, const void* q, const void* k, const void* v, void* o, void* stream) {
+  if (!live(h, kKvMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  arl2_status s = check_io(h->cfg, q, k, v, o);
+  if (s != ARL2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  s = kv_pass(h, q, k, v, o, st);
+  if (s == ARL2_OK) h->frames += 1;
+  return s;
+}
+
+int64_t arl2_kv_frames(arl2_kv_t h) { return live(h, kKvMagic) ? h->frames : -1; }
+int64_t arl2_kv_device_bytes(arl2_kv_t h) { return live(h, kKvMagic) ? h->bytes : -1; }
+
+arl2_status arl2_kv_last_error(arl2_kv_t h) {
+  if (!live(h, kKvMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  ARL2_TRY(cudaStreamSynchronize(h->last_stream));
+  uint32_t w = 0;
+  ARL2_TRY(cudaMemcpy(&w, h->err, sizeof(w), cudaMemcpyDeviceToHost));
+  if (w) ARL2_TRY(cudaMemset(h->err, 0, sizeof(w)));
+  return static_cast<arl2_status>(w);
+}
+
+arl2_status arl2_kv_destroy(arl2_kv_t h) {
+  if (!live(h, kKvMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    g_live.erase(h);
+  }
+  cudaStreamSynchronize(h->last_stream);
+  free_kv(h);
+  return ARL2_OK;
+}
+
+arl2_status arl2_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return ARL2_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* err = nullptr;
+  ARL2_TRY(dev_alloc(reinterpret_cast<void**>(&err), sizeof(uint32_t)));
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), st);
+  if (e == cudaSuccess) e = launch_wait_selftest(err, limit_ns, st);
+  uint32_t w = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&w, err, sizeof(uint32_t), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  cudaFree(err);
+  if (e != cudaSuccess) return from_cuda(e);
+  return static_cast<arl2_status>(w);
+}
+
+}  // extern "C"

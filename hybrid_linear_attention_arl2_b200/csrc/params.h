@@ -1,0 +1,85 @@
+// Launch parameters and launcher declarations shared by the library's
+// translation units (kernels and the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace arl2 {
+
+// Fused intra-frame softmax + inter-frame read-out (attn_bf16.cu).
+struct AttnParams {
+  __nv_bfloat16* o;     // [B, q_len, H, 128]
+  int q_len;            // query tokens per stream
+  int kv_len;           // valid key/value tokens per stream
+  int heads;
+  float scale_log2;     // softmax scale * log2(e)
+  uint32_t flags;       // 1: intra only, 2: inter only
+  int has_inter;        // 1: add Q MqT^T
+  uint32_t* err;        // device error word
+  uint64_t wait_limit_ns;
+};
+
+// State write and read-out preparation (state_bf16.cu).
+struct StateParams {
+  const float* S_prev;      // [B, H, 128, 128]
+  const float* alpha;       // [B, H]
+  const float* beta;        // [B, H, L]
+  float* partial;           // [B, H, n_chunks, 128, 128]
+  float* S_next;            // [B, H, 128, 128]
+  __nv_bfloat16* S_next_bf; // [B, H, 128, 128]
+  __nv_bfloat16* mqt;       // [B, H, 128, 128]
+  int L;
+  int heads;
+  int n_chunks;
+  float corr;
+  uint32_t* err;
+  uint64_t wait_limit_ns;
+};
+
+// float32 path (f32_path.cu).
+struct F32AttnParams {
+  const float* q;      // [B, q_len, H, d]
+  const float* k;      // [B, kv_stride, H, d]
+  const float* v;
+  float* o;            // [B, q_len, H, d]
+  const float* phi_q;  // [H, d, d] (null: no read-out)
+  const float* S;      // [B, H, d, d]
+  int q_len, kv_len, kv_stride, heads, d;
+  float scale;
+  uint32_t flags;
+};
+
+struct F32CommitParams {
+  const float* k;      // [B, L, H, d]
+  const float* v;
+  const float* phi_k;  // [H, d, d]
+  const float* phi_v;
+  const float* S_prev; // [B, H, d, d]
+  float* S_next;
+  const float* alpha;  // [B, H]
+  const float* beta;   // [B, H, L]
+  int L, heads, d;
+  float corr;
+};
+
+cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tmq, const AttnParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_state_partial(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tpk,
+                                 const CUtensorMap& tpv, const CUtensorMap& ts, const StateParams& p, int batch,
+                                 cudaStream_t stream);
+cudaError_t launch_state_finalize(const StateParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_readout_prep(const CUtensorMap& ts, const CUtensorMap& tphiq, const StateParams& p, int batch,
+                                cudaStream_t stream);
+cudaError_t launch_f32_attn(const F32AttnParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_f32_commit(const F32CommitParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_transpose_bf16(const __nv_bfloat16* src, __nv_bfloat16* dst, int slabs, cudaStream_t stream);
+cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t stream);
+cudaError_t launch_wait_selftest(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
+
+// Sets the dynamic shared-memory limit of `func` once per device.
+cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* done_mask);
+
+}  // namespace arl2

@@ -1,0 +1,158 @@
+/*
+ * arl2.h -- C ABI of libarl2.so: the per-frame hot path of the ARL2 hybrid
+ * attention module on NVIDIA B200 (sm_100a).
+ *
+ * Sources.  "ARL2 summary" is the technical summary on the page "Attend
+ * Locally, Remember Linearly: Linear Attention as Cross-Frame Memory for
+ * Autoregressive Video Diffusion" (gist.science; German, Italian, Japanese and
+ * Korean editions carry the same text).  "ARL2 abstract" is the authors'
+ * English abstract of arXiv 2605.16579v2 (fugumt.com paper_check page).
+ *
+ * What one hybrid layer computes, per stream b and head h, for frame N:
+ *   intra-frame branch   O_intra = softmax(Q K^T * scale) V over the frame's
+ *                        L tokens, bidirectional, no mask
+ *                        (ARL2 summary, section 2.1, intra-frame branch);
+ *   feature maps         Q' = Q phi_q, K' = rownorm2(K phi_k), V' = V phi_v
+ *                        (section 2.1, adaptation by per-head grouped 1x1 maps);
+ *   inter-frame read-out O_inter = Q' S_{N-1}   (section 2.1, output);
+ *   output               O = O_intra + O_inter;
+ *   state write          S_N = alpha S_{N-1} + c K'^T diag(beta)(V' - K' S_{N-1})
+ *                        (section 2.1, state update), once per frame on the clean
+ *                        pass only, every token reading the same S_{N-1}
+ *                        (section 2.2, frame-level access and clean-pass updates;
+ *                        ARL2 abstract).
+ *
+ * Conventions shared by every call:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned, contiguous, in the handle's dtype (float32 or bf16).
+ *       Q, K, V, O : [B, L, H, d] token-major (row = token, then head, then
+ *                    channel); O must not overlap Q, K or V.
+ *       phi_*      : [H, d, d] row-major, Q' = Q phi (q'_j = sum_i q_i phi[i][j]).
+ *       alpha      : float32 [B, H]      (one decay gate per stream and head).
+ *       beta       : float32 [B, H, L]   (one write strength per token).
+ *       state      : float32 [B, H, d, d], S[b][h][i][j] with i over K' and
+ *                    j over V' channels.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream; their return value covers argument
+ *     and launch errors only.  Errors raised inside kernels (a bounded wait that
+ *     ran out) are recorded in the handle and returned by arl2_last_error().
+ *   - A handle must not be used from two streams at once; calls on one handle
+ *     execute in stream order.
+ *   - No C++ exception crosses this interface.
+ *   - Supported shapes: bf16 needs head_dim = 128; float32 needs head_dim <= 128
+ *     and tokens_per_frame <= 4096.  Anything else returns ARL2_ERR_UNSUPPORTED.
+ */
+#ifndef ARL2_H
+#define ARL2_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ARL2_OK = 0,
+  ARL2_ERR_INVALID_ARGUMENT = 1, /* null or misaligned pointer, bad handle, bad size */
+  ARL2_ERR_UNSUPPORTED = 2,      /* a shape or dtype outside the supported set */
+  ARL2_ERR_OUT_OF_MEMORY = 3,    /* a device allocation of the library failed */
+  ARL2_ERR_CUDA = 4,             /* a CUDA runtime call or kernel launch failed */
+  ARL2_ERR_TIMEOUT = 5,          /* a bounded device-side wait ran out */
+  ARL2_ERR_NO_DEVICE = 6         /* no usable CUDA device / driver */
+} arl2_status;
+
+typedef enum { ARL2_F32 = 0, ARL2_BF16 = 1 } arl2_dtype;
+
+/* Test-only flags of arl2_config.flags: return only one branch of O. */
+#define ARL2_INTRA_ONLY 1u
+#define ARL2_INTER_ONLY 2u
+
+typedef struct {
+  int32_t batch;            /* B independent streams, >= 1 */
+  int32_t heads;            /* H, >= 1 */
+  int32_t head_dim;         /* d */
+  int32_t tokens_per_frame; /* L, >= 1 */
+  int32_t dtype;            /* arl2_dtype of Q, K, V, O and phi */
+  float softmax_scale;      /* 0 => 1/sqrt(head_dim) */
+  float corr_scale;         /* c of the state write; < 0 => 1/L (mean over the frame's tokens) */
+  uint32_t flags;           /* 0, or ARL2_INTRA_ONLY / ARL2_INTER_ONLY (tests only) */
+} arl2_config;
+
+typedef struct arl2_state* arl2_state_t;
+typedef struct arl2_kv* arl2_kv_t;
+
+/* Create a hybrid-layer handle with S_0 = 0 and frame counter 0.
+ * phi_q, phi_k, phi_v: device [H, d, d] in cfg->dtype; the library copies them
+ * (the caller may free them after the call returns).  The handle owns its
+ * state double buffer and work space on the current device.
+ * Errors: INVALID_ARGUMENT (null pointers, bad sizes), UNSUPPORTED (shape),
+ * OUT_OF_MEMORY (no partial handle is left behind), CUDA. */
+arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const void* phi_k,
+                            const void* phi_v, void* stream, arl2_state_t* out);
+
+/* One denoising step of a frame (ARL2 summary, section 2.2, clean-pass updates:
+ * denoising steps query the state and never write it):
+ *   O = softmax(Q K^T * scale) V + (Q phi_q) S_{N-1}.
+ * Reads the state, writes only O. */
+arl2_status arl2_frame_query(arl2_state_t h, const void* q, const void* k, const void* v, void* o,
+                             void* stream);
+
+/* The clean pass of frame N: O as in arl2_frame_query from S_{N-1}, then the
+ * frame's single state write
+ *   S_N = alpha S_{N-1} + c K'^T diag(beta) (V' - K' S_{N-1}),
+ * then the frame counter increments (ARL2 summary, sections 2.1 and 2.2). */
+arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, const void* v,
+                              const float* alpha, const float* beta, void* o, void* stream);
+
+/* Copy the current state (float32 [B, H, d, d]) to device memory `dst` and the
+ * frame counter to *frame (host pointer, may be null).  Synchronous with
+ * respect to `stream` for *frame only; the copy is enqueued on `stream`. */
+arl2_status arl2_state_get(arl2_state_t h, float* dst, int64_t* frame, void* stream);
+
+/* Replace the current state with device memory `src` (float32 [B, H, d, d]) and
+ * set the frame counter: checkpoint / resume of a stream. */
+arl2_status arl2_state_set(arl2_state_t h, const float* src, int64_t frame, void* stream);
+
+/* Synchronise the handle's last stream and return (and clear) the first error
+ * recorded by its kernels, ARL2_OK if none. */
+arl2_status arl2_last_error(arl2_state_t h);
+
+/* Device bytes held by the handle (constant over the stream's life). */
+int64_t arl2_state_device_bytes(arl2_state_t h);
+
+/* Wall-clock limit of one device-side wait in the handle's kernels (default
+ * 1 second).  0 restores the default. */
+arl2_status arl2_state_set_wait_limit(arl2_state_t h, uint64_t limit_ns);
+
+arl2_status arl2_state_destroy(arl2_state_t h);
+
+/* ---- Softmax layers kept from the teacher, with a growing KV cache --------
+ * (ARL2 summary, section 1: the KV cache grows with every generated block.)
+ * The queries of frame n attend, with no mask, to the clean keys and values
+ * of frames 0..n-1 followed by the current pass's own K and V.  A query pass
+ * leaves the cache's committed frames unchanged; a commit appends its K and V
+ * as frame n.  The cache is [B, max_frames * L, H, d] in cfg->dtype. */
+arl2_status arl2_kv_init(const arl2_config* cfg, int32_t max_frames, void* stream, arl2_kv_t* out);
+arl2_status arl2_kv_query(arl2_kv_t kv, const void* q, const void* k, const void* v, void* o,
+                          void* stream);
+arl2_status arl2_kv_commit(arl2_kv_t kv, const void* q, const void* k, const void* v, void* o,
+                           void* stream);
+int64_t arl2_kv_frames(arl2_kv_t kv);
+int64_t arl2_kv_device_bytes(arl2_kv_t kv);
+arl2_status arl2_kv_last_error(arl2_kv_t kv);
+arl2_status arl2_kv_destroy(arl2_kv_t kv);
+
+/* ---- Diagnostics -----------------------------------------------------------
+ * Run one kernel whose bounded wait is on a barrier that nothing completes,
+ * with the given limit; returns ARL2_ERR_TIMEOUT when the limit worked (the
+ * kernel returned and reported it) -- used by the failure-detection tests. */
+arl2_status arl2_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+const char* arl2_status_string(arl2_status s);
+int32_t arl2_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARL2_H */

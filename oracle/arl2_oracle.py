@@ -38,7 +38,7 @@ import numpy as np
 
 __all__ = [
     "feature_maps", "intra_softmax", "inter_readout", "frame_query",
-    "frame_commit", "kv_attention", "stream_reference",
+    "frame_commit", "state_update", "kv_attention", "stream_reference",
 ]
 
 EPS_NORM = 1e-12
@@ -111,11 +111,18 @@ def frame_commit(S, Q, K, V, phi, alpha, beta, corr_scale=1.0, scale=None):
     Returns (O [B, L, H, d], S_N [B, H, d, d])."""
     S = _f64(S)
     O = frame_query(S, Q, K, V, phi, scale)
-    _, Kp, Vp = feature_maps(Q, K, V, *phi)
+    return O, state_update(S, K, V, phi, alpha, beta, corr_scale)
+
+
+def state_update(S, K, V, phi, alpha, beta, corr_scale=1.0):
+    """The state write of a commit alone (ARL2 summary, §2.1
+    "Zustandsaktualisierung"): S_N = alpha S + c K'^T diag(beta)(V' - K' S),
+    every token of the frame reading the same S = S_{N-1} (§2.2)."""
+    S = _f64(S)
+    _, Kp, Vp = feature_maps(K, K, V, *phi)
     R = _f64(beta)[..., None] * (Vp - Kp @ S)
     delta = np.swapaxes(Kp, -1, -2) @ R
-    S_new = _f64(alpha)[..., None, None] * S + float(corr_scale) * delta
-    return O, S_new
+    return _f64(alpha)[..., None, None] * S + float(corr_scale) * delta
 
 
 def kv_attention(Q, K_ctx, V_ctx, scale=None):

@@ -1,0 +1,71 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/arl2.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+
+import pytest
+
+from hybrid_linear_attention_arl2_b200 import arl2, build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return arl2.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = arl2.declared_symbols()
+    assert len(names) >= 19
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(names) == set(arl2._SIGS), "binding and header disagree"
+
+
+def test_status_strings_and_version(lib):
+    assert arl2.arl2_abi_version() == 1
+    for s, name in arl2.STATUS.items():
+        assert arl2.arl2_status_string(s)
+    assert arl2.arl2_status_string(99) == "unknown status"
+
+
+def _init(cfg, phis=(16, 16, 16)):
+    h = ctypes.c_void_p()
+    return arl2.load_library().arl2_state_init(ctypes.byref(cfg) if cfg is not None else None,
+                                               *phis, None, ctypes.byref(h))
+
+
+def test_host_validation_of_config(lib):
+    ok = arl2.make_config(1, 2, 128, 64, arl2.ARL2_BF16)
+    assert _init(None) == 1
+    assert arl2.load_library().arl2_state_init(ctypes.byref(ok), 16, 16, 16, None, None) == 1  # null out
+    assert _init(arl2.make_config(0, 2, 128, 64, arl2.ARL2_BF16)) == 1
+    assert _init(arl2.make_config(1, 2, 128, 0, arl2.ARL2_BF16)) == 1
+    assert _init(arl2.make_config(1, 2, 64, 64, arl2.ARL2_BF16)) == 2       # bf16 needs d = 128
+    assert _init(arl2.make_config(1, 2, 256, 64, arl2.ARL2_F32)) == 2       # f32 d <= 128
+    assert _init(arl2.make_config(1, 2, 32, 5000, arl2.ARL2_F32)) == 2      # f32 L <= 4096
+    assert _init(arl2.make_config(1, 2, 128, 64, 7)) == 2                   # unknown dtype
+    assert _init(arl2.make_config(1, 2, 128, 64, arl2.ARL2_BF16, flags=3)) == 1
+    assert _init(arl2.make_config(1, 2, 128, 64, arl2.ARL2_BF16, softmax_scale=-1.0)) == 1
+    assert _init(ok, phis=(None, 16, 16)) == 1                              # null phi
+    assert _init(ok, phis=(17, 16, 16)) == 1                                # misaligned phi
+
+
+def test_foreign_handles_rejected(lib):
+    L = arl2.load_library()
+    bogus = ctypes.c_void_p(0x1000)
+    assert L.arl2_frame_query(bogus, 16, 16, 16, 16, None) == 1
+    assert L.arl2_frame_commit(None, 16, 16, 16, 16, 16, 16, None) == 1
+    assert L.arl2_state_destroy(bogus) == 1
+    assert L.arl2_state_device_bytes(bogus) == -1
+    assert L.arl2_kv_query(bogus, 16, 16, 16, 16, None) == 1
+    assert L.arl2_kv_frames(bogus) == -1
+    assert L.arl2_selftest_wait_timeout(0, None) == 1
+
+
+def test_kv_validation(lib):
+    L = arl2.load_library()
+    h = ctypes.c_void_p()
+    cfg = arl2.make_config(1, 2, 128, 64, arl2.ARL2_BF16)
+    assert L.arl2_kv_init(ctypes.byref(cfg), 0, None, ctypes.byref(h)) == 1
+    assert L.arl2_kv_init(None, 4, None, ctypes.byref(h)) == 1
