@@ -145,6 +145,9 @@ struct arl2_state {
   __nv_bfloat16* mqt;    // (phi_q S[cur])^T (bf16 path)
   float* partial;        // per-chunk state-write partials (bf16 path)
   int n_chunks;
+  float* attn_scratch;   // partial rows of split query blocks (bf16 path)
+  unsigned* attn_ready;  // their ready flags, zero between launches
+  int sms;
   uint32_t* err;
   int64_t frame;
   int64_t bytes;
@@ -162,6 +165,9 @@ struct arl2_kv {
   int64_t frames;
   void* kc;  // [B, max_frames*L, H, d]
   void* vc;
+  float* attn_scratch;
+  unsigned* attn_ready;
+  int sms;
   uint32_t* err;
   int64_t bytes;
   cudaStream_t last_stream;
@@ -178,14 +184,14 @@ bool live(const T* h, uint64_t magic) {
 
 void free_state(arl2_state* h) {
   for (void* p : {h->phi[0], h->phi[1], h->phi[2], (void*)h->S[0], (void*)h->S[1], (void*)h->S_bf, (void*)h->mqt,
-                  (void*)h->partial, (void*)h->err})
+                  (void*)h->partial, (void*)h->attn_scratch, (void*)h->attn_ready, (void*)h->err})
     if (p) cudaFree(p);
   h->magic = 0;
   delete h;
 }
 
 void free_kv(arl2_kv* h) {
-  for (void* p : {h->kc, h->vc, (void*)h->err})
+  for (void* p : {h->kc, h->vc, (void*)h->attn_scratch, (void*)h->attn_ready, (void*)h->err})
     if (p) cudaFree(p);
   h->magic = 0;
   delete h;
@@ -238,9 +244,12 @@ arl2_status run_attention(arl2_state* h, const void* q, const void* k, const voi
   p.scale_log2 = h->scale * 1.4426950408889634f;
   p.flags = c.flags;
   p.has_inter = 1;
+  p.scratch = h->attn_scratch;
+  p.ready = h->attn_ready;
   p.err = h->err;
   p.wait_limit_ns = h->wait_ns;
-  ARL2_TRY(launch_attn_bf16(tq, tk, tv, h->tm_mqt, p, c.batch, st));
+  if (!attn_partition(p, c.batch, h->sms)) return ARL2_ERR_UNSUPPORTED;
+  ARL2_TRY(launch_attn_bf16(tq, tk, tv, h->tm_mqt, p, st));
   return ARL2_OK;
 }
 
@@ -314,6 +323,9 @@ arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const voi
   alloc(reinterpret_cast<void**>(&h->S[1]), s_bytes);
   alloc(reinterpret_cast<void**>(&h->err), 256);
   if (cfg->dtype == ARL2_BF16) {
+    if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || h->sms < 1) h->sms = 1;
+    alloc(reinterpret_cast<void**>(&h->attn_scratch), size_t(h->sms) * 2 * kAttnSlotFloats * sizeof(float));
+    alloc(reinterpret_cast<void**>(&h->attn_ready), size_t(h->sms) * 2 * sizeof(unsigned));
     alloc(reinterpret_cast<void**>(&h->S_bf), size_t(B) * H * d * d * 2);
     alloc(reinterpret_cast<void**>(&h->mqt), size_t(B) * H * d * d * 2);
     alloc(reinterpret_cast<void**>(&h->partial), size_t(B) * H * h->n_chunks * d * d * sizeof(float));
@@ -341,6 +353,7 @@ arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const voi
   if (cfg->dtype == ARL2_BF16) {
     if (e == cudaSuccess) e = cudaMemsetAsync(h->S_bf, 0, size_t(B) * H * d * d * 2, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(h->mqt, 0, size_t(B) * H * d * d * 2, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->attn_ready, 0, size_t(h->sms) * 2 * sizeof(unsigned), st);
     if (e == cudaSuccess &&
         !(make_mat_map(&h->tm_phiq, h->phi[0], H) && make_mat_map(&h->tm_phik_t, h->phi[1], H) &&
           make_mat_map(&h->tm_phiv_t, h->phi[2], H) && make_mat_map(&h->tm_s_bf, h->S_bf, B * H) &&
@@ -461,7 +474,11 @@ arl2_status arl2_last_error(arl2_state_t h) {
   ARL2_TRY(cudaStreamSynchronize(h->last_stream));
   uint32_t w = 0;
   ARL2_TRY(cudaMemcpy(&w, h->err, sizeof(w), cudaMemcpyDeviceToHost));
-  if (w) ARL2_TRY(cudaMemset(h->err, 0, sizeof(w)));
+  if (w) {
+    // a kernel that gave up may have left partial-ready flags raised
+    ARL2_TRY(cudaMemset(h->err, 0, sizeof(w)));
+    if (h->attn_ready) ARL2_TRY(cudaMemset(h->attn_ready, 0, size_t(h->sms) * 2 * sizeof(unsigned)));
+  }
   return static_cast<arl2_status>(w);
 }
 
@@ -508,8 +525,14 @@ arl2_status arl2_kv_init(const arl2_config* cfg, int32_t max_frames, void* strea
   h->last_stream = st;
   const size_t esz = cfg->dtype == ARL2_F32 ? 4 : 2;
   const size_t bytes = size_t(cfg->batch) * size_t(tokens) * cfg->heads * cfg->head_dim * esz;
+  if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || h->sms < 1) h->sms = 1;
+  const size_t scratch_bytes = size_t(h->sms) * 2 * kAttnSlotFloats * sizeof(float);
+  const size_t ready_bytes = size_t(h->sms) * 2 * sizeof(unsigned);
   cudaError_t e = dev_alloc(&h->kc, bytes);
   if (e == cudaSuccess) e = dev_alloc(&h->vc, bytes);
+  if (e == cudaSuccess && cfg->dtype == ARL2_BF16) e = dev_alloc(reinterpret_cast<void**>(&h->attn_scratch), scratch_bytes);
+  if (e == cudaSuccess && cfg->dtype == ARL2_BF16) e = dev_alloc(reinterpret_cast<void**>(&h->attn_ready), ready_bytes);
+  if (e == cudaSuccess && cfg->dtype == ARL2_BF16) e = cudaMemsetAsync(h->attn_ready, 0, ready_bytes, st);
   if (e == cudaSuccess) e = dev_alloc(reinterpret_cast<void**>(&h->err), 256);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->kc, 0, bytes, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->vc, 0, bytes, st);
@@ -518,7 +541,7 @@ arl2_status arl2_kv_init(const arl2_config* cfg, int32_t max_frames, void* strea
     free_kv(h);
     return from_cuda(e);
   }
-  h->bytes = int64_t(2 * bytes + 256);
+  h->bytes = int64_t(2 * bytes + 256) + (cfg->dtype == ARL2_BF16 ? int64_t(scratch_bytes + ready_bytes) : 0);
   h->magic = kKvMagic;
   {
     std::lock_guard<std::mutex> g(g_mu);
@@ -577,9 +600,12 @@ arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, voi
   p.scale_log2 = h->scale * 1.4426950408889634f;
   p.flags = 0;
   p.has_inter = 0;
+  p.scratch = h->attn_scratch;
+  p.ready = h->attn_ready;
   p.err = h->err;
   p.wait_limit_ns = h->wait_ns;
-  ARL2_TRY(launch_attn_bf16(tq, tk, tv, tq, p, c.batch, st));
+  if (!attn_partition(p, c.batch, h->sms)) return ARL2_ERR_UNSUPPORTED;
+  ARL2_TRY(launch_attn_bf16(tq, tk, tv, tq, p, st));
   return ARL2_OK;
 }
 
@@ -613,7 +639,11 @@ arl2_status arl2_kv_last_error(arl2_kv_t h) {
   ARL2_TRY(cudaStreamSynchronize(h->last_stream));
   uint32_t w = 0;
   ARL2_TRY(cudaMemcpy(&w, h->err, sizeof(w), cudaMemcpyDeviceToHost));
-  if (w) ARL2_TRY(cudaMemset(h->err, 0, sizeof(w)));
+  if (w) {
+    // a kernel that gave up may have left partial-ready flags raised
+    ARL2_TRY(cudaMemset(h->err, 0, sizeof(w)));
+    if (h->attn_ready) ARL2_TRY(cudaMemset(h->attn_ready, 0, size_t(h->sms) * 2 * sizeof(unsigned)));
+  }
   return static_cast<arl2_status>(w);
 }
 

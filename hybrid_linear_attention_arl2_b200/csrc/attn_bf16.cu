@@ -6,17 +6,31 @@
 // The first term is the intra-frame branch (ARL2 summary, section 2.1: the
 // original bidirectional softmax attention within each frame).  The second is
 // the inter-frame read-out O_inter = Q' S_{N-1} = (Q phi_q) S_{N-1}, computed
-// as Q (phi_q S_{N-1}): the product phi_q S is formed once per state write, so
-// a pass costs one extra 128 x 128 x 128 MMA per query tile.
+// as Q (phi_q S_{N-1}): phi_q S is formed once per state write, so a pass
+// costs one extra 128 x 128 x 128 MMA per 128 query rows.
 //
-// One CTA = 128 query rows of one (stream, head).  Warp roles:
-//   warp 0      TMA producer: Q once, then K_j and V_j per key tile, then MqT;
-//   warp 1      tcgen05 issuer: S = Q K_j^T, O += P V_j, X = Q MqT^T;
-//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane).
-// Tensor memory (256 columns): [0,128) S_j fp32, overwritten in place by
-// P_j (bf16 pairs, columns [0,64)) and finally by X; [128,256) the O
-// accumulator.  Two CTAs fit on an SM (99.5 KB shared memory, 256 TMEM
-// columns each), so one CTA's softmax overlaps the other's MMAs.
+// Work decomposition.  Query tiles of 128 rows are paired into blocks of 256
+// rows (sub-tiles A and B) that share every K/V tile.  The work of a launch is
+// the sequence of (block, key tile) units over all (stream, head) pairs; each
+// unit weighs the number of query tiles it covers.  A persistent grid of one
+// CTA per SM takes contiguous, equal-weight ranges of that sequence
+// ("stream-K"), so the grid stays full whatever the number of query tiles.  A
+// block whose key range is split across CTAs is finished by the CTA holding
+// its first key tiles: the others store their unnormalised partial output and
+// softmax statistics (m, l) to a scratch slot and raise a ready flag; the
+// finishing CTA combines the partials in key order (deterministic) and adds
+// the read-out.  Ready flags are reset by their consumer, so every launch
+// leaves them at zero.
+//
+// Roles (384 threads):
+//   warp 0       TMA producer: per block, Q of both sub-tiles; K_j, V_j (and
+//                MqT for blocks this CTA finishes) through a 4-slot ring;
+//   warp 1       tcgen05 issuer: S = Q K_j^T, O += P V_j, X = Q MqT^T;
+//   warp 2       tensor-memory allocator;
+//   warps 4..7   softmax + epilogue of sub-tile A (one row per thread);
+//   warps 8..11  softmax + epilogue of sub-tile B.
+// Tensor memory (512 columns): S_A [0,128), S_B [128,256) (P written in
+// place as bf16 pairs, then X), O_A [256,384), O_B [384,512).
 //
 // The same kernel without the read-out serves the softmax layers that keep a
 // growing KV cache (the K/V tensor maps then cover the cache).
@@ -26,216 +40,504 @@
 
 namespace arl2 {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 384;
+constexpr int kRing = 4;
 constexpr uint32_t kTile = 32768;  // 128 rows x 128 bf16
 constexpr uint32_t kHalf = 16384;  // one 64-column box
-constexpr int kAttnSmem = 3 * kTile + 256 + 1024;
+constexpr int kAttnSmem = (2 + kRing) * kTile + 512 + 1024;
+constexpr int kSlotFloats = kAttnSlotFloats;
+// Register split: the launch gives every thread kLaunchRegs; warpgroup 0
+// (producer, MMA issuer, allocator) drops to kCtlRegs and the two softmax
+// warpgroups rise to kSoftmaxRegs.  128 * kCtlRegs + 256 * kSoftmaxRegs must
+// not exceed 384 * kLaunchRegs, or setmaxnreg.inc would wait forever; the
+// launcher refuses to run unless the compiled kernel has exactly kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr int kCtlRegs = 72;
+constexpr int kSoftmaxRegs = 216;
+static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs <= kAttnThreads * kLaunchRegs, "register split too large");
 
-enum { B_Q, B_KF, B_KE, B_VF, B_VE, B_SF, B_PF, B_OF, B_MQ, B_XF, B_DRAIN, B_COUNT };
+enum {
+  B_QF = 0,                       // [2]
+  B_QE = 2,                       // [2]
+  B_RF = 4,                       // [kRing]
+  B_RE = 4 + kRing,               // [kRing]
+  B_SF = 4 + 2 * kRing,           // [2]
+  B_PF = B_SF + 2,                // [2]
+  B_PV = B_PF + 2,                // [2]
+  B_XF = B_PV + 2,                // [2]
+  B_ED = B_XF + 2,                // [2]
+  B_DRAIN = B_ED + 2,
+  B_COUNT
+};
+
+// ------------------------------------------------------------------ partition
+// Units are (block, key tile) pairs in (stream, head, block, key tile) order;
+// the host cuts them into per-CTA ranges of equal weight (AttnParams::range).
+struct Seg {
+  int bh, blk, j0, j1;
+};
+
+__device__ __forceinline__ bool next_seg(const AttnParams& p, unsigned& u, unsigned u_end, Seg& s) {
+  if (u >= u_end) return false;
+  const unsigned per = unsigned(p.n_blk) * unsigned(p.nkv);
+  s.bh = int(u / per);
+  const unsigned r = u - unsigned(s.bh) * per;
+  s.blk = int(r / unsigned(p.nkv));
+  s.j0 = int(r - unsigned(s.blk) * unsigned(p.nkv));
+  s.j1 = int(min(unsigned(p.nkv), unsigned(s.j0) + (u_end - u)));
+  u += unsigned(s.j1 - s.j0);
+  return true;
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   bool ok = mbar_wait(bar, parity, w);
   return __all_sync(0xffffffffu, ok);
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 2)
+__device__ __forceinline__ void named_bar(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// End of one segment for one sub-tile (a warpgroup, one row per thread).
+//  * a segment that does not start at key tile 0 stores its unnormalised O
+//    rows and (m, l) to this CTA's slot and raises the slot's ready flag;
+//  * a segment that starts at key tile 0 writes the final rows: its own
+//    accumulator, combined with the partials of the CTAs that hold the rest of
+//    the block's keys (in key order), normalised, plus the read-out X.
+// Arrives on `ed_bar` once the tensor-memory reads are done.  Returns false if
+// a wait gave up.
+__device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg s, const int cta,
+                                              const int sub, const int lane, const int row, const uint32_t lane_off,
+                                              const uint32_t tS, const uint32_t tO, const bool warp_on,
+                                              const bool row_ok, const int q_row, const float m, const float l,
+                                              uint64_t* ed_bar, volatile int* abort_flag) {
+  const int wg_thread = threadIdx.x - 128 - sub * 128;  // 0..127 within the warpgroup
+  const bool writer = s.j0 == 0, full = writer && s.j1 == p.nkv;
+  const bool use_intra = !(p.flags & 2u);
+  const bool use_inter = p.has_inter && !(p.flags & 1u);
+  bool ok = true;
+  if (!writer) {
+    float* slot = p.scratch + (size_t(cta) * 2 + sub) * kSlotFloats;
+    if (warp_on) {
+      uint32_t r[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tO + lane_off + c * 32, slice32(r, c));
+      tmem_wait_ld();
+      if (row_ok) {
+        float4* d4 = reinterpret_cast<float4*>(slot + row * 128);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
+                              __uint_as_float(r[4 * i + 3]));
+        slot[16384 + row] = m;
+        slot[16384 + 128 + row] = l;
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(ed_bar);
+    __threadfence();
+    named_bar(1 + sub, 128);
+    if (wg_thread == 0) st_release(p.ready + cta * 2 + sub, 1u);
+    return true;
+  }
+  int contrib[8];
+  int n_contrib = 0;
+  if (!full) {
+    bool complete = false;
+    for (int c2 = cta + 1; c2 < p.grid && n_contrib < 8; ++c2) {
+      const unsigned a0 = p.range[c2], a1 = p.range[c2 + 1];
+      if (a0 == a1) continue;
+      unsigned uu = a0;
+      Seg s2;
+      next_seg(p, uu, a1, s2);
+      if (s2.bh != s.bh || s2.blk != s.blk) break;
+      contrib[n_contrib++] = c2;
+      if (s2.j1 == p.nkv) {
+        complete = true;
+        break;
+      }
+    }
+    if (!complete) {  // the host partition bounds a block to 8 pieces; never expected
+      record_error(p.err, kDevBadShape);
+      *abort_flag = 1;
+    }
+    if (wg_thread == 0) {  // wait until every contributor's partial is visible
+      for (int k = 0; k < n_contrib && !*abort_flag; ++k) {
+        const unsigned* f = p.ready + contrib[k] * 2 + sub;
+        const uint64_t t0 = global_timer_ns();
+        while (ld_acquire(f) == 0u) {
+          if (*abort_flag || global_timer_ns() - t0 > p.wait_limit_ns) {
+            *abort_flag = 1;
+            record_error(p.err, kDevTimeout);
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+    }
+    named_bar(1 + sub, 128);
+    ok = !*abort_flag;
+    if (ok)
+      for (int k = 0; k < n_contrib; ++k) (void)ld_acquire(p.ready + contrib[k] * 2 + sub);
+  }
+  float M = m, inv_l = 0.f;
+  if (ok && row_ok) {
+    for (int k = 0; k < n_contrib; ++k)
+      M = fmaxf(M, p.scratch[(size_t(contrib[k]) * 2 + sub) * kSlotFloats + 16384 + row]);
+    float Lsum = l * fast_exp2(m - M);
+    for (int k = 0; k < n_contrib; ++k) {
+      const float* sl = p.scratch + (size_t(contrib[k]) * 2 + sub) * kSlotFloats;
+      Lsum = fmaf(sl[16384 + 128 + row], fast_exp2(sl[16384 + row] - M), Lsum);
+    }
+    inv_l = 1.f / Lsum;
+  }
+  const float a_self = fast_exp2(m - M) * inv_l;
+  if (ok && warp_on) {
+    const int b = s.bh / p.heads, h = s.bh % p.heads;
+    __nv_bfloat16* dst = p.o + ((size_t(b) * p.q_len + q_row) * p.heads + h) * 128;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t ro[32], rx[32];
+      tmem_ld32(tO + lane_off + c * 32, ro);
+      if (p.has_inter) tmem_ld32(tS + lane_off + c * 32, rx);
+      tmem_wait_ld();
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * a_self);
+        for (int k = 0; k < n_contrib; ++k) {
+          const float* sl = p.scratch + (size_t(contrib[k]) * 2 + sub) * kSlotFloats;
+          const float a = fast_exp2(sl[16384 + row] - M) * inv_l;
+          const float4* s4 = reinterpret_cast<const float4*>(sl + row * 128 + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 x = s4[i];
+            ro[4 * i] = __float_as_uint(fmaf(x.x, a, __uint_as_float(ro[4 * i])));
+            ro[4 * i + 1] = __float_as_uint(fmaf(x.y, a, __uint_as_float(ro[4 * i + 1])));
+            ro[4 * i + 2] = __float_as_uint(fmaf(x.z, a, __uint_as_float(ro[4 * i + 2])));
+            ro[4 * i + 3] = __float_as_uint(fmaf(x.w, a, __uint_as_float(ro[4 * i + 3])));
+          }
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t q[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 8 * g + 2 * e;
+            float v0 = use_intra ? __uint_as_float(ro[i]) : 0.f;
+            float v1 = use_intra ? __uint_as_float(ro[i + 1]) : 0.f;
+            if (use_inter) {
+              v0 += __uint_as_float(rx[i]);
+              v1 += __uint_as_float(rx[i + 1]);
+            }
+            q[e] = pack_bf16x2(v0, v1);
+          }
+          d4[g] = make_uint4(q[0], q[1], q[2], q[3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(ed_bar);
+  if (!full) {
+    named_bar(1 + sub, 128);  // every row has read the partials
+    if (wg_thread == 0)
+      for (int k = 0; k < n_contrib; ++k) p.ready[contrib[k] * 2 + sub] = 0u;
+  }
+  return ok;
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
 attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_mq,
                  const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTile;  // also MqT after the last S MMA
-  uint8_t* sV = smem + 2 * kTile;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 3 * kTile);
+  uint8_t* sQ = smem;                   // [2] sub-tiles
+  uint8_t* sR = smem + 2 * kTile;       // [kRing] K / V / MqT tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (2 + kRing) * kTile);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int nkv = (p.kv_len + 127) >> 7;
+  const int cta = blockIdx.x;
+  const unsigned u_begin = p.range[cta], u_end = p.range[cta + 1];
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], i == B_PF ? 4u : 1u);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], (i == B_PF || i == B_PF + 1 || i == B_ED || i == B_ED + 1) ? 4u : 1u);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(tmem_holder, 256);
+  if (warp == 2) tmem_alloc(tmem_holder, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tS = tmem, tO = tmem + 128;
   const WaitCtl w{abort_flag, p.err, p.wait_limit_ns};
-
+  if (warp < 4) {
+    regs_dec<kCtlRegs>();
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------------- producer
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_v);
-      const int x0 = h * 128;
-      mbar_expect_tx(&bars[B_Q], kTile);
-      tma_load_3d(sQ, &tm_q, &bars[B_Q], x0, qt * 128, b);
-      tma_load_3d(sQ + kHalf, &tm_q, &bars[B_Q], x0 + 64, qt * 128, b);
+      uint32_t ring = 0, q_use[2] = {0, 0};
       bool ok = true;
-      for (int j = 0; j < nkv; ++j) {
-        if (j > 0 && !(ok = mbar_wait(&bars[B_KE], (j - 1) & 1, w))) break;
-        mbar_expect_tx(&bars[B_KF], kTile);
-        tma_load_3d(sK, &tm_k, &bars[B_KF], x0, j * 128, b);
-        tma_load_3d(sK + kHalf, &tm_k, &bars[B_KF], x0 + 64, j * 128, b);
-        if (j > 0 && !(ok = mbar_wait(&bars[B_VE], (j - 1) & 1, w))) break;
-        mbar_expect_tx(&bars[B_VF], kTile);
-        tma_load_3d(sV, &tm_v, &bars[B_VF], x0, j * 128, b);
-        tma_load_3d(sV + kHalf, &tm_v, &bars[B_VF], x0 + 64, j * 128, b);
-      }
-      if (ok && p.has_inter && mbar_wait(&bars[B_KE], (nkv - 1) & 1, w)) {
-        mbar_expect_tx(&bars[B_MQ], kTile);
-        const int slab = b * p.heads + h;
-        tma_load_3d(sK, &tm_mq, &bars[B_MQ], 0, 0, slab);
-        tma_load_3d(sK + kHalf, &tm_mq, &bars[B_MQ], 64, 0, slab);
+      unsigned u = u_begin;
+      Seg s;
+      while (ok && next_seg(p, u, u_end, s)) {
+        const int b = s.bh / p.heads, h = s.bh % p.heads;
+        const bool has_b = s.blk < p.n_pair;
+        const int qt_a = has_b ? 2 * s.blk : p.n_qt - 1;
+        const bool writer = s.j0 == 0;
+        const int n = s.j1 - s.j0;
+        const int ntiles = 2 * n + ((writer && p.has_inter) ? 1 : 0);
+        const int x0 = h * 128;
+        auto put = [&](int t) -> bool {
+          const uint32_t slot = ring % kRing;
+          if (ring >= kRing && !mbar_wait(&bars[B_RE + slot], ((ring / kRing) - 1) & 1, w)) return false;
+          uint8_t* dst = sR + slot * kTile;
+          mbar_expect_tx(&bars[B_RF + slot], kTile);
+          if (t < 2 * n) {
+            const int j = s.j0 + (t >> 1);
+            const CUtensorMap* m = (t & 1) ? &tm_v : &tm_k;
+            tma_load_3d(dst, m, &bars[B_RF + slot], x0, j * 128, b);
+            tma_load_3d(dst + kHalf, m, &bars[B_RF + slot], x0 + 64, j * 128, b);
+          } else {
+            tma_load_3d(dst, &tm_mq, &bars[B_RF + slot], 0, 0, s.bh);
+            tma_load_3d(dst + kHalf, &tm_mq, &bars[B_RF + slot], 64, 0, s.bh);
+          }
+          ++ring;
+          return true;
+        };
+        const int pre = min(2, ntiles);
+        for (int t = 0; ok && t < pre; ++t) ok = put(t);
+        for (int sub = 0; ok && sub < (has_b ? 2 : 1); ++sub) {
+          if (q_use[sub] > 0 && !(ok = mbar_wait(&bars[B_QE + sub], (q_use[sub] - 1) & 1, w))) break;
+          mbar_expect_tx(&bars[B_QF + sub], kTile);
+          uint8_t* dst = sQ + sub * kTile;
+          const int row = (qt_a + sub) * 128;
+          tma_load_3d(dst, &tm_q, &bars[B_QF + sub], x0, row, b);
+          tma_load_3d(dst + kHalf, &tm_q, &bars[B_QF + sub], x0 + 64, row, b);
+          ++q_use[sub];
+        }
+        for (int t = pre; ok && t < ntiles; ++t) ok = put(t);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK), va = smem_u32(sV);
+      const uint32_t qa0 = smem_u32(sQ), ra0 = smem_u32(sR);
       const uint32_t id_o = idesc_bf16(128, 128, 0, 1);  // P (TMEM) x V (MN-major)
-      bool ok = mbar_wait(&bars[B_Q], 0, w);
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int valid = min(128, p.kv_len - j * 128);
-        const int ns = min(128, (valid + 15) & ~15);
-        if (!(ok = mbar_wait(&bars[B_KF], j & 1, w))) break;
-        if (j > 0 && !(ok = mbar_wait(&bars[B_OF], (j - 1) & 1, w))) break;
+      const uint32_t id_x = idesc_bf16(128, 128, 0, 0);
+      uint32_t ring = 0, q_use[2] = {0, 0}, it[2] = {0, 0}, segs[2] = {0, 0};
+      bool ok = true;
+      unsigned u = u_begin;
+      Seg s;
+      auto get = [&](uint32_t& slot) -> bool {
+        slot = ring % kRing;
+        if (!mbar_wait(&bars[B_RF + slot], (ring / kRing) & 1, w)) return false;
+        ++ring;
         tc_fence_after();
-        const uint32_t id_s = idesc_bf16(128, ns, 0, 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tS, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), id_s, kk > 0);
+        return true;
+      };
+      while (ok && next_seg(p, u, u_end, s)) {
+        const bool has_b = s.blk < p.n_pair;
+        const int nsub = has_b ? 2 : 1;
+        const bool writer = s.j0 == 0;
+        for (int sub = 0; ok && sub < nsub; ++sub) {
+          ok = mbar_wait(&bars[B_QF + sub], q_use[sub] & 1, w);
+          ++q_use[sub];
+          if (ok && segs[sub] > 0) ok = mbar_wait(&bars[B_ED + sub], (segs[sub] - 1) & 1, w);
         }
-        mma_commit(&bars[B_SF]);
-        mma_commit(&bars[B_KE]);
-        if (!(ok = mbar_wait(&bars[B_PF], j & 1, w))) break;
-        if (!(ok = mbar_wait(&bars[B_VF], j & 1, w))) break;
-        tc_fence_after();
-        const int nk = (valid + 15) >> 4;
-        for (int kk = 0; kk < nk; ++kk)
-          mma_ts(tO, tS + kk * 8, smem_desc_sw128(va + kk * 2048, kHalf, 1024), id_o, (j > 0 || kk > 0));
-        mma_commit(&bars[B_OF]);
-        mma_commit(&bars[B_VE]);
-      }
-      if (ok && p.has_inter && mbar_wait(&bars[B_OF], (nkv - 1) & 1, w) && mbar_wait(&bars[B_MQ], 0, w)) {
-        tc_fence_after();
-        const uint32_t id_x = idesc_bf16(128, 128, 0, 0);
+        for (int t = 0; ok && t < s.j1 - s.j0; ++t) {
+          const int j = s.j0 + t;
+          const int valid = min(128, p.kv_len - j * 128);
+          const int ns = min(128, (valid + 15) & ~15);
+          const uint32_t id_s = idesc_bf16(128, ns, 0, 0);
+          uint32_t slot;
+          if (!(ok = get(slot))) break;
+          const uint32_t ka = ra0 + slot * kTile;
+          for (int sub = 0; ok && sub < nsub; ++sub) {
+            if (t > 0 && !(ok = mbar_wait(&bars[B_PV + sub], (it[sub] - 1) & 1, w))) break;
+            tc_fence_after();
+            const uint32_t qa = qa0 + sub * kTile;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tS, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), id_x, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+              mma_ss(tmem + sub * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
+                     id_s, kk > 0);
+            }
+            mma_commit(&bars[B_SF + sub]);
+          }
+          if (!ok) break;
+          mma_commit(&bars[B_RE + slot]);
+          if (!(ok = get(slot))) break;
+          const uint32_t va = ra0 + slot * kTile;
+          const int nk = (valid + 15) >> 4;
+          for (int sub = 0; ok && sub < nsub; ++sub) {
+            if (!(ok = mbar_wait(&bars[B_PF + sub], it[sub] & 1, w))) break;
+            tc_fence_after();
+            for (int kk = 0; kk < nk; ++kk)
+              mma_ts(tmem + 256 + sub * 128, tmem + sub * 128 + kk * 8,
+                     smem_desc_sw128(va + kk * 2048, kHalf, 1024), id_o, (t > 0 || kk > 0));
+            mma_commit(&bars[B_PV + sub]);
+            ++it[sub];
+          }
+          if (!ok) break;
+          mma_commit(&bars[B_RE + slot]);
         }
-        mma_commit(&bars[B_XF]);
+        if (ok && writer && p.has_inter) {
+          uint32_t slot;
+          if ((ok = get(slot))) {
+            const uint32_t ma = ra0 + slot * kTile;
+            for (int sub = 0; ok && sub < nsub; ++sub) {
+              if (!(ok = mbar_wait(&bars[B_PV + sub], (it[sub] - 1) & 1, w))) break;
+              tc_fence_after();
+              const uint32_t qa = qa0 + sub * kTile;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                mma_ss(tmem + sub * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ma + off, 16, 1024),
+                       id_x, kk > 0);
+              }
+              mma_commit(&bars[B_XF + sub]);
+            }
+            if (ok) mma_commit(&bars[B_RE + slot]);
+          }
+        }
+        if (!ok) break;
+        for (int sub = 0; sub < nsub; ++sub) {
+          mma_commit(&bars[B_QE + sub]);
+          ++segs[sub];
+        }
       }
     }
+  }
   } else {
+    regs_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------------ softmax + epilogue
+    const int sub = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const uint32_t tS = tmem + sub * 128, tO = tmem + 256 + sub * 128;
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    uint32_t it = 0, xs = 0;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      if (!(ok = warp_wait(&bars[B_SF], j & 1, w))) break;
-      tc_fence_after();
-      const int valid = min(128, p.kv_len - j * 128);
-      float mx = -INFINITY;
+    unsigned u = u_begin;
+    Seg s;
+    while (ok && next_seg(p, u, u_end, s)) {
+      const bool has_b = s.blk < p.n_pair;
+      if (sub == 1 && !has_b) continue;
+      const int b = s.bh / p.heads, h = s.bh % p.heads;
+      const int qt = (has_b ? 2 * s.blk : p.n_qt - 1) + sub;
+      const int q_row = qt * 128 + row;
+      const bool row_ok = q_row < p.q_len;
+      const bool warp_on = qt * 128 + quarter * 32 < p.q_len;  // warp-uniform
+      const bool writer = s.j0 == 0, full = writer && s.j1 == p.nkv;
+      float m = -INFINITY, l = 0.f;
+      for (int t = 0; t < s.j1 - s.j0; ++t) {
+        if (!(ok = warp_wait(&bars[B_SF + sub], it & 1, w))) break;
+        tc_fence_after();
+        if (warp_on) {
+          const int j = s.j0 + t;
+          const int valid = min(128, p.kv_len - j * 128);
+          // the whole 128-column row of S in one round trip
+          uint32_t r[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + lane_off + c * 32, r);
-        tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + c * 32, slice32(r, c));
+          tmem_wait_ld();
+          if (valid < 128) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(r[i]));
-      }
-      mx *= sl2;
-      // Lazy rescaling: the running max moves only when it grows by more than
-      // 2^8, so P stays <= 256 and the O accumulator is touched rarely.
-      if (j == 0) {
-        m = mx;
-      } else {
-        const bool need = mx > m + 8.f;
-        if (__any_sync(0xffffffffu, need)) {
-          const float f = need ? fast_exp2(m - mx) : 1.f;
-          if (need) m = mx;
-          l *= f;
+            for (int i = 0; i < 128; ++i)
+              if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+          }
+          float m4[4] = {__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]),
+                         __uint_as_float(r[3])};
+#pragma unroll
+          for (int i = 4; i < 128; i += 8) {
+            m4[0] = fmax3(m4[0], __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+            m4[1] = fmax3(m4[1], __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+            m4[2] = fmax3(m4[2], __uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
+            m4[3] = fmax3(m4[3], __uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
+          }
+          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+          // Lazy rescaling: the running max moves only when it grows by more
+          // than 8 (a factor 256), so P stays <= 256 and O is touched rarely.
+          // O is rescaled after P is written (the S row is dead by then) and
+          // before P is signalled, so PV always sees a consistent O.
+          float f = 1.f;
+          bool any_rescale = false;
+          if (t == 0) {
+            m = mx;
+          } else {
+            const bool need = mx > m + 8.f;
+            any_rescale = __any_sync(0xffffffffu, need);
+            if (need) {
+              f = fast_exp2(m - mx);
+              m = mx;
+            }
+          }
+          // P = exp2(S * scale * log2(e) - m), packed to bf16 pairs over S's first 64 columns
+          const float nm = -m;
+          float l0 = 0.f, l1 = 0.f;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + lane_off + c * 32, r);
-            tmem_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-            tmem_st32(tO + lane_off + c * 32, r);
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1;
+              ffma2(x0, x1, __uint_as_float(r[c * 32 + 2 * i]), __uint_as_float(r[c * 32 + 2 * i + 1]), sl2, sl2,
+                    nm, nm);
+              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+              fadd2(l0, l1, l0, l1, p0, p1);
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + lane_off + c * 16, pk);
+          }
+          l = fmaf(l, f, l0 + l1);
+          if (any_rescale) {
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + lane_off + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+              tmem_st32(tO + lane_off + c * 32, o);
+            }
           }
           tmem_wait_st();
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_PF + sub]);
+        ++it;
       }
-      const float nm = -m;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + lane_off + c * 32, r);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = c * 32 + 2 * i;
-          const float p0 = col < valid ? fast_exp2(fmaf(__uint_as_float(r[2 * i]), sl2, nm)) : 0.f;
-          const float p1 = col + 1 < valid ? fast_exp2(fmaf(__uint_as_float(r[2 * i + 1]), sl2, nm)) : 0.f;
-          l += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + lane_off + c * 16, pk);
+      if (!ok) break;
+      if (!(ok = warp_wait(&bars[B_PV + sub], (it - 1) & 1, w))) break;
+      if (writer && p.has_inter) {
+        if (!(ok = warp_wait(&bars[B_XF + sub], xs & 1, w))) break;
+        ++xs;
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_PF]);
-    }
-    if (ok) ok = warp_wait(&bars[B_OF], (nkv - 1) & 1, w);
-    if (ok && p.has_inter) ok = warp_wait(&bars[B_XF], 0, w);
-    if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      const bool use_intra = !(p.flags & 2u);
-      const bool use_inter = p.has_inter && !(p.flags & 1u);
-      const int q_row = qt * 128 + row;
-      __nv_bfloat16* dst = p.o + ((size_t(b) * p.q_len + q_row) * p.heads + h) * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t ro[32], rx[32];
-        tmem_ld32(tO + lane_off + c * 32, ro);
-        if (p.has_inter) tmem_ld32(tS + lane_off + c * 32, rx);
-        tmem_wait_ld();
-        uint32_t packed[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float v0 = use_intra ? __uint_as_float(ro[2 * i]) * inv_l : 0.f;
-          float v1 = use_intra ? __uint_as_float(ro[2 * i + 1]) * inv_l : 0.f;
-          if (use_inter) {
-            v0 += __uint_as_float(rx[2 * i]);
-            v1 += __uint_as_float(rx[2 * i + 1]);
-          }
-          packed[i] = pack_bf16x2(v0, v1);
-        }
-        if (q_row < p.q_len) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            d4[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-        }
-      }
+      if (!segment_epilogue(p, s, cta, sub, lane, row, lane_off, tS, tO, warp_on, row_ok, q_row, m, l,
+                            &bars[B_ED + sub], abort_flag))
+        ok = false;
     }
   }
 
@@ -247,9 +549,8 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // shared and tensor memory are released.
     if (warp == 1 && lane == 0) {
       mma_commit(&bars[B_DRAIN]);
-      WaitCtl drain{abort_flag, nullptr, 10000000ull};
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(&bars[B_DRAIN], 0) && global_timer_ns() - t0 < drain.limit_ns) {
+      while (!mbar_try_wait(&bars[B_DRAIN], 0) && global_timer_ns() - t0 < 10000000ull) {
       }
     }
     if (warp == 0 && lane == 0) {
@@ -259,20 +560,67 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     __syncthreads();
   }
-  if (warp == 1) {
+  if (warp == 2) {
+    __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tmq, const AttnParams& p, int batch, cudaStream_t stream) {
+                             const CUtensorMap& tmq, const AttnParams& p, cudaStream_t stream) {
   static unsigned done = 0;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(attn_bf16_kernel), kAttnSmem, &done);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.q_len + 127) / 128, p.heads, batch);
-  attn_bf16_kernel<<<grid, kAttnThreads, kAttnSmem, stream>>>(tq, tk, tv, tmq, p);
-  return cudaGetLastError();
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attn_bf16_kernel);
+    if (e != cudaSuccess) return e;
+    regs = fa.numRegs;
+  }
+  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;  // the register split needs this count
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = kAttnSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the combine waits on peers
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_bf16_kernel, tq, tk, tv, tmq, p);
+}
+
+bool attn_partition(AttnParams& p, int batch, int sms) {
+  p.n_qt = (p.q_len + 127) / 128;
+  p.n_pair = p.n_qt / 2;
+  p.n_blk = p.n_pair + (p.n_qt & 1);
+  p.nkv = (p.kv_len + 127) / 128;
+  const long long bh = (long long)batch * p.heads;
+  const long long units = bh * p.n_blk * p.nkv;
+  if (units >= (1LL << 31)) return false;
+  p.total_weight = bh * p.n_qt * p.nkv;
+  // Each CTA takes at least a sixth of a two-tile block, so a block is split
+  // across at most eight CTAs (the finishing CTA reads at most seven partials).
+  const long long w_min = (2LL * p.nkv + 5) / 6;
+  long long g = p.total_weight / (w_min > 0 ? w_min : 1);
+  if (g < 1) g = 1;
+  if (g > sms) g = sms;
+  if (g > kAttnMaxGrid) g = kAttnMaxGrid;
+  p.grid = int(g);
+  // CTA c starts at the first unit whose start weight is >= W * c / grid.
+  const long long wbh = (long long)p.n_qt * p.nkv;
+  const long long pair_w = (long long)p.n_pair * 2 * p.nkv;
+  auto units_before = [&](long long w) {
+    const long long b_h = w / wbh, r = w - b_h * wbh;
+    long long u = b_h * (long long)p.n_blk * p.nkv;
+    u += r <= pair_w ? (r + 1) / 2 : (long long)p.n_pair * p.nkv + (r - pair_w);
+    return u;
+  };
+  for (int c = 0; c <= p.grid; ++c) p.range[c] = unsigned(units_before(p.total_weight * c / p.grid));
+  return true;
 }
 
 }  // namespace arl2

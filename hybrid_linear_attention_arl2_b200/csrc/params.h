@@ -9,18 +9,33 @@
 
 namespace arl2 {
 
-// Fused intra-frame softmax + inter-frame read-out (attn_bf16.cu).
+constexpr int kAttnMaxGrid = 192;  // persistent CTAs at most (>= the SM count of a B200)
+
+// Fused intra-frame softmax + inter-frame read-out (attn_bf16.cu): a
+// persistent grid over (query-tile pair, key tile) units, see the kernel.
 struct AttnParams {
   __nv_bfloat16* o;     // [B, q_len, H, 128]
   int q_len;            // query tokens per stream
   int kv_len;           // valid key/value tokens per stream
   int heads;
+  int n_qt;             // query tiles of 128 per (stream, head)
+  int n_pair;           // n_qt / 2: blocks with two sub-tiles
+  int n_blk;            // blocks per (stream, head): n_pair + n_qt % 2
+  int nkv;              // key tiles of 128
+  long long total_weight;  // B * H * n_qt * nkv
+  int grid;             // persistent CTAs (<= kAttnMaxGrid)
+  unsigned range[kAttnMaxGrid + 1];  // CTA c takes units [range[c], range[c + 1])
   float scale_log2;     // softmax scale * log2(e)
   uint32_t flags;       // 1: intra only, 2: inter only
   int has_inter;        // 1: add Q MqT^T
+  float* scratch;       // [grid][2][kAttnSlotFloats] partial rows and (m, l)
+  unsigned* ready;      // [grid][2] partial-ready flags, zero between launches
   uint32_t* err;        // device error word
   uint64_t wait_limit_ns;
 };
+
+// floats of one partial slot (one sub-tile of one CTA): 128 x 128 O rows, m[128], l[128]
+constexpr int kAttnSlotFloats = 128 * 128 + 256;
 
 // State write and read-out preparation (state_bf16.cu).
 struct StateParams {
@@ -66,7 +81,10 @@ struct F32CommitParams {
 };
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tmq, const AttnParams& p, int batch, cudaStream_t stream);
+                             const CUtensorMap& tmq, const AttnParams& p, cudaStream_t stream);
+// Fills the partition fields of `p` for B streams on a device with `sms` SMs;
+// false if the problem is too large for 32-bit unit indices.
+bool attn_partition(AttnParams& p, int batch, int sms);
 cudaError_t launch_state_partial(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tpk,
                                  const CUtensorMap& tpv, const CUtensorMap& ts, const StateParams& p, int batch,
                                  cudaStream_t stream);
