@@ -84,7 +84,7 @@ def test_long_stream_flat_time_and_memory():
     # timing and memory of the same stream, inputs resident
     phi = [dev(x, "bf16") for x in wl.phi(0)]
     layer = arl2.HybridLayer(1, cfg.heads, 128, cfg.tokens, arl2.ARL2_BF16, *phi, corr_scale=cfg.corr_scale)
-    pool = [tuple(dev(x, "bf16") for x in wl.pool_entry(0, i)) for i in range(cfg.pool)]
+    pool = [tuple(dev(x[None], "bf16") for x in wl.pool_entry(0, i)) for i in range(cfg.pool)]
     gates = [(torch.from_numpy(wl.alpha(0, n)).cuda(), torch.from_numpy(wl.beta(0, n)).cuda())
              for n in range(cfg.frames)]
     O = torch.empty_like(pool[0][0])
@@ -130,7 +130,7 @@ def test_attention_stack_sample():
     def trip(l, n, p):
         i = wl.pool_index(l, n, p)
         if i not in pool:
-            pool[i] = tuple(dev(x, "bf16") for x in wl.pool_entry(0, i))
+            pool[i] = tuple(dev(x[None], "bf16") for x in wl.pool_entry(0, i))
         return pool[i]
 
     S_ref = {l: np.zeros((1, cfg.heads, 128, 128)) for l in (0, 21)}
