@@ -63,9 +63,8 @@ enum {
   B_RE = 4 + kRing,               // [kRing]
   B_SF = 4 + 2 * kRing,           // [2]
   B_PF = B_SF + 2,                // [2]
-  B_PV = B_PF + 2,                // [2]
-  B_XF = B_PV + 2,                // [2]
-  B_ED = B_XF + 2,                // [2]
+  B_SD = B_PF + 2,                // [2] segment done: every MMA of the segment completed
+  B_ED = B_SD + 2,                // [2]
   B_DRAIN = B_ED + 2,
   B_COUNT
 };
@@ -340,9 +339,17 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      const uint32_t qa0 = smem_u32(sQ), ra0 = smem_u32(sR);
+      // Order per key tile t (sub-tile B lags one tile behind A):
+      //   S_A(t), PV_B(t-1), S_B(t), PV_A(t)
+      // so that each softmax warpgroup has two MMAs' time to produce P.  An S
+      // MMA is issued right after the PV that reads the P it overwrites:
+      // tcgen05.mma operations of one thread execute in issue order.
       const uint32_t id_o = idesc_bf16(128, 128, 0, 1);  // P (TMEM) x V (MN-major)
       const uint32_t id_x = idesc_bf16(128, 128, 0, 0);
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dr0 = smem_desc_sw128(smem_u32(sR), 16, 1024);       // K-major ring tile
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(sR), kHalf, 1024);    // MN-major ring tile
+      constexpr uint32_t kTile16 = kTile >> 4, kHalf16 = kHalf >> 4;       // descriptor address units
       uint32_t ring = 0, q_use[2] = {0, 0}, it[2] = {0, 0}, segs[2] = {0, 0};
       bool ok = true;
       unsigned u = u_begin;
@@ -354,73 +361,92 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_after();
         return true;
       };
+      // S = Q K^T over the 8 K-steps of one tile
+      auto mma_s = [&](int sub, uint32_t kslot, uint32_t id_s) {
+        const uint64_t a = dq0 + sub * kTile16, b = dr0 + kslot * kTile16;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
+          mma_ss(tmem + sub * 128, a + off, b + off, id_s, kk > 0);
+        }
+      };
+      // O += P V over the key tokens of one tile (P in TMEM over S's columns)
+      auto mma_pv = [&](int sub, uint32_t vslot, int nk, bool first) {
+        const uint64_t b = dv0 + vslot * kTile16;
+        for (int kk = 0; kk < nk; ++kk)
+          mma_ts(tmem + 256 + sub * 128, tmem + sub * 128 + kk * 8, b + kk * (2048 >> 4), id_o, (!first || kk > 0));
+      };
+      auto tile_shape = [&](int j, uint32_t& id_s, int& nk) {
+        const int valid = min(128, p.kv_len - j * 128);
+        id_s = idesc_bf16(128, min(128, (valid + 15) & ~15), 0, 0);
+        nk = (valid + 15) >> 4;
+      };
       while (ok && next_seg(p, u, u_end, s)) {
         const bool has_b = s.blk < p.n_pair;
         const int nsub = has_b ? 2 : 1;
         const bool writer = s.j0 == 0;
+        const int n = s.j1 - s.j0;
         for (int sub = 0; ok && sub < nsub; ++sub) {
           ok = mbar_wait(&bars[B_QF + sub], q_use[sub] & 1, w);
           ++q_use[sub];
           if (ok && segs[sub] > 0) ok = mbar_wait(&bars[B_ED + sub], (segs[sub] - 1) & 1, w);
         }
-        for (int t = 0; ok && t < s.j1 - s.j0; ++t) {
-          const int j = s.j0 + t;
-          const int valid = min(128, p.kv_len - j * 128);
-          const int ns = min(128, (valid + 15) & ~15);
-          const uint32_t id_s = idesc_bf16(128, ns, 0, 0);
-          uint32_t slot;
-          if (!(ok = get(slot))) break;
-          const uint32_t ka = ra0 + slot * kTile;
-          for (int sub = 0; ok && sub < nsub; ++sub) {
-            if (t > 0 && !(ok = mbar_wait(&bars[B_PV + sub], (it[sub] - 1) & 1, w))) break;
-            tc_fence_after();
-            const uint32_t qa = qa0 + sub * kTile;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-              mma_ss(tmem + sub * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                     id_s, kk > 0);
+        uint32_t vprev = 0;
+        int nk_prev = 0;
+        for (int t = 0; ok && t < n; ++t) {
+          uint32_t id_s, kslot, vslot;
+          int nk;
+          tile_shape(s.j0 + t, id_s, nk);
+          if (!(ok = get(kslot))) break;
+          mma_s(0, kslot, id_s);
+          mma_commit(&bars[B_SF + 0]);
+          if (has_b) {
+            if (t > 0) {
+              if (!(ok = mbar_wait(&bars[B_PF + 1], it[1] & 1, w))) break;
+              tc_fence_after();
+              mma_pv(1, vprev, nk_prev, t == 1);
+              ++it[1];
+              mma_commit(&bars[B_RE + vprev]);
             }
-            mma_commit(&bars[B_SF + sub]);
+            mma_s(1, kslot, id_s);
+            mma_commit(&bars[B_SF + 1]);
           }
-          if (!ok) break;
-          mma_commit(&bars[B_RE + slot]);
-          if (!(ok = get(slot))) break;
-          const uint32_t va = ra0 + slot * kTile;
-          const int nk = (valid + 15) >> 4;
-          for (int sub = 0; ok && sub < nsub; ++sub) {
-            if (!(ok = mbar_wait(&bars[B_PF + sub], it[sub] & 1, w))) break;
+          mma_commit(&bars[B_RE + kslot]);
+          if (!(ok = get(vslot))) break;
+          if (!(ok = mbar_wait(&bars[B_PF + 0], it[0] & 1, w))) break;
+          tc_fence_after();
+          mma_pv(0, vslot, nk, t == 0);
+          ++it[0];
+          if (!has_b) mma_commit(&bars[B_RE + vslot]);
+          vprev = vslot;
+          nk_prev = nk;
+        }
+        if (ok && has_b && n > 0) {
+          if ((ok = mbar_wait(&bars[B_PF + 1], it[1] & 1, w))) {
             tc_fence_after();
-            for (int kk = 0; kk < nk; ++kk)
-              mma_ts(tmem + 256 + sub * 128, tmem + sub * 128 + kk * 8,
-                     smem_desc_sw128(va + kk * 2048, kHalf, 1024), id_o, (t > 0 || kk > 0));
-            mma_commit(&bars[B_PV + sub]);
-            ++it[sub];
+            mma_pv(1, vprev, nk_prev, n == 1);
+            ++it[1];
+            mma_commit(&bars[B_RE + vprev]);
           }
-          if (!ok) break;
-          mma_commit(&bars[B_RE + slot]);
         }
         if (ok && writer && p.has_inter) {
-          uint32_t slot;
-          if ((ok = get(slot))) {
-            const uint32_t ma = ra0 + slot * kTile;
-            for (int sub = 0; ok && sub < nsub; ++sub) {
-              if (!(ok = mbar_wait(&bars[B_PV + sub], (it[sub] - 1) & 1, w))) break;
-              tc_fence_after();
-              const uint32_t qa = qa0 + sub * kTile;
+          uint32_t mslot;
+          if ((ok = get(mslot))) {
+            const uint64_t b = dr0 + mslot * kTile16;
+            for (int sub = 0; sub < nsub; ++sub) {
+              const uint64_t a = dq0 + sub * kTile16;
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                mma_ss(tmem + sub * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ma + off, 16, 1024),
-                       id_x, kk > 0);
+                const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
+                mma_ss(tmem + sub * 128, a + off, b + off, id_x, kk > 0);
               }
-              mma_commit(&bars[B_XF + sub]);
             }
-            if (ok) mma_commit(&bars[B_RE + slot]);
+            mma_commit(&bars[B_RE + mslot]);
           }
         }
         if (!ok) break;
         for (int sub = 0; sub < nsub; ++sub) {
+          mma_commit(&bars[B_SD + sub]);
           mma_commit(&bars[B_QE + sub]);
           ++segs[sub];
         }
@@ -436,7 +462,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t tS = tmem + sub * 128, tO = tmem + 256 + sub * 128;
     const float sl2 = p.scale_log2;
-    uint32_t it = 0, xs = 0;
+    uint32_t it = 0, segs_done = 0;
     bool ok = true;
     unsigned u = u_begin;
     Seg s;
@@ -529,11 +555,8 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         ++it;
       }
       if (!ok) break;
-      if (!(ok = warp_wait(&bars[B_PV + sub], (it - 1) & 1, w))) break;
-      if (writer && p.has_inter) {
-        if (!(ok = warp_wait(&bars[B_XF + sub], xs & 1, w))) break;
-        ++xs;
-      }
+      if (!(ok = warp_wait(&bars[B_SD + sub], segs_done & 1, w))) break;
+      ++segs_done;
       tc_fence_after();
       if (!segment_epilogue(p, s, cta, sub, lane, row, lane_off, tS, tO, warp_on, row_ok, q_row, m, l,
                             &bars[B_ED + sub], abort_flag))
