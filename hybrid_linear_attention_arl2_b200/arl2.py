@@ -59,6 +59,7 @@ _SIGS = {
     "arl2_kv_last_error": (_I32, [_VP]),
     "arl2_kv_destroy": (_I32, [_VP]),
     "arl2_selftest_wait_timeout": (_I32, [_U64, _VP]),
+    "arl2_selftest_exp2": (_I32, [_VP, _VP, _I64, _VP]),
     "arl2_status_string": (ctypes.c_char_p, [_I32]),
     "arl2_abi_version": (_I32, []),
 }
@@ -193,6 +194,10 @@ def arl2_kv_destroy(h) -> None:
 
 def arl2_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     return load_library().arl2_selftest_wait_timeout(limit_ns, _stream(stream))
+
+
+def arl2_selftest_exp2(x, y, stream=None) -> None:
+    _check(load_library().arl2_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "arl2_selftest_exp2")
 
 
 def arl2_status_string(status: int) -> str:

@@ -673,4 +673,11 @@ arl2_status arl2_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   return static_cast<arl2_status>(w);
 }
 
+arl2_status arl2_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
+  if (!x || !y || n < 0) return ARL2_ERR_INVALID_ARGUMENT;
+  if (n == 0) return ARL2_OK;
+  ARL2_TRY(launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)));
+  return ARL2_OK;
+}
+
 }  // extern "C"

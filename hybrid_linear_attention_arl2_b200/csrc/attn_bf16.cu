@@ -51,6 +51,7 @@ constexpr int kSlotFloats = kAttnSlotFloats;
 // warpgroups rise to kSoftmaxRegs.  128 * kCtlRegs + 256 * kSoftmaxRegs must
 // not exceed 384 * kLaunchRegs, or setmaxnreg.inc would wait forever; the
 // launcher refuses to run unless the compiled kernel has exactly kLaunchRegs.
+constexpr int kPolyPairs = 6;  // of every 16 exp2 pairs of a full tile, this many run on the FMA pipe
 constexpr int kLaunchRegs = 168;
 constexpr int kCtlRegs = 72;
 constexpr int kSoftmaxRegs = 216;
@@ -518,22 +519,47 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               m = mx;
             }
           }
-          // P = exp2(S * scale * log2(e) - m), packed to bf16 pairs over S's first 64 columns
+          // P = exp2(S * scale * log2(e) - m), packed to bf16 pairs over S's first 64
+          // columns.  On full tiles kPolyPairs of every 16 pairs take the FMA-pipe
+          // exp2 so that the MUFU is not the limit; the masked last tile (columns
+          // at -inf) takes the MUFU for all of them.
           const float nm = -m;
           float l0 = 0.f, l1 = 0.f;
+          if (valid == 128) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float x0, x1;
-              ffma2(x0, x1, __uint_as_float(r[c * 32 + 2 * i]), __uint_as_float(r[c * 32 + 2 * i + 1]), sl2, sl2,
-                    nm, nm);
-              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-              fadd2(l0, l1, l0, l1, p0, p1);
-              pk[i] = pack_bf16x2(p0, p1);
+              for (int i = 0; i < 16; ++i) {
+                float x0, x1, p0, p1;
+                ffma2(x0, x1, __uint_as_float(r[c * 32 + 2 * i]), __uint_as_float(r[c * 32 + 2 * i + 1]), sl2, sl2,
+                      nm, nm);
+                if (i >= 16 - kPolyPairs) {
+                  exp2_poly2(p0, p1, x0, x1);
+                } else {
+                  p0 = fast_exp2(x0);
+                  p1 = fast_exp2(x1);
+                }
+                fadd2(l0, l1, l0, l1, p0, p1);
+                pk[i] = pack_bf16x2(p0, p1);
+              }
+              tmem_st16(tS + lane_off + c * 16, pk);
             }
-            tmem_st16(tS + lane_off + c * 16, pk);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float x0, x1;
+                ffma2(x0, x1, __uint_as_float(r[c * 32 + 2 * i]), __uint_as_float(r[c * 32 + 2 * i + 1]), sl2, sl2,
+                      nm, nm);
+                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                fadd2(l0, l1, l0, l1, p0, p1);
+                pk[i] = pack_bf16x2(p0, p1);
+              }
+              tmem_st16(tS + lane_off + c * 16, pk);
+            }
           }
           l = fmaf(l, f, l0 + l1);
           if (any_rescale) {

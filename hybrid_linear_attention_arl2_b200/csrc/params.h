@@ -96,6 +96,7 @@ cudaError_t launch_f32_commit(const F32CommitParams& p, int batch, cudaStream_t 
 cudaError_t launch_transpose_bf16(const __nv_bfloat16* src, __nv_bfloat16* dst, int slabs, cudaStream_t stream);
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
+cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
 
 // Sets the dynamic shared-memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* done_mask);

@@ -53,6 +53,23 @@ cudaError_t launch_wait_selftest(uint32_t* err, uint64_t limit_ns, cudaStream_t 
   return cudaGetLastError();
 }
 
+// y = 2^x through the attention kernel's FMA-pipe exp2 (for its accuracy test).
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    exp2_poly2(y[i], y[i + 1], x[i], x[i + 1]);
+  } else if (i < n) {
+    float d;
+    exp2_poly2(y[i], d, x[i], 0.f);
+  }
+}
+
+cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream) {
+  const long long pairs = (n + 1) / 2;
+  exp2_poly_kernel<<<unsigned((pairs + 255) / 256), 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
+
 cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* done_mask) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -148,6 +148,12 @@ arl2_status arl2_kv_destroy(arl2_kv_t kv);
  * kernel returned and reported it) -- used by the failure-detection tests. */
 arl2_status arl2_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
+/* y[i] = 2^x[i] (device float32 arrays of n values) through the FMA-pipe
+ * exponential the attention kernel uses for part of its softmax (a degree-3
+ * polynomial after rounding x to an integer; inputs clamped to [-125, 125];
+ * relative error <= 1.0e-4).  For accuracy tests of that routine. */
+arl2_status arl2_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
+
 const char* arl2_status_string(arl2_status s);
 int32_t arl2_abi_version(void);
 

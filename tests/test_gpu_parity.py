@@ -258,3 +258,22 @@ def test_invalid_device_arguments():
     layer.close()
     with pytest.raises(arl2.Arl2Error):
         arl2.arl2_frame_query(h, Q, K, V, torch.empty_like(Q))  # use after destroy
+
+
+def test_fma_pipe_exp2_against_cuda_exp2f():
+    """The FMA-pipe exp2 used for part of the softmax stays within its stated
+    relative error bound (1e-4) of CUDA's exp2f over the clamped range, and is
+    exact at integers."""
+    x = torch.cat([torch.linspace(-125.0, 125.0, 1_000_001, device="cuda"),
+                   torch.arange(-125, 126, device="cuda", dtype=torch.float32),
+                   torch.rand(200_000, device="cuda") * -30.0])
+    y = torch.empty_like(x)
+    arl2.arl2_selftest_exp2(x, y)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel <= 1.0e-4, rel
+    # at integers f = 0: the result is c0 * 2^n with c0 the polynomial's constant term
+    ints = torch.arange(-125, 126, device="cuda", dtype=torch.float32)
+    yi = torch.empty_like(ints)
+    arl2.arl2_selftest_exp2(ints, yi)
+    assert torch.equal(yi / torch.exp2(ints), torch.full_like(ints, yi[125].item()))
