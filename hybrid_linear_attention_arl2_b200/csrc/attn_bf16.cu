@@ -259,6 +259,124 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
   return ok;
 }
 
+// The tcgen05 issuer (one thread).  Order per key tile t, with sub-tile B one
+// tile behind A:   S_A(t), PV_B(t-1), S_B(t), PV_A(t)
+// so that each softmax warpgroup has two MMA groups' time to produce P.  An S
+// MMA is issued right after the PV that reads the P it overwrites: tcgen05.mma
+// operations of one thread execute in issue order.  All state is in scalars
+// (no arrays indexed at run time) so the issue loop stays in registers.
+__device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, const uint32_t tmem,
+                                           const uint32_t q_addr, const uint32_t r_addr, const unsigned u_begin,
+                                           const unsigned u_end, const WaitCtl& w) {
+  constexpr uint32_t kTile16 = kTile >> 4, kHalf16 = kHalf >> 4;  // descriptor address units
+  const uint32_t id_o = idesc_bf16(128, 128, 0, 1);                 // P (TMEM) x V (MN-major)
+  const uint32_t id_x = idesc_bf16(128, 128, 0, 0);
+  const uint64_t dqa = smem_desc_sw128(q_addr, 16, 1024), dqb = dqa + kTile16;
+  const uint64_t dr0 = smem_desc_sw128(r_addr, 16, 1024);     // K-major ring tile
+  const uint64_t dv0 = smem_desc_sw128(r_addr, kHalf, 1024);  // MN-major ring tile
+  const uint32_t tSA = tmem, tSB = tmem + 128, tOA = tmem + 256, tOB = tmem + 384;
+  uint32_t ring = 0, qa_use = 0, qb_use = 0, ita = 0, itb = 0, sega = 0, segb = 0;
+  unsigned u = u_begin;
+  Seg s;
+  while (next_seg(p, u, u_end, s)) {
+    const bool has_b = s.blk < p.n_pair;
+    const int n = s.j1 - s.j0;
+    if (!mbar_wait(&bars[B_QF + 0], qa_use & 1, w)) return;
+    ++qa_use;
+    if (sega > 0 && !mbar_wait(&bars[B_ED + 0], (sega - 1) & 1, w)) return;
+    if (has_b) {
+      if (!mbar_wait(&bars[B_QF + 1], qb_use & 1, w)) return;
+      ++qb_use;
+      if (segb > 0 && !mbar_wait(&bars[B_ED + 1], (segb - 1) & 1, w)) return;
+    }
+    uint32_t vprev = 0;
+    int nk_prev = 0;
+    for (int t = 0; t < n; ++t) {
+      const int j = s.j0 + t;
+      const int valid = min(128, p.kv_len - j * 128);
+      const uint32_t id_s = idesc_bf16(128, min(128, (valid + 15) & ~15), 0, 0);
+      const int nk = (valid + 15) >> 4;
+      // K_j
+      const uint32_t kslot = ring & (kRing - 1);
+      if (!mbar_wait(&bars[B_RF + kslot], (ring / kRing) & 1, w)) return;
+      ++ring;
+      tc_fence_after();
+      const uint64_t dk = dr0 + kslot * kTile16;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
+        mma_ss(tSA, dqa + off, dk + off, id_s, kk > 0);
+      }
+      mma_commit(&bars[B_SF + 0]);
+      if (has_b) {
+        if (t > 0) {
+          if (!mbar_wait(&bars[B_PF + 1], itb & 1, w)) return;
+          ++itb;
+          tc_fence_after();
+          const uint64_t dvp = dv0 + vprev * kTile16;
+          for (int kk = 0; kk < nk_prev; ++kk) mma_ts(tOB, tSB + kk * 8, dvp + kk * 128, id_o, (t > 1 || kk > 0));
+          mma_commit(&bars[B_RE + vprev]);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
+          mma_ss(tSB, dqb + off, dk + off, id_s, kk > 0);
+        }
+        mma_commit(&bars[B_SF + 1]);
+      }
+      mma_commit(&bars[B_RE + kslot]);
+      // V_j
+      const uint32_t vslot = ring & (kRing - 1);
+      if (!mbar_wait(&bars[B_RF + vslot], (ring / kRing) & 1, w)) return;
+      ++ring;
+      if (!mbar_wait(&bars[B_PF + 0], ita & 1, w)) return;
+      ++ita;
+      tc_fence_after();
+      const uint64_t dvv = dv0 + vslot * kTile16;
+      for (int kk = 0; kk < nk; ++kk) mma_ts(tOA, tSA + kk * 8, dvv + kk * 128, id_o, (t > 0 || kk > 0));
+      if (!has_b) mma_commit(&bars[B_RE + vslot]);
+      vprev = vslot;
+      nk_prev = nk;
+    }
+    if (has_b && n > 0) {
+      if (!mbar_wait(&bars[B_PF + 1], itb & 1, w)) return;
+      ++itb;
+      tc_fence_after();
+      const uint64_t dvp = dv0 + vprev * kTile16;
+      for (int kk = 0; kk < nk_prev; ++kk) mma_ts(tOB, tSB + kk * 8, dvp + kk * 128, id_o, (n > 1 || kk > 0));
+      mma_commit(&bars[B_RE + vprev]);
+    }
+    if (s.j0 == 0 && p.has_inter) {  // X = Q MqT^T for the rows this CTA finishes
+      const uint32_t mslot = ring & (kRing - 1);
+      if (!mbar_wait(&bars[B_RF + mslot], (ring / kRing) & 1, w)) return;
+      ++ring;
+      tc_fence_after();
+      const uint64_t dm = dr0 + mslot * kTile16;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
+        mma_ss(tSA, dqa + off, dm + off, id_x, kk > 0);
+      }
+      if (has_b) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
+          mma_ss(tSB, dqb + off, dm + off, id_x, kk > 0);
+        }
+      }
+      mma_commit(&bars[B_RE + mslot]);
+    }
+    mma_commit(&bars[B_SD + 0]);
+    mma_commit(&bars[B_QE + 0]);
+    ++sega;
+    if (has_b) {
+      mma_commit(&bars[B_SD + 1]);
+      mma_commit(&bars[B_QE + 1]);
+      ++segb;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_mq,
@@ -294,7 +412,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_v);
-      uint32_t ring = 0, q_use[2] = {0, 0};
+      uint32_t ring = 0, qa_use = 0, qb_use = 0;
       bool ok = true;
       unsigned u = u_begin;
       Seg s;
@@ -326,13 +444,14 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int pre = min(2, ntiles);
         for (int t = 0; ok && t < pre; ++t) ok = put(t);
         for (int sub = 0; ok && sub < (has_b ? 2 : 1); ++sub) {
-          if (q_use[sub] > 0 && !(ok = mbar_wait(&bars[B_QE + sub], (q_use[sub] - 1) & 1, w))) break;
+          const uint32_t used = sub ? qb_use : qa_use;
+          if (used > 0 && !(ok = mbar_wait(&bars[B_QE + sub], (used - 1) & 1, w))) break;
           mbar_expect_tx(&bars[B_QF + sub], kTile);
           uint8_t* dst = sQ + sub * kTile;
           const int row = (qt_a + sub) * 128;
           tma_load_3d(dst, &tm_q, &bars[B_QF + sub], x0, row, b);
           tma_load_3d(dst + kHalf, &tm_q, &bars[B_QF + sub], x0 + 64, row, b);
-          ++q_use[sub];
+          if (sub) ++qb_use; else ++qa_use;
         }
         for (int t = pre; ok && t < ntiles; ++t) ok = put(t);
       }
@@ -340,118 +459,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      // Order per key tile t (sub-tile B lags one tile behind A):
-      //   S_A(t), PV_B(t-1), S_B(t), PV_A(t)
-      // so that each softmax warpgroup has two MMAs' time to produce P.  An S
-      // MMA is issued right after the PV that reads the P it overwrites:
-      // tcgen05.mma operations of one thread execute in issue order.
-      const uint32_t id_o = idesc_bf16(128, 128, 0, 1);  // P (TMEM) x V (MN-major)
-      const uint32_t id_x = idesc_bf16(128, 128, 0, 0);
-      const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t dr0 = smem_desc_sw128(smem_u32(sR), 16, 1024);       // K-major ring tile
-      const uint64_t dv0 = smem_desc_sw128(smem_u32(sR), kHalf, 1024);    // MN-major ring tile
-      constexpr uint32_t kTile16 = kTile >> 4, kHalf16 = kHalf >> 4;       // descriptor address units
-      uint32_t ring = 0, q_use[2] = {0, 0}, it[2] = {0, 0}, segs[2] = {0, 0};
-      bool ok = true;
-      unsigned u = u_begin;
-      Seg s;
-      auto get = [&](uint32_t& slot) -> bool {
-        slot = ring % kRing;
-        if (!mbar_wait(&bars[B_RF + slot], (ring / kRing) & 1, w)) return false;
-        ++ring;
-        tc_fence_after();
-        return true;
-      };
-      // S = Q K^T over the 8 K-steps of one tile
-      auto mma_s = [&](int sub, uint32_t kslot, uint32_t id_s) {
-        const uint64_t a = dq0 + sub * kTile16, b = dr0 + kslot * kTile16;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
-          mma_ss(tmem + sub * 128, a + off, b + off, id_s, kk > 0);
-        }
-      };
-      // O += P V over the key tokens of one tile (P in TMEM over S's columns)
-      auto mma_pv = [&](int sub, uint32_t vslot, int nk, bool first) {
-        const uint64_t b = dv0 + vslot * kTile16;
-        for (int kk = 0; kk < nk; ++kk)
-          mma_ts(tmem + 256 + sub * 128, tmem + sub * 128 + kk * 8, b + kk * (2048 >> 4), id_o, (!first || kk > 0));
-      };
-      auto tile_shape = [&](int j, uint32_t& id_s, int& nk) {
-        const int valid = min(128, p.kv_len - j * 128);
-        id_s = idesc_bf16(128, min(128, (valid + 15) & ~15), 0, 0);
-        nk = (valid + 15) >> 4;
-      };
-      while (ok && next_seg(p, u, u_end, s)) {
-        const bool has_b = s.blk < p.n_pair;
-        const int nsub = has_b ? 2 : 1;
-        const bool writer = s.j0 == 0;
-        const int n = s.j1 - s.j0;
-        for (int sub = 0; ok && sub < nsub; ++sub) {
-          ok = mbar_wait(&bars[B_QF + sub], q_use[sub] & 1, w);
-          ++q_use[sub];
-          if (ok && segs[sub] > 0) ok = mbar_wait(&bars[B_ED + sub], (segs[sub] - 1) & 1, w);
-        }
-        uint32_t vprev = 0;
-        int nk_prev = 0;
-        for (int t = 0; ok && t < n; ++t) {
-          uint32_t id_s, kslot, vslot;
-          int nk;
-          tile_shape(s.j0 + t, id_s, nk);
-          if (!(ok = get(kslot))) break;
-          mma_s(0, kslot, id_s);
-          mma_commit(&bars[B_SF + 0]);
-          if (has_b) {
-            if (t > 0) {
-              if (!(ok = mbar_wait(&bars[B_PF + 1], it[1] & 1, w))) break;
-              tc_fence_after();
-              mma_pv(1, vprev, nk_prev, t == 1);
-              ++it[1];
-              mma_commit(&bars[B_RE + vprev]);
-            }
-            mma_s(1, kslot, id_s);
-            mma_commit(&bars[B_SF + 1]);
-          }
-          mma_commit(&bars[B_RE + kslot]);
-          if (!(ok = get(vslot))) break;
-          if (!(ok = mbar_wait(&bars[B_PF + 0], it[0] & 1, w))) break;
-          tc_fence_after();
-          mma_pv(0, vslot, nk, t == 0);
-          ++it[0];
-          if (!has_b) mma_commit(&bars[B_RE + vslot]);
-          vprev = vslot;
-          nk_prev = nk;
-        }
-        if (ok && has_b && n > 0) {
-          if ((ok = mbar_wait(&bars[B_PF + 1], it[1] & 1, w))) {
-            tc_fence_after();
-            mma_pv(1, vprev, nk_prev, n == 1);
-            ++it[1];
-            mma_commit(&bars[B_RE + vprev]);
-          }
-        }
-        if (ok && writer && p.has_inter) {
-          uint32_t mslot;
-          if ((ok = get(mslot))) {
-            const uint64_t b = dr0 + mslot * kTile16;
-            for (int sub = 0; sub < nsub; ++sub) {
-              const uint64_t a = dq0 + sub * kTile16;
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
-                mma_ss(tmem + sub * 128, a + off, b + off, id_x, kk > 0);
-              }
-            }
-            mma_commit(&bars[B_RE + mslot]);
-          }
-        }
-        if (!ok) break;
-        for (int sub = 0; sub < nsub; ++sub) {
-          mma_commit(&bars[B_SD + sub]);
-          mma_commit(&bars[B_QE + sub]);
-          ++segs[sub];
-        }
-      }
+      mma_issuer(p, bars, tmem, smem_u32(sQ), smem_u32(sR), u_begin, u_end, w);
     }
   }
   } else {
