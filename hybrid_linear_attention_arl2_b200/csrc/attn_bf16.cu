@@ -259,7 +259,9 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
   return ok;
 }
 
-// The tcgen05 issuer (one thread).  Order per key tile t, with sub-tile B one
+// The tcgen05 issuer (one warp: every lane runs the loop and waits, so all
+// operands are warp-uniform; the elected lane issues).  Order per key tile t,
+// with sub-tile B one
 // tile behind A:   S_A(t), PV_B(t-1), S_B(t), PV_A(t)
 // so that each softmax warpgroup has two MMA groups' time to produce P.  An S
 // MMA is issued right after the PV that reads the P it overwrites: tcgen05.mma
@@ -268,6 +270,7 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
 __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, const uint32_t tmem,
                                            const uint32_t q_addr, const uint32_t r_addr, const unsigned u_begin,
                                            const unsigned u_end, const WaitCtl& w) {
+  const bool leader = elect_one();
   constexpr uint32_t kTile16 = kTile >> 4, kHalf16 = kHalf >> 4;  // descriptor address units
   const uint32_t id_o = idesc_bf16(128, 128, 0, 1);                 // P (TMEM) x V (MN-major)
   const uint32_t id_x = idesc_bf16(128, 128, 0, 0);
@@ -281,13 +284,13 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, 
   while (next_seg(p, u, u_end, s)) {
     const bool has_b = s.blk < p.n_pair;
     const int n = s.j1 - s.j0;
-    if (!mbar_wait(&bars[B_QF + 0], qa_use & 1, w)) return;
+    if (!warp_wait(&bars[B_QF + 0], qa_use & 1, w)) return;
     ++qa_use;
-    if (sega > 0 && !mbar_wait(&bars[B_ED + 0], (sega - 1) & 1, w)) return;
+    if (sega > 0 && !warp_wait(&bars[B_ED + 0], (sega - 1) & 1, w)) return;
     if (has_b) {
-      if (!mbar_wait(&bars[B_QF + 1], qb_use & 1, w)) return;
+      if (!warp_wait(&bars[B_QF + 1], qb_use & 1, w)) return;
       ++qb_use;
-      if (segb > 0 && !mbar_wait(&bars[B_ED + 1], (segb - 1) & 1, w)) return;
+      if (segb > 0 && !warp_wait(&bars[B_ED + 1], (segb - 1) & 1, w)) return;
     }
     uint32_t vprev = 0;
     int nk_prev = 0;
@@ -298,82 +301,104 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, 
       const int nk = (valid + 15) >> 4;
       // K_j
       const uint32_t kslot = ring & (kRing - 1);
-      if (!mbar_wait(&bars[B_RF + kslot], (ring / kRing) & 1, w)) return;
+      if (!warp_wait(&bars[B_RF + kslot], (ring / kRing) & 1, w)) return;
       ++ring;
       tc_fence_after();
       const uint64_t dk = dr0 + kslot * kTile16;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
-        mma_ss(tSA, dqa + off, dk + off, id_s, kk > 0);
-      }
-      mma_commit(&bars[B_SF + 0]);
-      if (has_b) {
-        if (t > 0) {
-          if (!mbar_wait(&bars[B_PF + 1], itb & 1, w)) return;
-          ++itb;
-          tc_fence_after();
-          const uint64_t dvp = dv0 + vprev * kTile16;
-          for (int kk = 0; kk < nk_prev; ++kk) mma_ts(tOB, tSB + kk * 8, dvp + kk * 128, id_o, (t > 1 || kk > 0));
-          mma_commit(&bars[B_RE + vprev]);
-        }
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
-          mma_ss(tSB, dqb + off, dk + off, id_s, kk > 0);
+          mma_ss(tSA, dqa + off, dk + off, id_s, kk > 0);
         }
-        mma_commit(&bars[B_SF + 1]);
+        mma_commit(&bars[B_SF + 0]);
       }
-      mma_commit(&bars[B_RE + kslot]);
+      __syncwarp();
+      if (has_b) {
+        if (t > 0) {
+          if (!warp_wait(&bars[B_PF + 1], itb & 1, w)) return;
+          ++itb;
+          tc_fence_after();
+          const uint64_t dvp = dv0 + vprev * kTile16;
+          if (leader) {
+            for (int kk = 0; kk < nk_prev; ++kk) mma_ts(tOB, tSB + kk * 8, dvp + kk * 128, id_o, (t > 1 || kk > 0));
+            mma_commit(&bars[B_RE + vprev]);
+          }
+          __syncwarp();
+        }
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
+            mma_ss(tSB, dqb + off, dk + off, id_s, kk > 0);
+          }
+          mma_commit(&bars[B_SF + 1]);
+        }
+        __syncwarp();
+      }
+      if (leader) mma_commit(&bars[B_RE + kslot]);
+      __syncwarp();
       // V_j
       const uint32_t vslot = ring & (kRing - 1);
-      if (!mbar_wait(&bars[B_RF + vslot], (ring / kRing) & 1, w)) return;
+      if (!warp_wait(&bars[B_RF + vslot], (ring / kRing) & 1, w)) return;
       ++ring;
-      if (!mbar_wait(&bars[B_PF + 0], ita & 1, w)) return;
+      if (!warp_wait(&bars[B_PF + 0], ita & 1, w)) return;
       ++ita;
       tc_fence_after();
       const uint64_t dvv = dv0 + vslot * kTile16;
-      for (int kk = 0; kk < nk; ++kk) mma_ts(tOA, tSA + kk * 8, dvv + kk * 128, id_o, (t > 0 || kk > 0));
-      if (!has_b) mma_commit(&bars[B_RE + vslot]);
+      if (leader) {
+        for (int kk = 0; kk < nk; ++kk) mma_ts(tOA, tSA + kk * 8, dvv + kk * 128, id_o, (t > 0 || kk > 0));
+        if (!has_b) mma_commit(&bars[B_RE + vslot]);
+      }
+      __syncwarp();
       vprev = vslot;
       nk_prev = nk;
     }
     if (has_b && n > 0) {
-      if (!mbar_wait(&bars[B_PF + 1], itb & 1, w)) return;
+      if (!warp_wait(&bars[B_PF + 1], itb & 1, w)) return;
       ++itb;
       tc_fence_after();
       const uint64_t dvp = dv0 + vprev * kTile16;
-      for (int kk = 0; kk < nk_prev; ++kk) mma_ts(tOB, tSB + kk * 8, dvp + kk * 128, id_o, (n > 1 || kk > 0));
-      mma_commit(&bars[B_RE + vprev]);
+      if (leader) {
+        for (int kk = 0; kk < nk_prev; ++kk) mma_ts(tOB, tSB + kk * 8, dvp + kk * 128, id_o, (n > 1 || kk > 0));
+        mma_commit(&bars[B_RE + vprev]);
+      }
+      __syncwarp();
     }
     if (s.j0 == 0 && p.has_inter) {  // X = Q MqT^T for the rows this CTA finishes
       const uint32_t mslot = ring & (kRing - 1);
-      if (!mbar_wait(&bars[B_RF + mslot], (ring / kRing) & 1, w)) return;
+      if (!warp_wait(&bars[B_RF + mslot], (ring / kRing) & 1, w)) return;
       ++ring;
       tc_fence_after();
       const uint64_t dm = dr0 + mslot * kTile16;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
-        mma_ss(tSA, dqa + off, dm + off, id_x, kk > 0);
-      }
-      if (has_b) {
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
-          mma_ss(tSB, dqb + off, dm + off, id_x, kk > 0);
+          mma_ss(tSA, dqa + off, dm + off, id_x, kk > 0);
         }
+        if (has_b) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalf16 + (kk & 3) * 2;
+            mma_ss(tSB, dqb + off, dm + off, id_x, kk > 0);
+          }
+        }
+        mma_commit(&bars[B_RE + mslot]);
       }
-      mma_commit(&bars[B_RE + mslot]);
+      __syncwarp();
     }
-    mma_commit(&bars[B_SD + 0]);
-    mma_commit(&bars[B_QE + 0]);
+    if (leader) {
+      mma_commit(&bars[B_SD + 0]);
+      mma_commit(&bars[B_QE + 0]);
+      if (has_b) {
+        mma_commit(&bars[B_SD + 1]);
+        mma_commit(&bars[B_QE + 1]);
+      }
+    }
+    __syncwarp();
     ++sega;
-    if (has_b) {
-      mma_commit(&bars[B_SD + 1]);
-      mma_commit(&bars[B_QE + 1]);
-      ++segb;
-    }
+    if (has_b) ++segb;
   }
 }
 
@@ -407,11 +432,15 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (warp < 4) {
     regs_dec<kCtlRegs>();
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- producer
-      tma_prefetch(&tm_q);
-      tma_prefetch(&tm_k);
-      tma_prefetch(&tm_v);
+    {
+      // ---------------------------------------------------------------- producer (whole warp,
+      // the elected lane issues the copies)
+      const bool leader = elect_one();
+      if (leader) {
+        tma_prefetch(&tm_q);
+        tma_prefetch(&tm_k);
+        tma_prefetch(&tm_v);
+      }
       uint32_t ring = 0, qa_use = 0, qb_use = 0;
       bool ok = true;
       unsigned u = u_begin;
@@ -426,18 +455,21 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int x0 = h * 128;
         auto put = [&](int t) -> bool {
           const uint32_t slot = ring % kRing;
-          if (ring >= kRing && !mbar_wait(&bars[B_RE + slot], ((ring / kRing) - 1) & 1, w)) return false;
+          if (ring >= kRing && !warp_wait(&bars[B_RE + slot], ((ring / kRing) - 1) & 1, w)) return false;
           uint8_t* dst = sR + slot * kTile;
-          mbar_expect_tx(&bars[B_RF + slot], kTile);
-          if (t < 2 * n) {
-            const int j = s.j0 + (t >> 1);
-            const CUtensorMap* m = (t & 1) ? &tm_v : &tm_k;
-            tma_load_3d(dst, m, &bars[B_RF + slot], x0, j * 128, b);
-            tma_load_3d(dst + kHalf, m, &bars[B_RF + slot], x0 + 64, j * 128, b);
-          } else {
-            tma_load_3d(dst, &tm_mq, &bars[B_RF + slot], 0, 0, s.bh);
-            tma_load_3d(dst + kHalf, &tm_mq, &bars[B_RF + slot], 64, 0, s.bh);
+          if (leader) {
+            mbar_expect_tx(&bars[B_RF + slot], kTile);
+            if (t < 2 * n) {
+              const int j = s.j0 + (t >> 1);
+              const CUtensorMap* m = (t & 1) ? &tm_v : &tm_k;
+              tma_load_3d(dst, m, &bars[B_RF + slot], x0, j * 128, b);
+              tma_load_3d(dst + kHalf, m, &bars[B_RF + slot], x0 + 64, j * 128, b);
+            } else {
+              tma_load_3d(dst, &tm_mq, &bars[B_RF + slot], 0, 0, s.bh);
+              tma_load_3d(dst + kHalf, &tm_mq, &bars[B_RF + slot], 64, 0, s.bh);
+            }
           }
+          __syncwarp();
           ++ring;
           return true;
         };
@@ -445,22 +477,23 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int t = 0; ok && t < pre; ++t) ok = put(t);
         for (int sub = 0; ok && sub < (has_b ? 2 : 1); ++sub) {
           const uint32_t used = sub ? qb_use : qa_use;
-          if (used > 0 && !(ok = mbar_wait(&bars[B_QE + sub], (used - 1) & 1, w))) break;
-          mbar_expect_tx(&bars[B_QF + sub], kTile);
+          if (used > 0 && !(ok = warp_wait(&bars[B_QE + sub], (used - 1) & 1, w))) break;
           uint8_t* dst = sQ + sub * kTile;
           const int row = (qt_a + sub) * 128;
-          tma_load_3d(dst, &tm_q, &bars[B_QF + sub], x0, row, b);
-          tma_load_3d(dst + kHalf, &tm_q, &bars[B_QF + sub], x0 + 64, row, b);
+          if (leader) {
+            mbar_expect_tx(&bars[B_QF + sub], kTile);
+            tma_load_3d(dst, &tm_q, &bars[B_QF + sub], x0, row, b);
+            tma_load_3d(dst + kHalf, &tm_q, &bars[B_QF + sub], x0 + 64, row, b);
+          }
+          __syncwarp();
           if (sub) ++qb_use; else ++qa_use;
         }
         for (int t = pre; ok && t < ntiles; ++t) ok = put(t);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-      mma_issuer(p, bars, tmem, smem_u32(sQ), smem_u32(sR), u_begin, u_end, w);
-    }
+    // ---------------------------------------------------------------- MMA issuer (whole warp)
+    mma_issuer(p, bars, tmem, smem_u32(sQ), smem_u32(sR), u_begin, u_end, w);
   }
   } else {
     regs_inc<kSoftmaxRegs>();
