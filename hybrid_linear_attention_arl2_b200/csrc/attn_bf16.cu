@@ -44,8 +44,11 @@ constexpr int kAttnThreads = 384;
 constexpr int kRing = 4;
 constexpr uint32_t kTile = 32768;  // 128 rows x 128 bf16
 constexpr uint32_t kHalf = 16384;  // one 64-column box
-constexpr int kAttnSmem = (2 + kRing) * kTile + 512 + 1024;
+constexpr int kAttnSmem = (2 + kRing) * kTile + 32768 + 512 + 1024;
 constexpr int kSlotFloats = kAttnSlotFloats;
+constexpr int kSlotStats = 128 * 64;  // floats before (m, l) in a slot: 128 x 128 bf16 partial O
+constexpr int kMaxContrib = 8;        // partials a finishing CTA may combine
+constexpr uint32_t kStageBytes = 8 * 4096;  // per softmax warp: 32 rows x 128 B of output
 // Register split: the launch gives every thread kLaunchRegs; warpgroup 0
 // (producer, MMA issuer, allocator) drops to kCtlRegs and the two softmax
 // warpgroups rise to kSoftmaxRegs.  128 * kCtlRegs + 256 * kSoftmaxRegs must
@@ -108,9 +111,37 @@ __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Stages 32 rows x 64 columns (bf16, one 128-byte half row per lane) through
+// this warp's 4 KB of shared memory and writes them out four rows per store
+// instruction (whole 128-byte row segments: coalesced).
+__device__ __forceinline__ void store_rows_half(const AttnParams& p, uint8_t* stage, const int lane, const int b,
+                                                const int h, const int row0, const int half, const uint32_t (&pk)[32]) {
+  // write: chunk c of this lane's row at 16-byte column c ^ (lane & 7) (bank-conflict free)
+  uint4* st = reinterpret_cast<uint4*>(stage);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    st[lane * 8 + (c ^ (lane & 7))] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = 4 * it + (lane >> 3), c = lane & 7;
+    const uint4 v = st[r * 8 + (c ^ (r & 7))];
+    const int q_row = row0 + r;
+    if (q_row < p.q_len) {
+      __nv_bfloat16* dst = p.o + ((size_t(b) * p.q_len + q_row) * p.heads + h) * 128 + half * 64 + c * 8;
+      *reinterpret_cast<uint4*>(dst) = v;
+    }
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
 // End of one segment for one sub-tile (a warpgroup, one row per thread).
 //  * a segment that does not start at key tile 0 stores its unnormalised O
-//    rows and (m, l) to this CTA's slot and raises the slot's ready flag;
+//    rows (bf16, chunk-major) and (m, l) to this CTA's slot and raises the
+//    slot's ready flag;
 //  * a segment that starts at key tile 0 writes the final rows: its own
 //    accumulator, combined with the partials of the CTAs that hold the rest of
 //    the block's keys (in key order), normalised, plus the read-out X.
@@ -120,12 +151,11 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
                                               const int sub, const int lane, const int row, const uint32_t lane_off,
                                               const uint32_t tS, const uint32_t tO, const bool warp_on,
                                               const bool row_ok, const int q_row, const float m, const float l,
-                                              uint64_t* ed_bar, volatile int* abort_flag) {
+                                              uint64_t* ed_bar, volatile int* abort_flag, uint8_t* stage) {
   const int wg_thread = threadIdx.x - 128 - sub * 128;  // 0..127 within the warpgroup
   const bool writer = s.j0 == 0, full = writer && s.j1 == p.nkv;
   const bool use_intra = !(p.flags & 2u);
   const bool use_inter = p.has_inter && !(p.flags & 1u);
-  bool ok = true;
   if (!writer) {
     float* slot = p.scratch + (size_t(cta) * 2 + sub) * kSlotFloats;
     if (warp_on) {
@@ -134,13 +164,18 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
       for (int c = 0; c < 4; ++c) tmem_ld32(tO + lane_off + c * 32, slice32(r, c));
       tmem_wait_ld();
       if (row_ok) {
-        float4* d4 = reinterpret_cast<float4*>(slot + row * 128);
+        // bf16, chunk-major: 16-byte chunk i of row r at uint4 index i * 128 + r, so the
+        // 32 rows of a warp write one contiguous 512-byte span per instruction
+        uint4* d4 = reinterpret_cast<uint4*>(slot) + row;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
-                              __uint_as_float(r[4 * i + 3]));
-        slot[16384 + row] = m;
-        slot[16384 + 128 + row] = l;
+        for (int i = 0; i < 16; ++i)
+          d4[i * 128] = make_uint4(
+              pack_bf16x2(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+              pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+              pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+              pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+        slot[kSlotStats + row] = m;
+        slot[kSlotStats + 128 + row] = l;
       }
     }
     tc_fence_before();
@@ -151,11 +186,12 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
     if (wg_thread == 0) st_release(p.ready + cta * 2 + sub, 1u);
     return true;
   }
-  int contrib[8];
+  int contrib[kMaxContrib];
   int n_contrib = 0;
+  bool ok = true;
   if (!full) {
     bool complete = false;
-    for (int c2 = cta + 1; c2 < p.grid && n_contrib < 8; ++c2) {
+    for (int c2 = cta + 1; c2 < p.grid && n_contrib < kMaxContrib; ++c2) {
       const unsigned a0 = p.range[c2], a1 = p.range[c2 + 1];
       if (a0 == a1) continue;
       unsigned uu = a0;
@@ -168,7 +204,7 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
         break;
       }
     }
-    if (!complete) {  // the host partition bounds a block to 8 pieces; never expected
+    if (!complete) {  // the host partition bounds a block to kMaxContrib + 1 pieces; never expected
       record_error(p.err, kDevBadShape);
       *abort_flag = 1;
     }
@@ -182,7 +218,6 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
             record_error(p.err, kDevTimeout);
             break;
           }
-          __nanosleep(64);
         }
       }
     }
@@ -191,66 +226,91 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
     if (ok)
       for (int k = 0; k < n_contrib; ++k) (void)ld_acquire(p.ready + contrib[k] * 2 + sub);
   }
-  float M = m, inv_l = 0.f;
-  if (ok && row_ok) {
-    for (int k = 0; k < n_contrib; ++k)
-      M = fmaxf(M, p.scratch[(size_t(contrib[k]) * 2 + sub) * kSlotFloats + 16384 + row]);
-    float Lsum = l * fast_exp2(m - M);
-    for (int k = 0; k < n_contrib; ++k) {
+  // combined statistics: all contributors' (m, l) loaded in one batch
+  float M = m, a_self = 0.f;
+  float mk[kMaxContrib], lk[kMaxContrib];
+#pragma unroll
+  for (int k = 0; k < kMaxContrib; ++k) {
+    mk[k] = -INFINITY;
+    lk[k] = 0.f;
+    if (ok && row_ok && k < n_contrib) {
       const float* sl = p.scratch + (size_t(contrib[k]) * 2 + sub) * kSlotFloats;
-      Lsum = fmaf(sl[16384 + 128 + row], fast_exp2(sl[16384 + row] - M), Lsum);
+      mk[k] = sl[kSlotStats + row];
+      lk[k] = sl[kSlotStats + 128 + row];
     }
-    inv_l = 1.f / Lsum;
   }
-  const float a_self = fast_exp2(m - M) * inv_l;
+  if (ok && row_ok) {
+#pragma unroll
+    for (int k = 0; k < kMaxContrib; ++k) M = fmaxf(M, mk[k]);
+    float Lsum = l * fast_exp2(m - M);
+#pragma unroll
+    for (int k = 0; k < kMaxContrib; ++k) {
+      mk[k] = fast_exp2(mk[k] - M);  // now the contributor's weight
+      Lsum = fmaf(lk[k], mk[k], Lsum);
+    }
+    const float inv_l = 1.f / Lsum;
+    a_self = fast_exp2(m - M) * inv_l;
+#pragma unroll
+    for (int k = 0; k < kMaxContrib; ++k) mk[k] *= inv_l;
+  }
   if (ok && warp_on) {
     const int b = s.bh / p.heads, h = s.bh % p.heads;
-    __nv_bfloat16* dst = p.o + ((size_t(b) * p.q_len + q_row) * p.heads + h) * 128;
+    const int row0 = (q_row - row) + (row & ~31);  // first query row of this warp
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t ro[32], rx[32];
-      tmem_ld32(tO + lane_off + c * 32, ro);
-      if (p.has_inter) tmem_ld32(tS + lane_off + c * 32, rx);
-      tmem_wait_ld();
-      if (row_ok) {
+    for (int half = 0; half < 2; ++half) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int col = half * 64 + qq * 32;
+        uint32_t ro[32], rx[32];
+        tmem_ld32(tO + lane_off + col, ro);
+        if (p.has_inter) tmem_ld32(tS + lane_off + col, rx);
+        tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * a_self);
-        for (int k = 0; k < n_contrib; ++k) {
-          const float* sl = p.scratch + (size_t(contrib[k]) * 2 + sub) * kSlotFloats;
-          const float a = fast_exp2(sl[16384 + row] - M) * inv_l;
-          const float4* s4 = reinterpret_cast<const float4*>(sl + row * 128 + c * 32);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 x = s4[i];
-            ro[4 * i] = __float_as_uint(fmaf(x.x, a, __uint_as_float(ro[4 * i])));
-            ro[4 * i + 1] = __float_as_uint(fmaf(x.y, a, __uint_as_float(ro[4 * i + 1])));
-            ro[4 * i + 2] = __float_as_uint(fmaf(x.z, a, __uint_as_float(ro[4 * i + 2])));
-            ro[4 * i + 3] = __float_as_uint(fmaf(x.w, a, __uint_as_float(ro[4 * i + 3])));
+        for (int k = 0; k < kMaxContrib; ++k) {
+          if (row_ok && k < n_contrib) {
+            const uint4* s4 = reinterpret_cast<const uint4*>(p.scratch + (size_t(contrib[k]) * 2 + sub) * kSlotFloats) +
+                              (col / 8) * 128 + row;
+            uint4 x[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) x[i] = s4[i * 128];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t w4[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                ro[8 * i + 2 * e] = __float_as_uint(fmaf(bf16_lo(w4[e]), mk[k], __uint_as_float(ro[8 * i + 2 * e])));
+                ro[8 * i + 2 * e + 1] =
+                    __float_as_uint(fmaf(bf16_hi(w4[e]), mk[k], __uint_as_float(ro[8 * i + 2 * e + 1])));
+              }
+            }
           }
         }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t q[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 8 * g + 2 * e;
-            float v0 = use_intra ? __uint_as_float(ro[i]) : 0.f;
-            float v1 = use_intra ? __uint_as_float(ro[i + 1]) : 0.f;
-            if (use_inter) {
-              v0 += __uint_as_float(rx[i]);
-              v1 += __uint_as_float(rx[i + 1]);
-            }
-            q[e] = pack_bf16x2(v0, v1);
+        for (int i = 0; i < 16; ++i) {
+          float v0 = use_intra ? __uint_as_float(ro[2 * i]) : 0.f;
+          float v1 = use_intra ? __uint_as_float(ro[2 * i + 1]) : 0.f;
+          if (use_inter) {
+            v0 += __uint_as_float(rx[2 * i]);
+            v1 += __uint_as_float(rx[2 * i + 1]);
           }
-          d4[g] = make_uint4(q[0], q[1], q[2], q[3]);
+          pk[qq * 16 + i] = pack_bf16x2(v0, v1);
         }
       }
+      if (half == 1) {  // every tensor-memory read of this segment is done
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ed_bar);
+      }
+      store_rows_half(p, stage, lane, b, h, row0, half, pk);
     }
+  } else {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(ed_bar);
   }
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive(ed_bar);
   if (!full) {
     named_bar(1 + sub, 128);  // every row has read the partials
     if (wg_thread == 0)
@@ -410,7 +470,8 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                   // [2] sub-tiles
   uint8_t* sR = smem + 2 * kTile;       // [kRing] K / V / MqT tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (2 + kRing) * kTile);
+  uint8_t* sStage = smem + (2 + kRing) * kTile;  // [8 softmax warps][4 KB] output staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (2 + kRing) * kTile + kStageBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -626,7 +687,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       ++segs_done;
       tc_fence_after();
       if (!segment_epilogue(p, s, cta, sub, lane, row, lane_off, tS, tO, warp_on, row_ok, q_row, m, l,
-                            &bars[B_ED + sub], abort_flag))
+                            &bars[B_ED + sub], abort_flag, sStage + (warp - 4) * 4096))
         ok = false;
     }
   }

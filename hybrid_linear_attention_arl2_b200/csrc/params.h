@@ -28,14 +28,16 @@ struct AttnParams {
   float scale_log2;     // softmax scale * log2(e)
   uint32_t flags;       // 1: intra only, 2: inter only
   int has_inter;        // 1: add Q MqT^T
-  float* scratch;       // [grid][2][kAttnSlotFloats] partial rows and (m, l)
+  float* scratch;       // [grid][2][kAttnSlotFloats] partial O (bf16, chunk-major) and (m, l)
   unsigned* ready;      // [grid][2] partial-ready flags, zero between launches
   uint32_t* err;        // device error word
   uint64_t wait_limit_ns;
 };
 
-// floats of one partial slot (one sub-tile of one CTA): 128 x 128 O rows, m[128], l[128]
-constexpr int kAttnSlotFloats = 128 * 128 + 256;
+// floats of one partial slot (one sub-tile of one CTA): 128 x 128 unnormalised O
+// values in bf16, stored chunk-major (16-byte chunk i of row r at byte (i * 128 + r) * 16),
+// then m[128] and l[128] in fp32
+constexpr int kAttnSlotFloats = 128 * 64 + 256;
 
 // State write and read-out preparation (state_bf16.cu).
 struct StateParams {
