@@ -54,7 +54,7 @@ constexpr uint32_t kStageBytes = 8 * 4096;  // per softmax warp: 32 rows x 128 B
 // warpgroups rise to kSoftmaxRegs.  128 * kCtlRegs + 256 * kSoftmaxRegs must
 // not exceed 384 * kLaunchRegs, or setmaxnreg.inc would wait forever; the
 // launcher refuses to run unless the compiled kernel has exactly kLaunchRegs.
-constexpr int kPolyPairs = 6;  // of every 16 exp2 pairs of a full tile, this many run on the FMA pipe
+constexpr int kPolyPairs = 5;  // of every 16 exp2 pairs of a full tile, this many run on the FMA pipe
 constexpr int kLaunchRegs = 168;
 constexpr int kCtlRegs = 72;
 constexpr int kSoftmaxRegs = 216;
@@ -186,19 +186,22 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
     if (wg_thread == 0) st_release(p.ready + cta * 2 + sub, 1u);
     return true;
   }
-  int contrib[kMaxContrib];
+  // Contributors: the CTAs after this one whose first segment continues this
+  // block (empty ranges skipped), as a bit mask over cta + 1 + i.
+  uint32_t cmask = 0;
   int n_contrib = 0;
   bool ok = true;
   if (!full) {
     bool complete = false;
-    for (int c2 = cta + 1; c2 < p.grid && n_contrib < kMaxContrib; ++c2) {
+    for (int c2 = cta + 1; c2 < p.grid && c2 <= cta + 32 && n_contrib < kMaxContrib; ++c2) {
       const unsigned a0 = p.range[c2], a1 = p.range[c2 + 1];
       if (a0 == a1) continue;
       unsigned uu = a0;
       Seg s2;
       next_seg(p, uu, a1, s2);
       if (s2.bh != s.bh || s2.blk != s.blk) break;
-      contrib[n_contrib++] = c2;
+      cmask |= 1u << (c2 - cta - 1);
+      ++n_contrib;
       if (s2.j1 == p.nkv) {
         complete = true;
         break;
@@ -209,8 +212,8 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
       *abort_flag = 1;
     }
     if (wg_thread == 0) {  // wait until every contributor's partial is visible
-      for (int k = 0; k < n_contrib && !*abort_flag; ++k) {
-        const unsigned* f = p.ready + contrib[k] * 2 + sub;
+      for (uint32_t mm = cmask; mm && !*abort_flag; mm &= mm - 1) {
+        const unsigned* f = p.ready + (cta + 1 + __ffs(mm) - 1) * 2 + sub;
         const uint64_t t0 = global_timer_ns();
         while (ld_acquire(f) == 0u) {
           if (*abort_flag || global_timer_ns() - t0 > p.wait_limit_ns) {
@@ -221,12 +224,17 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
         }
       }
     }
+    // thread 0's acquire and this barrier order every thread's reads of the partials
     named_bar(1 + sub, 128);
     ok = !*abort_flag;
-    if (ok)
-      for (int k = 0; k < n_contrib; ++k) (void)ld_acquire(p.ready + contrib[k] * 2 + sub);
   }
-  // combined statistics: all contributors' (m, l) loaded in one batch
+  // slot of the k-th contributor (k < n_contrib)
+  auto slot_of = [&](int k) -> const float* {
+    uint32_t mm = cmask;
+    for (int i = 0; i < k; ++i) mm &= mm - 1;
+    return p.scratch + (size_t(cta + __ffs(mm)) * 2 + sub) * kSlotFloats;
+  };
+  // combined statistics, all contributors' (m, l) loaded in one batch
   float M = m, a_self = 0.f;
   float mk[kMaxContrib], lk[kMaxContrib];
 #pragma unroll
@@ -234,7 +242,7 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
     mk[k] = -INFINITY;
     lk[k] = 0.f;
     if (ok && row_ok && k < n_contrib) {
-      const float* sl = p.scratch + (size_t(contrib[k]) * 2 + sub) * kSlotFloats;
+      const float* sl = slot_of(k);
       mk[k] = sl[kSlotStats + row];
       lk[k] = sl[kSlotStats + 128 + row];
     }
@@ -258,6 +266,13 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
     const int row0 = (q_row - row) + (row & ~31);  // first query row of this warp
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
+      // this half row of the first contributor, fetched before the tensor-memory reads
+      uint4 xh[8];
+      if (row_ok && n_contrib > 0) {
+        const uint4* s4 = reinterpret_cast<const uint4*>(slot_of(0)) + half * 8 * 128 + row;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xh[i] = s4[i * 128];
+      }
       uint32_t pk[32];
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
@@ -271,11 +286,15 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
 #pragma unroll
         for (int k = 0; k < kMaxContrib; ++k) {
           if (row_ok && k < n_contrib) {
-            const uint4* s4 = reinterpret_cast<const uint4*>(p.scratch + (size_t(contrib[k]) * 2 + sub) * kSlotFloats) +
-                              (col / 8) * 128 + row;
             uint4 x[4];
+            if (k == 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) x[i] = s4[i * 128];
+              for (int i = 0; i < 4; ++i) x[i] = xh[qq * 4 + i];
+            } else {
+              const uint4* s4 = reinterpret_cast<const uint4*>(slot_of(k)) + (col / 8) * 128 + row;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) x[i] = s4[i * 128];
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const uint32_t w4[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
@@ -314,7 +333,7 @@ __device__ __forceinline__ bool segment_epilogue(const AttnParams& p, const Seg 
   if (!full) {
     named_bar(1 + sub, 128);  // every row has read the partials
     if (wg_thread == 0)
-      for (int k = 0; k < n_contrib; ++k) p.ready[contrib[k] * 2 + sub] = 0u;
+      for (uint32_t mm = cmask; mm; mm &= mm - 1) p.ready[(cta + __ffs(mm)) * 2 + sub] = 0u;
   }
   return ok;
 }
@@ -595,16 +614,16 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int i = 0; i < 128; ++i)
               if (i >= valid) r[i] = __float_as_uint(-INFINITY);
           }
-          float m4[4] = {__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]),
-                         __uint_as_float(r[3])};
+          // row max: a two-input max tree over 8 independent chains
+          float m8[8];
 #pragma unroll
-          for (int i = 4; i < 128; i += 8) {
-            m4[0] = fmax3(m4[0], __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-            m4[1] = fmax3(m4[1], __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-            m4[2] = fmax3(m4[2], __uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
-            m4[3] = fmax3(m4[3], __uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
-          }
-          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+          for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(r[k]);
+#pragma unroll
+          for (int i = 8; i < 128; i += 8)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], __uint_as_float(r[i + k]));
+          const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
           // Lazy rescaling: the running max moves only when it grows by more
           // than 8 (a factor 256), so P stays <= 256 and O is touched rarely.
           // O is rescaled after P is written (the S row is dead by then) and
@@ -626,23 +645,25 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           // exp2 so that the MUFU is not the limit; the masked last tile (columns
           // at -inf) takes the MUFU for all of them.
           const float nm = -m;
-          float l0 = 0.f, l1 = 0.f;
+          float l4[4] = {0.f, 0.f, 0.f, 0.f};
           if (valid == 128) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint32_t pk[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                float x0, x1, p0, p1;
-                ffma2(x0, x1, __uint_as_float(r[c * 32 + 2 * i]), __uint_as_float(r[c * 32 + 2 * i + 1]), sl2, sl2,
-                      nm, nm);
-                if (i >= 16 - kPolyPairs) {
-                  exp2_poly2(p0, p1, x0, x1);
+                const float x0 = fmaf(__uint_as_float(r[c * 32 + 2 * i]), sl2, nm);
+                const float x1 = fmaf(__uint_as_float(r[c * 32 + 2 * i + 1]), sl2, nm);
+                float p0, p1;
+                if (i >= 16 - kPolyPairs) {  // x <= 8 here: the lazy max is at most 8 below the row max
+                  p0 = exp2_poly(x0);
+                  p1 = exp2_poly(x1);
                 } else {
                   p0 = fast_exp2(x0);
                   p1 = fast_exp2(x1);
                 }
-                fadd2(l0, l1, l0, l1, p0, p1);
+                l4[(2 * i) & 3] += p0;
+                l4[(2 * i + 1) & 3] += p1;
                 pk[i] = pack_bf16x2(p0, p1);
               }
               tmem_st16(tS + lane_off + c * 16, pk);
@@ -653,17 +674,16 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               uint32_t pk[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                float x0, x1;
-                ffma2(x0, x1, __uint_as_float(r[c * 32 + 2 * i]), __uint_as_float(r[c * 32 + 2 * i + 1]), sl2, sl2,
-                      nm, nm);
-                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-                fadd2(l0, l1, l0, l1, p0, p1);
+                const float p0 = fast_exp2(fmaf(__uint_as_float(r[c * 32 + 2 * i]), sl2, nm));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(r[c * 32 + 2 * i + 1]), sl2, nm));
+                l4[(2 * i) & 3] += p0;
+                l4[(2 * i + 1) & 3] += p1;
                 pk[i] = pack_bf16x2(p0, p1);
               }
               tmem_st16(tS + lane_off + c * 16, pk);
             }
           }
-          l = fmaf(l, f, l0 + l1);
+          l = fmaf(l, f, (l4[0] + l4[1]) + (l4[2] + l4[3]));
           if (any_rescale) {
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {

@@ -264,28 +264,28 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 2^x0, 2^x1 on the FMA pipe (leaves the MUFU free for the other lanes of the
+// 2^x on the FMA pipe (leaves the MUFU free for the other columns of the
 // softmax).  x = n + f with n = round(x) and f in [-1/2, 1/2]: adding 1.5 * 2^23
 // rounds x to an integer held in the low mantissa bits; 2^f is the degree-3
 // polynomial interpolating 2^f at the four Chebyshev nodes of [-1/2, 1/2]
 // (coefficients from gen_exp2_poly.py, max relative error 1.0e-4, below the
 // 2^-9 of the bf16 P it feeds); 2^n is added to the exponent field with one
-// integer multiply-add.  x is clamped to [-125, 125] (results stay normal).
-__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+// shift-add.  x is clamped below at -125 (results stay normal); callers keep
+// x <= 125.
+__device__ __forceinline__ float exp2_poly(float x) {
   constexpr float kRound = 12582912.f;  // 1.5 * 2^23
   constexpr float c0 = 0.999924541f, c1 = 0.693136752f, c2 = 0.242639482f, c3 = 0.0558382832f;
-  x0 = fminf(fmaxf(x0, -125.f), 125.f);
-  x1 = fminf(fmaxf(x1, -125.f), 125.f);
-  float t0, t1, r0, r1, f0, f1, p0, p1;
-  fadd2(t0, t1, x0, x1, kRound, kRound);      // round(x) in the low mantissa bits of t
-  fadd2(r0, r1, t0, t1, -kRound, -kRound);    // round(x) as a float
-  ffma2(f0, f1, r0, r1, -1.f, -1.f, x0, x1);  // f = x - round(x)
-  ffma2(p0, p1, f0, f1, c3, c3, c2, c2);
-  ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
-  ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
+  x = fmaxf(x, -125.f);
+  const float t = x + kRound;       // round(x) in the low mantissa bits of t
+  const float f = x - (t - kRound);  // x - round(x)
+  const float pf = fmaf(fmaf(fmaf(c3, f, c2), f, c1), f, c0);
   // exponent field += round(x): (bits(t) << 23) is round(x) << 23 modulo 2^32
-  y0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(p0));
-  y1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1));
+  return __uint_as_float((__float_as_uint(t) << 23) + __float_as_uint(pf));
+}
+
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  y0 = exp2_poly(fminf(x0, 125.f));
+  y1 = exp2_poly(fminf(x1, 125.f));
 }
 
 // A 32-column slice of a 128-column register row, for the tcgen05.ld/st helpers.
