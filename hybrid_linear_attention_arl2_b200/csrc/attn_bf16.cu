@@ -69,7 +69,8 @@ enum {
   B_PF = B_SF + 2,                // [2]
   B_SD = B_PF + 2,                // [2] segment done: every MMA of the segment completed
   B_ED = B_SD + 2,                // [2]
-  B_DRAIN = B_ED + 2,
+  B_TURN = B_ED + 2,              // [2] exponential-section turn of sub-tile A / B
+  B_DRAIN = B_TURN + 2,
   B_COUNT
 };
 
@@ -499,7 +500,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const unsigned u_begin = p.range[cta], u_end = p.range[cta + 1];
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], (i == B_PF || i == B_PF + 1 || i == B_ED || i == B_ED + 1) ? 4u : 1u);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(&bars[i], (i == B_PF || i == B_PF + 1 || i == B_ED || i == B_ED + 1 || i == B_TURN || i == B_TURN + 1) ? 4u : 1u);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -584,7 +585,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t tS = tmem + sub * 128, tO = tmem + 256 + sub * 128;
     const float sl2 = p.scale_log2;
-    uint32_t it = 0, segs_done = 0;
+    uint32_t it = 0, segs_done = 0, turns = 0;
     bool ok = true;
     unsigned u = u_begin;
     Seg s;
@@ -601,9 +602,14 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int t = 0; t < s.j1 - s.j0; ++t) {
         if (!(ok = warp_wait(&bars[B_SF + sub], it & 1, w))) break;
         tc_fence_after();
+        const int j = s.j0 + t;
+        const int valid = min(128, p.kv_len - j * 128);
+        // The two warpgroups take turns for the exponentials (when the block
+        // has both sub-tiles), so each runs its section with the SMSPs' issue
+        // slots and MUFU to itself.
+        const bool take_turn = has_b && !(sub == 0 && turns == 0);
+        const uint32_t turn_parity = sub == 0 ? (turns - 1) & 1 : turns & 1;
         if (warp_on) {
-          const int j = s.j0 + t;
-          const int valid = min(128, p.kv_len - j * 128);
           // the whole 128-column row of S in one round trip
           uint32_t r[128];
 #pragma unroll
@@ -626,8 +632,6 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                  fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
           // Lazy rescaling: the running max moves only when it grows by more
           // than 8 (a factor 256), so P stays <= 256 and O is touched rarely.
-          // O is rescaled after P is written (the S row is dead by then) and
-          // before P is signalled, so PV always sees a consistent O.
           float f = 1.f;
           bool any_rescale = false;
           if (t == 0) {
@@ -640,51 +644,41 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               m = mx;
             }
           }
+          if (take_turn && !(ok = warp_wait(&bars[B_TURN + sub], turn_parity, w))) break;
           // P = exp2(S * scale * log2(e) - m), packed to bf16 pairs over S's first 64
           // columns.  On full tiles kPolyPairs of every 16 pairs take the FMA-pipe
           // exp2 so that the MUFU is not the limit; the masked last tile (columns
           // at -inf) takes the MUFU for all of them.
           const float nm = -m;
-          float l4[4] = {0.f, 0.f, 0.f, 0.f};
-          if (valid == 128) {
+          float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t pk[16];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float x0 = fmaf(__uint_as_float(r[c * 32 + 2 * i]), sl2, nm);
-                const float x1 = fmaf(__uint_as_float(r[c * 32 + 2 * i + 1]), sl2, nm);
-                float p0, p1;
-                if (i >= 16 - kPolyPairs) {  // x <= 8 here: the lazy max is at most 8 below the row max
-                  p0 = exp2_poly(x0);
-                  p1 = exp2_poly(x1);
-                } else {
-                  p0 = fast_exp2(x0);
-                  p1 = fast_exp2(x1);
-                }
-                l4[(2 * i) & 3] += p0;
-                l4[(2 * i + 1) & 3] += p1;
-                pk[i] = pack_bf16x2(p0, p1);
+            for (int i = 0; i < 16; ++i) {
+              const float x0 = fmaf(__uint_as_float(r[c * 32 + 2 * i]), sl2, nm);
+              const float x1 = fmaf(__uint_as_float(r[c * 32 + 2 * i + 1]), sl2, nm);
+              float p0, p1;
+              if (valid == 128 && i >= 16 - kPolyPairs) {  // x <= 8: the lazy max is at most 8 below
+                p0 = exp2_poly(x0);
+                p1 = exp2_poly(x1);
+              } else {
+                p0 = fast_exp2(x0);
+                p1 = fast_exp2(x1);
               }
-              tmem_st16(tS + lane_off + c * 16, pk);
+              l8[(2 * i) & 7] += p0;
+              l8[(2 * i + 1) & 7] += p1;
+              pk[i] = pack_bf16x2(p0, p1);
             }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t pk[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float p0 = fast_exp2(fmaf(__uint_as_float(r[c * 32 + 2 * i]), sl2, nm));
-                const float p1 = fast_exp2(fmaf(__uint_as_float(r[c * 32 + 2 * i + 1]), sl2, nm));
-                l4[(2 * i) & 3] += p0;
-                l4[(2 * i + 1) & 3] += p1;
-                pk[i] = pack_bf16x2(p0, p1);
-              }
-              tmem_st16(tS + lane_off + c * 16, pk);
-            }
+            tmem_st16(tS + lane_off + c * 16, pk);
           }
-          l = fmaf(l, f, (l4[0] + l4[1]) + (l4[2] + l4[3]));
-          if (any_rescale) {
+          if (has_b) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_TURN + (sub ^ 1)]);
+          }
+          l = fmaf(l, f, ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7])));
+          tmem_wait_st();
+          if (any_rescale) {  // rare: O is rescaled before P is signalled, so PV sees a consistent O
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               uint32_t o[32];
@@ -694,9 +688,14 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
               tmem_st32(tO + lane_off + c * 32, o);
             }
+            tmem_wait_st();
           }
-          tmem_wait_st();
+        } else if (has_b) {  // a warp with no valid rows still passes the turn on
+          if (take_turn && !(ok = warp_wait(&bars[B_TURN + sub], turn_parity, w))) break;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[B_TURN + (sub ^ 1)]);
         }
+        if (has_b) ++turns;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[B_PF + sub]);
