@@ -651,26 +651,42 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           // at -inf) takes the MUFU for all of them.
           const float nm = -m;
           float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          if (valid == 128) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float x0 = fmaf(__uint_as_float(r[c * 32 + 2 * i]), sl2, nm);
-              const float x1 = fmaf(__uint_as_float(r[c * 32 + 2 * i + 1]), sl2, nm);
-              float p0, p1;
-              if (valid == 128 && i >= 16 - kPolyPairs) {  // x <= 8: the lazy max is at most 8 below
-                p0 = exp2_poly(x0);
-                p1 = exp2_poly(x1);
-              } else {
-                p0 = fast_exp2(x0);
-                p1 = fast_exp2(x1);
+              for (int i = 0; i < 16; ++i) {
+                const float x0 = fmaf(__uint_as_float(r[c * 32 + 2 * i]), sl2, nm);
+                const float x1 = fmaf(__uint_as_float(r[c * 32 + 2 * i + 1]), sl2, nm);
+                float p0, p1;
+                if (i >= 16 - kPolyPairs) {  // x <= 8: the lazy max is at most 8 below the row max
+                  p0 = exp2_poly(x0);
+                  p1 = exp2_poly(x1);
+                } else {
+                  p0 = fast_exp2(x0);
+                  p1 = fast_exp2(x1);
+                }
+                l8[(2 * i) & 7] += p0;
+                l8[(2 * i + 1) & 7] += p1;
+                pk[i] = pack_bf16x2(p0, p1);
               }
-              l8[(2 * i) & 7] += p0;
-              l8[(2 * i + 1) & 7] += p1;
-              pk[i] = pack_bf16x2(p0, p1);
+              tmem_st16(tS + lane_off + c * 16, pk);
             }
-            tmem_st16(tS + lane_off + c * 16, pk);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float p0 = fast_exp2(fmaf(__uint_as_float(r[c * 32 + 2 * i]), sl2, nm));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(r[c * 32 + 2 * i + 1]), sl2, nm));
+                l8[(2 * i) & 7] += p0;
+                l8[(2 * i + 1) & 7] += p1;
+                pk[i] = pack_bf16x2(p0, p1);
+              }
+              tmem_st16(tS + lane_off + c * 16, pk);
+            }
           }
           if (has_b) {
             __syncwarp();
