@@ -23,7 +23,9 @@ ARL2_INTRA_ONLY, ARL2_INTER_ONLY = 1, 2
 STATUS = {
     0: "ARL2_OK", 1: "ARL2_ERR_INVALID_ARGUMENT", 2: "ARL2_ERR_UNSUPPORTED",
     3: "ARL2_ERR_OUT_OF_MEMORY", 4: "ARL2_ERR_CUDA", 5: "ARL2_ERR_TIMEOUT", 6: "ARL2_ERR_NO_DEVICE",
+    7: "ARL2_ERR_SCRATCH_LIMIT",
 }
+ARL2_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class Arl2Error(RuntimeError):
@@ -58,6 +60,8 @@ _SIGS = {
     "arl2_kv_device_bytes": (_I64, [_VP]),
     "arl2_kv_last_error": (_I32, [_VP]),
     "arl2_kv_destroy": (_I32, [_VP]),
+    "arl2_state_write_noalloc": (_I32, [ctypes.POINTER(arl2_config), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                        _VP]),
     "arl2_selftest_wait_timeout": (_I32, [_U64, _VP]),
     "arl2_selftest_exp2": (_I32, [_VP, _VP, _I64, _VP]),
     "arl2_status_string": (ctypes.c_char_p, [_I32]),
@@ -190,6 +194,16 @@ def arl2_kv_last_error(h) -> int:
 
 def arl2_kv_destroy(h) -> None:
     _check(load_library().arl2_kv_destroy(h), "arl2_kv_destroy")
+
+
+def arl2_state_write_noalloc(cfg: arl2_config, k, v, phi_k, phi_v, S_prev, alpha, beta, S_next, dev_error,
+                             stream=None) -> None:
+    """One frame's state write with no handle and no device allocation (its
+    work space is the library's static scratch array); ``dev_error`` is a
+    device uint32 that a kernel's timed-out wait sets."""
+    _check(load_library().arl2_state_write_noalloc(ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(phi_k), _ptr(phi_v),
+                                                   _ptr(S_prev), _ptr(alpha), _ptr(beta), _ptr(S_next),
+                                                   _ptr(dev_error), _stream(stream)), "arl2_state_write_noalloc")
 
 
 def arl2_selftest_wait_timeout(limit_ns: int, stream=None) -> int:

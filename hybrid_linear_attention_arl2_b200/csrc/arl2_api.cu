@@ -279,6 +279,7 @@ const char* arl2_status_string(arl2_status s) {
     case ARL2_ERR_CUDA: return "CUDA error";
     case ARL2_ERR_TIMEOUT: return "device-side wait timed out";
     case ARL2_ERR_NO_DEVICE: return "no CUDA device";
+    case ARL2_ERR_SCRATCH_LIMIT: return "sizes exceed the fixed scratch of the allocation-free state write";
   }
   return "unknown status";
 }
@@ -681,3 +682,106 @@ arl2_status arl2_selftest_exp2(const float* x, float* y, int64_t n, void* stream
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- state write without allocation
+// For callers that must not allocate device memory (inside a stream capture,
+// under a fixed memory budget, or beside a runtime that owns the allocator),
+// arl2_state_write_noalloc runs the commit's state-write kernels with their
+// work space in this static array instead of cudaMalloc'd buffers.  The array
+// is part of the library's device image: every GPU that loads the library
+// holds it until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ARL2_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Host code cannot use g_noalloc_scratch as a pointer: on the host the name is
+// only a stand-in for the device symbol.  Look up its device address once per
+// device, with that device current.
+arl2_status noalloc_scratch(int dev, unsigned char** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return ARL2_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return e != cudaSuccess ? from_cuda(e) : ARL2_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_noalloc_addr[dev]);
+  return ARL2_OK;
+}
+
+size_t round_kib(size_t n) { return (n + 1023) & ~size_t(1023); }
+
+}  // namespace
+
+extern "C" arl2_status arl2_state_write_noalloc(const arl2_config* cfg, const void* k, const void* v,
+                                                const void* phi_k, const void* phi_v, const float* S_prev,
+                                                const float* alpha, const float* beta, float* S_next,
+                                                uint32_t* dev_error, void* stream) {
+  arl2_status s = check_config(cfg);
+  if (s != ARL2_OK) return s;
+  if (cfg->dtype != ARL2_BF16) return ARL2_ERR_UNSUPPORTED;
+  const void* ptrs[] = {k, v, phi_k, phi_v, S_prev, alpha, beta, S_next, dev_error};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return ARL2_ERR_INVALID_ARGUMENT;
+  const int B = cfg->batch, H = cfg->heads, L = cfg->tokens_per_frame;
+  const size_t mat_bf = size_t(128) * 128 * 2;
+  const size_t state_bytes = size_t(B) * H * 128 * 128 * sizeof(float);
+  if (overlaps(S_prev, S_next, state_bytes)) return ARL2_ERR_INVALID_ARGUMENT;
+  const int n_chunks = (L + 127) / 128;
+  // Scratch layout: phi_k^T, phi_v^T [H,128,128] bf16; S_prev and S_next in
+  // bf16 [B,H,128,128]; per-chunk partials [B,H,n_chunks,128,128] fp32.
+  const size_t off_pk = 0;
+  const size_t off_pv = off_pk + round_kib(size_t(H) * mat_bf);
+  const size_t off_sb = off_pv + round_kib(size_t(H) * mat_bf);
+  const size_t off_nb = off_sb + round_kib(size_t(B) * H * mat_bf);
+  const size_t off_part = off_nb + round_kib(size_t(B) * H * mat_bf);
+  const size_t need = off_part + round_kib(size_t(B) * H * n_chunks * 128 * 128 * sizeof(float));
+  if (need > size_t(ARL2_NOALLOC_SCRATCH_BYTES)) return ARL2_ERR_SCRATCH_LIMIT;
+  if (!encode_fn()) return ARL2_ERR_NO_DEVICE;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ARL2_ERR_NO_DEVICE;
+  unsigned char* scratch = nullptr;
+  s = noalloc_scratch(dev, &scratch);
+  if (s != ARL2_OK) return s;
+  auto* pk_t = reinterpret_cast<__nv_bfloat16*>(scratch + off_pk);
+  auto* pv_t = reinterpret_cast<__nv_bfloat16*>(scratch + off_pv);
+  auto* s_bf = reinterpret_cast<__nv_bfloat16*>(scratch + off_sb);
+  auto* next_bf = reinterpret_cast<__nv_bfloat16*>(scratch + off_nb);
+  auto* partial = reinterpret_cast<float*>(scratch + off_part);
+
+  CUtensorMap tk, tv, tpk, tpv, ts;
+  if (!make_act_map(&tk, k, B, L, H) || !make_act_map(&tv, v, B, L, H) || !make_mat_map(&tpk, pk_t, H) ||
+      !make_mat_map(&tpv, pv_t, H) || !make_mat_map(&ts, s_bf, B * H))
+    return ARL2_ERR_CUDA;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Only the error word must start at zero: every other scratch byte the
+  // kernels read is written earlier in this same call.
+  ARL2_TRY(cudaMemsetAsync(dev_error, 0, sizeof(uint32_t), st));
+  ARL2_TRY(launch_transpose_bf16(static_cast<const __nv_bfloat16*>(phi_k), pk_t, H, st));
+  ARL2_TRY(launch_transpose_bf16(static_cast<const __nv_bfloat16*>(phi_v), pv_t, H, st));
+  ARL2_TRY(launch_to_bf16(S_prev, s_bf, size_t(B) * H * 128 * 128, st));
+  StateParams sp{};
+  sp.S_prev = S_prev;
+  sp.alpha = alpha;
+  sp.beta = beta;
+  sp.partial = partial;
+  sp.S_next = S_next;
+  sp.S_next_bf = next_bf;
+  sp.mqt = nullptr;
+  sp.L = L;
+  sp.heads = H;
+  sp.n_chunks = n_chunks;
+  sp.corr = cfg->corr_scale < 0.f ? 1.f / float(L) : cfg->corr_scale;
+  sp.err = dev_error;
+  sp.wait_limit_ns = kDefaultWaitNs;
+  ARL2_TRY(launch_state_partial(tk, tv, tpk, tpv, ts, sp, B, st));
+  ARL2_TRY(launch_state_finalize(sp, B, st));
+  return ARL2_OK;
+}

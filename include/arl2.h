@@ -58,7 +58,9 @@ typedef enum {
   ARL2_ERR_OUT_OF_MEMORY = 3,    /* a device allocation of the library failed */
   ARL2_ERR_CUDA = 4,             /* a CUDA runtime call or kernel launch failed */
   ARL2_ERR_TIMEOUT = 5,          /* a bounded device-side wait ran out */
-  ARL2_ERR_NO_DEVICE = 6         /* no usable CUDA device / driver */
+  ARL2_ERR_NO_DEVICE = 6,        /* no usable CUDA device / driver */
+  ARL2_ERR_SCRATCH_LIMIT = 7     /* sizes need more than the fixed scratch of
+                                    arl2_state_write_noalloc */
 } arl2_status;
 
 typedef enum { ARL2_F32 = 0, ARL2_BF16 = 1 } arl2_dtype;
@@ -141,6 +143,44 @@ int64_t arl2_kv_frames(arl2_kv_t kv);
 int64_t arl2_kv_device_bytes(arl2_kv_t kv);
 arl2_status arl2_kv_last_error(arl2_kv_t kv);
 arl2_status arl2_kv_destroy(arl2_kv_t kv);
+
+/* ---- State write without allocation ---------------------------------------
+ * The paper has no counterpart to this call; it is a deployment aid.  Some
+ * callers cannot call cudaMalloc: code that runs while a CUDA graph is being
+ * captured, a host that must keep a fixed device-memory budget for the
+ * process's whole life, or an embedding runtime whose allocator owns the
+ * device and forbids allocations behind its back.  For them this call
+ * computes one frame's state write,
+ *   S_next = alpha S_prev + c K'^T diag(beta) (V' - K' S_prev),
+ * K' = rownorm2(K phi_k), V' = V phi_v, with the same kernels as
+ * arl2_frame_commit, but with no handle and without allocating anything: its
+ * work space (transposed phi_k and phi_v, a bf16 copy of S_prev, and the
+ * per-128-token partial sums) lives in one static device array of
+ * ARL2_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
+ * the process exits.
+ *   cfg       : bf16 configuration (head_dim 128); flags and softmax_scale are
+ *               ignored; corr_scale < 0 means c = 1/L.
+ *   k, v      : device bf16 [B, L, H, 128];  phi_k, phi_v : device bf16 [H, 128, 128]
+ *               as given to arl2_state_init;
+ *   S_prev    : device float32 [B, H, 128, 128];  alpha : float32 [B, H];
+ *   beta      : float32 [B, H, L];  S_next : device float32 [B, H, 128, 128],
+ *               must not overlap S_prev;
+ *   dev_error : device uint32, set to 0 by the call and to an arl2_status by a
+ *               kernel whose bounded wait ran out (read it after a sync).
+ * All pointers are caller-owned and 16-byte aligned.  The scratch needed is
+ *   2 * H * 32768 + 2 * B * H * 32768 + B * H * ceil(L / 128) * 65536 bytes
+ * (each part rounded up to 1 KiB); more than ARL2_NOALLOC_SCRATCH_BYTES returns
+ * ARL2_ERR_SCRATCH_LIMIT before any CUDA call.  The first call on a device
+ * looks up the array's device address (once per device, with that device
+ * current); make that first call before any stream capture begins.  Every
+ * call shares the one array and leaves its contents behind, so calls whose
+ * kernels overlap on the GPU (other streams, other host threads) race:
+ * serialise them.  Errors: INVALID_ARGUMENT, UNSUPPORTED, SCRATCH_LIMIT, CUDA. */
+#define ARL2_NOALLOC_SCRATCH_BYTES (16u << 20)
+arl2_status arl2_state_write_noalloc(const arl2_config* cfg, const void* k, const void* v,
+                                     const void* phi_k, const void* phi_v, const float* S_prev,
+                                     const float* alpha, const float* beta, float* S_next,
+                                     uint32_t* dev_error, void* stream);
 
 /* ---- Diagnostics -----------------------------------------------------------
  * Run one kernel whose bounded wait is on a barrier that nothing completes,

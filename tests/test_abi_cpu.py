@@ -69,3 +69,24 @@ def test_kv_validation(lib):
     cfg = arl2.make_config(1, 2, 128, 64, arl2.ARL2_BF16)
     assert L.arl2_kv_init(ctypes.byref(cfg), 0, None, ctypes.byref(h)) == 1
     assert L.arl2_kv_init(None, 4, None, ctypes.byref(h)) == 1
+
+
+def test_noalloc_state_write_host_checks(lib):
+    """The allocation-free state write rejects, before any CUDA call, what it
+    cannot run: a float32 config, null or misaligned pointers, overlapping
+    states, and sizes whose work space exceeds its fixed static array."""
+    L = arl2.load_library()
+    ptrs = [16, 32, 48, 64, 1 << 20, 96, 112, 64 << 20, 144]
+    call = lambda cfg, p=ptrs: L.arl2_state_write_noalloc(ctypes.byref(cfg), *p, None)
+    assert call(arl2.make_config(1, 2, 32, 16, arl2.ARL2_F32)) == 2
+    assert call(arl2.make_config(1, 2, 64, 16, arl2.ARL2_BF16)) == 2
+    bad = list(ptrs)
+    bad[0] = None
+    assert call(arl2.make_config(1, 2, 128, 16, arl2.ARL2_BF16), bad) == 1
+    bad[0] = 17
+    assert call(arl2.make_config(1, 2, 128, 16, arl2.ARL2_BF16), bad) == 1
+    same = list(ptrs)
+    same[7] = same[4]                                                       # S_next over S_prev
+    assert call(arl2.make_config(1, 2, 128, 16, arl2.ARL2_BF16), same) == 1
+    assert call(arl2.make_config(4, 12, 128, 1560, arl2.ARL2_BF16)) == 7    # 4 streams x 1560 tokens
+    assert arl2.arl2_status_string(7).startswith("sizes exceed")
