@@ -85,10 +85,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
   return r == CUDA_SUCCESS;
 }
 
-// Token-major activations [B, tokens, H, 128] as a map over (H*128, tokens, B).
-bool make_act_map(CUtensorMap* m, const void* base, int B, int64_t tokens, int H) {
+// Token-major activations [B, tokens, H, 128] as a map over (H*128, tokens, B),
+// boxes of 64 columns x `rows` tokens.
+bool make_act_map(CUtensorMap* m, const void* base, int B, int64_t tokens, int H, uint32_t rows = 128) {
   const uint64_t row = uint64_t(H) * 128 * 2;
-  return make_map(m, base, uint64_t(H) * 128, uint64_t(tokens), uint64_t(B), row, row * uint64_t(tokens), 128);
+  return make_map(m, base, uint64_t(H) * 128, uint64_t(tokens), uint64_t(B), row, row * uint64_t(tokens), rows);
 }
 
 // Stacked 128 x 128 bf16 matrices [slabs, 128, 128] as a map over (128, 128, slabs).
@@ -232,13 +233,13 @@ arl2_status run_attention(arl2_state* h, const void* q, const void* k, const voi
     ARL2_TRY(launch_f32_attn(p, c.batch, st));
     return ARL2_OK;
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads) ||
       !make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads) ||
-      !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads))
+      !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads) ||
+      !make_act_map(&to, o, c.batch, c.tokens_per_frame, c.heads, 32))
     return ARL2_ERR_CUDA;
   AttnParams p{};
-  p.o = static_cast<__nv_bfloat16*>(o);
   p.q_len = p.kv_len = c.tokens_per_frame;
   p.heads = c.heads;
   p.scale_log2 = h->scale * 1.4426950408889634f;
@@ -249,7 +250,7 @@ arl2_status run_attention(arl2_state* h, const void* q, const void* k, const voi
   p.err = h->err;
   p.wait_limit_ns = h->wait_ns;
   if (!attn_partition(p, c.batch, h->sms)) return ARL2_ERR_UNSUPPORTED;
-  ARL2_TRY(launch_attn_bf16(tq, tk, tv, h->tm_mqt, p, st));
+  ARL2_TRY(launch_attn_bf16(tq, tk, tv, h->tm_mqt, to, p, st));
   return ARL2_OK;
 }
 
@@ -588,13 +589,13 @@ arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, voi
     ARL2_TRY(launch_f32_attn(p, c.batch, st));
     return ARL2_OK;
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads) ||
       !make_act_map(&tk, h->kc, c.batch, stride_tokens, c.heads) ||
-      !make_act_map(&tv, h->vc, c.batch, stride_tokens, c.heads))
+      !make_act_map(&tv, h->vc, c.batch, stride_tokens, c.heads) ||
+      !make_act_map(&to, o, c.batch, c.tokens_per_frame, c.heads, 32))
     return ARL2_ERR_CUDA;
   AttnParams p{};
-  p.o = static_cast<__nv_bfloat16*>(o);
   p.q_len = c.tokens_per_frame;
   p.kv_len = int(kv_tokens);
   p.heads = c.heads;
@@ -606,7 +607,7 @@ arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, voi
   p.err = h->err;
   p.wait_limit_ns = h->wait_ns;
   if (!attn_partition(p, c.batch, h->sms)) return ARL2_ERR_UNSUPPORTED;
-  ARL2_TRY(launch_attn_bf16(tq, tk, tv, tq, p, st));
+  ARL2_TRY(launch_attn_bf16(tq, tk, tv, tq, to, p, st));
   return ARL2_OK;
 }
 

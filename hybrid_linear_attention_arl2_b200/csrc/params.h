@@ -14,7 +14,6 @@ constexpr int kAttnMaxGrid = 192;  // persistent CTAs at most (>= the SM count o
 // Fused intra-frame softmax + inter-frame read-out (attn_bf16.cu): a
 // persistent grid over (query-tile pair, key tile) units, see the kernel.
 struct AttnParams {
-  __nv_bfloat16* o;     // [B, q_len, H, 128]
   int q_len;            // query tokens per stream
   int kv_len;           // valid key/value tokens per stream
   int heads;
@@ -22,20 +21,20 @@ struct AttnParams {
   int n_pair;           // n_qt / 2: blocks with two sub-tiles
   int n_blk;            // blocks per (stream, head): n_pair + n_qt % 2
   int nkv;              // key tiles of 128
-  long long total_weight;  // B * H * n_qt * nkv
+  long long total_units;   // B * H * n_blk * nkv
   int grid;             // persistent CTAs (<= kAttnMaxGrid)
   unsigned range[kAttnMaxGrid + 1];  // CTA c takes units [range[c], range[c + 1])
   float scale_log2;     // softmax scale * log2(e)
   uint32_t flags;       // 1: intra only, 2: inter only
   int has_inter;        // 1: add Q MqT^T
-  float* scratch;       // [grid][2][kAttnSlotFloats] partial O (bf16, chunk-major) and (m, l)
+  float* scratch;       // [grid][2][kAttnSlotFloats] normalised partial O (bf16, chunk-major) and (m, l)
   unsigned* ready;      // [grid][2] partial-ready flags, zero between launches
   uint32_t* err;        // device error word
   uint64_t wait_limit_ns;
 };
 
-// floats of one partial slot (one sub-tile of one CTA): 128 x 128 unnormalised O
-// values in bf16, stored chunk-major (16-byte chunk i of row r at byte (i * 128 + r) * 16),
+// floats of one partial slot (one sub-tile of one CTA): 128 x 128 O values
+// normalised by the slot's own l, in bf16, stored chunk-major (16-byte chunk i of row r at byte (i * 128 + r) * 16),
 // then m[128] and l[128] in fp32
 constexpr int kAttnSlotFloats = 128 * 64 + 256;
 
@@ -82,8 +81,12 @@ struct F32CommitParams {
   float corr;
 };
 
+// tq, tk, tv: Q, K, V maps; tmq: MqT map (read only when has_inter); tmo: the
+// output O [B, q_len, H, 128] in boxes of 64 columns x 32 rows, written with
+// tile stores.
 cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tmq, const AttnParams& p, cudaStream_t stream);
+                             const CUtensorMap& tmq, const CUtensorMap& tmo, const AttnParams& p,
+                             cudaStream_t stream);
 // Fills the partition fields of `p` for B streams on a device with `sms` SMs;
 // false if the problem is too large for 32-bit unit indices.
 bool attn_partition(AttnParams& p, int batch, int sms);

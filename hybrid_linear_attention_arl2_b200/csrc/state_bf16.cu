@@ -45,10 +45,6 @@ __device__ __forceinline__ bool warp_wait_s(uint64_t* bar, uint32_t parity, cons
   return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 enum { P_IN, P_MAPS, P_KP, P_S, P_KS, P_R, P_DS, P_DRAIN, P_COUNT };
 
 __global__ void __launch_bounds__(kStateThreads, 1)
