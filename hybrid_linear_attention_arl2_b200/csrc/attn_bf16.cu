@@ -66,7 +66,11 @@ constexpr int kMaxContrib = 8;        // partials a finishing CTA may combine
 // over the CTA must not exceed 512 * kLaunchRegs, or setmaxnreg.inc would wait
 // forever; the launcher refuses to run unless the compiled kernel has exactly
 // kLaunchRegs.
-constexpr int kPolyPairs = 5;  // of every 16 exp2 pairs of a full tile, this many run on the FMA pipe
+// Of every 16 exp2 pairs of a full tile, this many run on the FMA pipe
+// (exp2_poly) instead of the MUFU.  Measured on the 1560-token frame: 0 is
+// fastest (342 TFLOP/s against 320 with 5), the softmax being bound by issue
+// and latency rather than by the MUFU, so the option stays off.
+constexpr int kPolyPairs = 0;
 constexpr int kLaunchRegs = 128;
 constexpr int kCtlRegs = 56;
 constexpr int kEpiRegs = 72;

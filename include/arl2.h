@@ -189,9 +189,10 @@ arl2_status arl2_state_write_noalloc(const arl2_config* cfg, const void* k, cons
 arl2_status arl2_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /* y[i] = 2^x[i] (device float32 arrays of n values) through the FMA-pipe
- * exponential the attention kernel uses for part of its softmax (a degree-3
+ * exponential the attention kernel can use for part of its softmax (a degree-3
  * polynomial after rounding x to an integer; inputs clamped to [-125, 125];
- * relative error <= 1.0e-4).  For accuracy tests of that routine. */
+ * relative error <= 1.0e-4; off in the shipped configuration, where the MUFU
+ * alone measured faster).  For accuracy tests of that routine. */
 arl2_status arl2_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
 
 const char* arl2_status_string(arl2_status s);
