@@ -38,7 +38,7 @@ TOKENS_PER_STEP = None  # set from the config
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="arl2", choices=["arl2", "reference"])
     ap.add_argument("--config", type=int, default=1, choices=[1, 2, 4])
@@ -65,60 +65,101 @@ def frame_flops(cfg: W.Config) -> dict:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled every 10 ms by NVML while
+    the timed region runs (read-only queries; no setting of the GPU is changed).
+    Falls back to `nvidia-smi -lms 50` when NVML cannot be loaded."""
+
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
-        self.lines: list[str] = []
         self.thread = None
+        self.stop_flag = threading.Event()
+        self.samples: list[tuple[float, float, float, tuple]] = []  # (sm, sm_max, watts, reasons)
+        self.source = None
 
     def start(self):
         try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self._nvml_index(pynvml))
+            self.source = "nvml 10 ms"
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                        w = pynvml.nvmlDeviceGetPowerUsage(h) / 1e3
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    except pynvml.NVMLError:
+                        break
+                    self.samples.append((sm, smax, w, tuple(n for n, b in bits.items() if r & b)))
+                    self.stop_flag.wait(0.010)
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:  # NVML missing or refused: nvidia-smi below
+            pass
+        try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
             return
+        self.source = "nvidia-smi 50 ms"
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def _nvml_index(self, pynvml) -> int:
+        # CUDA_VISIBLE_DEVICES renumbers devices for CUDA but not for NVML
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            ids = [v.strip() for v in vis.split(",") if v.strip()]
+            if self.dev < len(ids) and ids[self.dev].isdigit():
+                return int(ids[self.dev])
+        return self.dev
+
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        if self.thread:
-            self.thread.join(timeout=2)
-        sm, smax, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
+            parts = [p.strip() for p in line.strip().split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
+                sm, smax, w = float(parts[1]), float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(power)}
+            self.samples.append((sm, smax, w, tuple(n for n, v in zip(self.REASONS, parts[5:9])
+                                                    if v.lower() == "active")))
+
+    def stop(self) -> dict:
+        self.stop_flag.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": self.source}
+        sm = [s[0] for s in self.samples]
+        reasons = sorted({r for s in self.samples for r in s[3]})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(s[1] for s in self.samples),
+                "sm_mhz_min": min(sm), "reasons": reasons, "samples": len(sm),
+                "power_w_max": max(s[2] for s in self.samples), "source": self.source}
 
 
 # ------------------------------------------------------------------ device workload
@@ -143,6 +184,18 @@ class DeviceStream:
 
     def triple(self, frame: int, pas: int):
         return self.pool[self.wl.pool_index(0, frame, pas)]
+
+
+def whole_job_rate(ms: float, steps: int, world: int, dist=None, device="cpu"):
+    """Frames/s of the whole job: every rank ran `steps` frames; the time is the
+    slowest rank's device time (max over ranks).  Returns (frames/s, max ms)."""
+    import torch
+    ms_max = float(ms)
+    if dist is not None and world > 1:
+        t = torch.tensor([ms_max], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    return steps * world / (ms_max / 1e3), ms_max
 
 
 def run_arl2(args, rank: int, world: int):
@@ -235,7 +288,6 @@ def run_arl2(args, rank: int, world: int):
         stream.synchronize()
         torch.cuda.synchronize()
         clocks.start()
-        time.sleep(0.3)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         attn_ev = []
@@ -275,14 +327,7 @@ def run_arl2(args, rank: int, world: int):
         attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
         attn_avg_ms = float(np.mean(attn_ms))
 
-    # max over ranks
-    ms_max = ms
-    if dist is not None:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    frames_total = steps_done * world
-    value = frames_total / (ms_max / 1e3)
+    value, ms_max = whole_job_rate(ms, steps_done, world, dist, device)
     ms_per_step = ms_max / steps_done
 
     result = {
@@ -344,12 +389,8 @@ def run_e2e(args, cfg, ds, layer, device, stream, dist, world):
                 d2h += O[p].numel() * 2
         e1.record(stream)
         e1.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": steps * world / (ms / 1e3), "unit": "frames/s",
+    value, _ = whole_job_rate(e0.elapsed_time(e1), steps, world, dist, device)
+    return {"value": value, "unit": "frames/s",
             "h2d_bytes_per_step": h2d // steps, "d2h_bytes_per_step": d2h // steps}
 
 
@@ -378,6 +419,32 @@ def cpu_oracle_rate(cfg: W.Config, budget_s: float = 12.0, sample_note=True):
     return {"value": frames / dt, "unit": "frames/s", "cores": cores, "kind": "oracle",
             "sample": f"{frames} whole frames (4 query passes + 1 commit each) of one {cfg.name} layer, "
                       f"numpy float64, {dt:.1f} s"}
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_bf16_kernel
+# launch on the single-hybrid-layer-bf16 workload, from one ncu capture of
+# `bench.py --profile-small --no-graphs`; reported only while the kernel sources
+# hash to the value the capture was taken on.
+ATTN_TRAFFIC = {"bytes": 15441920 + 3072, "sources_sha256": "728dba23c4cc4c06810cac0f6c12c1ff0ce36c646911302b34eac3a5a09fe06f",
+                "capture": "profiles/attn_bf16_kernel_single-hybrid-layer-bf16.md"}
+ATTN_SOURCES = ("hybrid_linear_attention_arl2_b200/csrc/attn_bf16.cu",
+                "hybrid_linear_attention_arl2_b200/csrc/sm100.cuh",
+                "hybrid_linear_attention_arl2_b200/csrc/params.h")
+
+
+def attn_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def attn_traffic():
+    if ATTN_TRAFFIC["bytes"] is None or ATTN_TRAFFIC["sources_sha256"] != attn_sources_sha256():
+        return None
+    return ATTN_TRAFFIC["bytes"]
 
 
 def peaks():
@@ -442,7 +509,7 @@ def main():
         "pct_bf16_peak": {"value": 100.0 * frame_tflops / peak_sus, "basis": f"sustained bf16 {src}",
                           "burst_basis": 100.0 * frame_tflops / peak_burst},
         "roofline": {"bound": "tensor", "kernel": "attn_bf16_kernel", "achieved": attn_tflops, "peak": peak_sus,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak_sus, "traffic": None,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak_sus, "traffic": attn_traffic(),
                      "peak_basis": f"bf16_tflops_sustained {src}"},
         "clocks": res["clocks"],
         "gpu_launches": res["launches_per_step"] * res["steps"],
