@@ -65,16 +65,17 @@ constexpr int kMaxContrib = 8;        // partials a finishing CTA may combine
 // kEpiRegs, and the two softmax warpgroups rise to kSoftmaxRegs.  The sum
 // over the CTA must not exceed 512 * kLaunchRegs, or setmaxnreg.inc would wait
 // forever; the launcher refuses to run unless the compiled kernel has exactly
-// kLaunchRegs.
+// kLaunchRegs.  80 / 64 / 184 measured fastest on the 1560-token frame (357
+// TFLOP/s against 338 with 56 / 72 / 192): the issuer spills less.
 // Of every 16 exp2 pairs of a full tile, this many run on the FMA pipe
 // (exp2_poly) instead of the MUFU.  Measured on the 1560-token frame: 0 is
 // fastest (342 TFLOP/s against 320 with 5), the softmax being bound by issue
 // and latency rather than by the MUFU, so the option stays off.
 constexpr int kPolyPairs = 0;
 constexpr int kLaunchRegs = 128;
-constexpr int kCtlRegs = 56;
-constexpr int kEpiRegs = 72;
-constexpr int kSoftmaxRegs = 192;
+constexpr int kCtlRegs = 80;
+constexpr int kEpiRegs = 64;
+constexpr int kSoftmaxRegs = 184;
 static_assert(128 * kCtlRegs + 128 * kEpiRegs + 256 * kSoftmaxRegs <= kAttnThreads * kLaunchRegs,
               "register split too large");
 
@@ -89,8 +90,9 @@ enum {
   B_SD = B_ST + 2,    // [2] every MMA of the segment completed
   B_ES = B_SD + 2,    // [2] epilogue done with the S columns (X read, or nothing to read) (4 warps)
   B_EO = B_ES + 2,    // [2] epilogue has read O from tensor memory (4 warps)
-  B_PRE = B_EO + 2,   // [2] contributors' partials and statistics in shared memory (4 warps; once per launch)
-  B_DRAIN = B_PRE + 2,
+  B_PRE = B_EO + 2,   // [2] contributors' flags acquired (1 arrival; once per launch)
+  B_PD = B_PRE + 2,   // [2] contributors' partials in shared memory (1 arrival + bulk-copy bytes; once per launch)
+  B_DRAIN = B_PD + 2,
   B_COUNT
 };
 
@@ -396,15 +398,11 @@ __device__ __forceinline__ void add_chunk(float* v, const uint4 x, const float w
   }
 }
 
-// Shared-memory places of a split block's contributor data once the CTA's
-// last MMA has released the K/V ring: partial k of sub-tile s at
-// part_slot(s, k) (chunk-major, as in the scratch slot) and its (m, l) rows in
-// ring slot 3.
+// Shared-memory place of partial k of sub-tile s of a split block
+// (chunk-major, as in the scratch slot): the first one in the staging buffer,
+// the others in the K/V ring once the CTA's last MMA has released it.
 __device__ __forceinline__ const uint8_t* part_slot(const uint8_t* stage, const uint8_t* ring, int s, int k) {
   return (s == 0 && k == 0) ? stage : ring + (s == 0 ? 0 : 1 + k) * kTile;
-}
-__device__ __forceinline__ const float* part_stats(const uint8_t* ring, int s, int k) {
-  return reinterpret_cast<const float*>(ring + 3 * kTile + (s * 2 + k) * 1024);
 }
 
 // The last segment of a CTA whose block continues in the next CTAs (a split
@@ -430,26 +428,27 @@ __device__ __forceinline__ bool split_epilogue(const AttnParams& p, uint64_t* ba
   const bool use_intra = !(p.flags & 2u);
   const bool use_inter = p.has_inter && !(p.flags & 1u);
   const bool in_smem = n_contrib <= 2;
-  if (!warp_wait(&bars[B_SD + sub], sd_parity, w)) return false;
+  // The contributors' flags are acquired (by the epilogue warpgroup): their
+  // statistics are read from global memory while the last MMAs may still run.
   if (!warp_wait(&bars[B_PRE + sub], 0, w)) return false;
-  tc_fence_after();
   float a_self = 0.f, wk[kMaxContrib];
 #pragma unroll
   for (int k = 0; k < kMaxContrib; ++k) wk[k] = 0.f;
   if (row_ok) {
     float mk[kMaxContrib], lk[kMaxContrib];
-    float M = m;
 #pragma unroll
     for (int k = 0; k < kMaxContrib; ++k) {
       mk[k] = -INFINITY;
       lk[k] = 0.f;
       if (k < n_contrib) {
-        const float* st = in_smem ? part_stats(ring, sub, k) : slot_of(p, cta + 1 + k, sub) + kSlotStats;
+        const float* st = slot_of(p, cta + 1 + k, sub) + kSlotStats;
         mk[k] = st[row];
         lk[k] = st[128 + row];
       }
-      M = fmaxf(M, mk[k]);
     }
+    float M = m;
+#pragma unroll
+    for (int k = 0; k < kMaxContrib; ++k) M = fmaxf(M, mk[k]);
     const float e_self = fast_exp2(m - M);
     float L = l * e_self;
 #pragma unroll
@@ -462,37 +461,50 @@ __device__ __forceinline__ bool split_epilogue(const AttnParams& p, uint64_t* ba
 #pragma unroll
     for (int k = 0; k < kMaxContrib; ++k) wk[k] *= inv;
   }
+  if (!warp_wait(&bars[B_SD + sub], sd_parity, w)) return false;
+  if (!warp_wait(&bars[B_PD + sub], 0, w)) return false;
+  tc_fence_after();
   uint8_t* wbox = obox + quarter * 8192;
   if (warp_on) {
+    const float2 as2 = make_float2(use_intra ? a_self : 0.f, use_intra ? a_self : 0.f);
 #pragma unroll 1
     for (int q = 0; q < 4; ++q) {  // 32 columns at a time
       uint32_t ro[32], rx[32];
       tmem_ld32(tO + lane_off + q * 32, ro);
-      if (p.has_inter) tmem_ld32(tS + lane_off + q * 32, rx);
+      if (use_inter) tmem_ld32(tS + lane_off + q * 32, rx);
       tmem_wait_ld();
-      float* v = reinterpret_cast<float*>(ro);
+      float2* v = reinterpret_cast<float2*>(ro);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = use_intra ? v[i] * a_self : 0.f;
+      for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(v[i], as2);
       if (use_intra) {
 #pragma unroll
         for (int k = 0; k < kMaxContrib; ++k) {
-          if (k >= n_contrib) break;
-          const uint8_t* base =
-              in_smem ? part_slot(stage, ring, sub, k) : reinterpret_cast<const uint8_t*>(slot_of(p, cta + 1 + k, sub));
+          if (k < n_contrib) {
+            const uint8_t* base = in_smem ? part_slot(stage, ring, sub, k)
+                                          : reinterpret_cast<const uint8_t*>(slot_of(p, cta + 1 + k, sub));
+            const float2 w2 = make_float2(wk[k], wk[k]);
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) add_chunk(v + 8 * ch, partial_chunk(base, q * 4 + ch, row), wk[k]);
+            for (int ch = 0; ch < 4; ++ch) {
+              const uint4 x = partial_chunk(base, q * 4 + ch, row);
+              const uint32_t x4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                v[4 * ch + e] = __ffma2_rn(make_float2(bf16_lo(x4[e]), bf16_hi(x4[e])), w2, v[4 * ch + e]);
+            }
+          }
         }
       }
       if (use_inter) {
+        const float2* x2 = reinterpret_cast<const float2*>(rx);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] += __uint_as_float(rx[i]);
+        for (int i = 0; i < 16; ++i) v[i] = __fadd2_rn(v[i], x2[i]);
       }
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         const int c16 = q * 4 + ch;  // 16-byte chunk of the row: box c16 / 8, chunk c16 % 8 swizzled by row
         *reinterpret_cast<uint4*>(wbox + (c16 >> 3) * 4096 + lane * 128 + (((c16 & 7) ^ (lane & 7)) << 4)) =
-            make_uint4(pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]), pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
-                       pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]), pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
+            make_uint4(pack_bf16x2(v[4 * ch + 0].x, v[4 * ch + 0].y), pack_bf16x2(v[4 * ch + 1].x, v[4 * ch + 1].y),
+                       pack_bf16x2(v[4 * ch + 2].x, v[4 * ch + 2].y), pack_bf16x2(v[4 * ch + 3].x, v[4 * ch + 3].y));
       }
     }
   }
@@ -506,7 +518,7 @@ __device__ __forceinline__ bool split_epilogue(const AttnParams& p, uint64_t* ba
       tma_store_3d(tm_o, wbox, h * 128, qt * 128 + quarter * 32, b);
       tma_store_3d(tm_o, wbox + 4096, h * 128 + 64, qt * 128 + quarter * 32, b);
       bulk_commit();
-      bulk_wait0();
+      bulk_wait_read0();  // the box is read before the CTA's shared memory goes away
     }
   }
   __syncwarp();
@@ -730,11 +742,16 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
       return false;
     }
     if (n_contrib > 0) {
-      // Split block (this CTA's last segment): acquire the contributors' flags,
-      // then copy their partials and statistics into shared memory for the
-      // softmax warpgroups' combine (split_epilogue): the first partial into the
-      // staging buffer while the MMAs still run, the rest into the K/V ring once
-      // the last MMA has released it.
+      // Split block (this CTA's last segment): acquire the contributors' flags
+      // (B_PRE: the softmax warpgroups may then read the contributors'
+      // statistics), then bring their partials into shared memory with bulk
+      // copies for the combine in split_epilogue (B_PD): the first partial of
+      // sub-tile A into the staging buffer at once, the others into the K/V
+      // ring once the CTA's last MMA has released it.  With more than two
+      // contributors the combine reads the partials from global memory.
+      const bool in_smem = n_contrib <= 2;
+      if (lane == 0 && staged) bulk_wait_read0();  // earlier tile stores have read the staging buffer
+      named_bar(NB_EPI, 128);
       if (et == 0) {
         for (int s2 = 0; s2 < nsub; ++s2)
           for (int k = 0; k < n_contrib && !*abort_flag; ++k) {
@@ -748,37 +765,27 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
               }
             }
           }
-        if (staged) bulk_wait_read0();  // earlier tile stores have read the staging buffer
-      } else if (lane == 0 && staged) {
-        bulk_wait_read0();
-      }
-      named_bar(NB_EPI, 128);
-      if (*abort_flag) return false;
-      if (n_contrib <= 2) {
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(slot_of(p, cta + 1, 0));
-#pragma unroll
-        for (int i = 0; i < 16; ++i) cp_async16(stage + (i * 128 + row) * 16, src + (i * 128 + row) * 16);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        if (!warp_wait(&bars[B_SD + 0], segc[0] & 1, w)) return false;  // the ring is idle from here on
-        for (int s2 = 0; s2 < nsub; ++s2)
-          for (int k = 0; k < n_contrib; ++k) {
-            const uint8_t* sl = reinterpret_cast<const uint8_t*>(slot_of(p, cta + 1 + k, s2));
-            if (s2 > 0 || k > 0) {
-              uint8_t* dst = const_cast<uint8_t*>(part_slot(stage, ring, s2, k));
-#pragma unroll
-              for (int i = 0; i < 16; ++i) cp_async16(dst + (i * 128 + row) * 16, sl + (i * 128 + row) * 16);
-            }
-            if (et < 64) {  // (m, l): 2 x 128 floats, 16 bytes per thread
-              uint8_t* dst = ring + 3 * kTile + (s2 * 2 + k) * 1024 + et * 16;
-              cp_async16(dst, sl + kSlotStats * 4 + et * 16);
+        if (!*abort_flag) {
+          fence_async_global();
+          for (int s2 = 0; s2 < nsub; ++s2) {
+            mbar_arrive(&bars[B_PRE + s2]);
+            mbar_expect_tx(&bars[B_PD + s2], in_smem ? uint32_t(n_contrib) * kTile : 0u);
+          }
+          if (in_smem) {
+            bulk_load(stage, slot_of(p, cta + 1, 0), kTile, &bars[B_PD + 0]);
+            if (n_contrib > 1 || nsub > 1) {
+              if (wait1(&bars[B_SD + nsub - 1], segc[nsub - 1] & 1, w)) {  // the ring is idle from here on
+                for (int s2 = 0; s2 < nsub; ++s2)
+                  for (int k = (s2 == 0 ? 1 : 0); k < n_contrib; ++k)
+                    bulk_load(const_cast<uint8_t*>(part_slot(stage, ring, s2, k)), slot_of(p, cta + 1 + k, s2), kTile,
+                              &bars[B_PD + s2]);
+              }
             }
           }
-        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-        named_bar(NB_EPI, 128);  // every thread's copies have landed
+        }
       }
       __syncwarp();
-      if (lane == 0)
-        for (int s2 = 0; s2 < nsub; ++s2) mbar_arrive(&bars[B_PRE + s2]);
+      if (*abort_flag) return false;
       // once the combine has read the partials (it arrives on B_ES), their flags
       // go back to zero for the next launch
       for (int s2 = 0; s2 < nsub; ++s2)
@@ -891,7 +898,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
-      const bool four = (i >= B_PF && i < B_PF + 2) || (i >= B_ST && i < B_ST + 2) || (i >= B_ES && i < B_PRE + 2);
+      const bool four = (i >= B_PF && i < B_PF + 2) || (i >= B_ST && i < B_ST + 2) || (i >= B_ES && i < B_EO + 2);
       mbar_init(&bars[i], four ? 4u : 1u);
     }
     *abort_flag = 0;
