@@ -28,7 +28,10 @@ namespace arl2 {
 constexpr uint32_t kTileB = 32768;
 constexpr uint32_t kHalfB = 16384;
 constexpr int kStateThreads = 192;
-constexpr int kPartialSmem = 4 * kTileB + 256 + 1024;
+// Three 32 KB tiles (K then K'; V then S_{N-1}; phi_k^T then phi_v^T then R):
+// two CTAs fit on an SM, so the 13 chunks x 12 heads of a 1560-token frame run
+// in one wave on 148 SMs.
+constexpr int kPartialSmem = 3 * kTileB + 256 + 1024;
 constexpr int kPrepSmem = 2 * kTileB + 256 + 1024;
 
 // Byte offset of bf16 element (row, col) of a 128-row tile stored as two
@@ -45,19 +48,18 @@ __device__ __forceinline__ bool warp_wait_s(uint64_t* bar, uint32_t parity, cons
   return __all_sync(0xffffffffu, ok);
 }
 
-enum { P_IN, P_MAPS, P_KP, P_S, P_KS, P_R, P_DS, P_DRAIN, P_COUNT };
+enum { P_IN, P_MK, P_PV, P_MV, P_KP, P_S, P_KS, P_R, P_DS, P_DRAIN, P_COUNT };
 
-__global__ void __launch_bounds__(kStateThreads, 1)
+__global__ void __launch_bounds__(kStateThreads, 2)
 state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_phik_t, const __grid_constant__ CUtensorMap tm_phiv_t,
                      const __grid_constant__ CUtensorMap tm_s_bf, const StateParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;               // K tile, then K' (bf16)
-  uint8_t* sV = smem + kTileB;      // V tile, then R (bf16)
-  uint8_t* sPk = smem + 2 * kTileB; // phi_k^T, then S_{N-1} (bf16)
-  uint8_t* sPv = smem + 3 * kTileB; // phi_v^T
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 4 * kTileB);
+  uint8_t* sV = smem + kTileB;      // V tile, then S_{N-1} (bf16)
+  uint8_t* sP = smem + 2 * kTileB;  // phi_k^T, then phi_v^T, then R (bf16)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 3 * kTileB);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + P_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -81,39 +83,46 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
   if (warp == 0) {
     if (lane == 0) {
       const int x0 = h * 128, t0 = chunk * 128;
-      mbar_expect_tx(&bars[P_IN], 4 * kTileB);
+      mbar_expect_tx(&bars[P_IN], 3 * kTileB);
       tma_load_3d(sK, &tm_k, &bars[P_IN], x0, t0, b);
       tma_load_3d(sK + kHalfB, &tm_k, &bars[P_IN], x0 + 64, t0, b);
       tma_load_3d(sV, &tm_v, &bars[P_IN], x0, t0, b);
       tma_load_3d(sV + kHalfB, &tm_v, &bars[P_IN], x0 + 64, t0, b);
-      tma_load_3d(sPk, &tm_phik_t, &bars[P_IN], 0, 0, h);
-      tma_load_3d(sPk + kHalfB, &tm_phik_t, &bars[P_IN], 64, 0, h);
-      tma_load_3d(sPv, &tm_phiv_t, &bars[P_IN], 0, 0, h);
-      tma_load_3d(sPv + kHalfB, &tm_phiv_t, &bars[P_IN], 64, 0, h);
-      if (mbar_wait(&bars[P_MAPS], 0, w)) {
-        mbar_expect_tx(&bars[P_S], kTileB);
-        tma_load_3d(sPk, &tm_s_bf, &bars[P_S], 0, 0, slab);
-        tma_load_3d(sPk + kHalfB, &tm_s_bf, &bars[P_S], 64, 0, slab);
+      tma_load_3d(sP, &tm_phik_t, &bars[P_IN], 0, 0, h);
+      tma_load_3d(sP + kHalfB, &tm_phik_t, &bars[P_IN], 64, 0, h);
+      if (mbar_wait(&bars[P_MK], 0, w)) {  // phi_k^T read: phi_v^T in its place
+        mbar_expect_tx(&bars[P_PV], kTileB);
+        tma_load_3d(sP, &tm_phiv_t, &bars[P_PV], 0, 0, h);
+        tma_load_3d(sP + kHalfB, &tm_phiv_t, &bars[P_PV], 64, 0, h);
+        if (mbar_wait(&bars[P_MV], 0, w)) {  // V read: S_{N-1} in its place
+          mbar_expect_tx(&bars[P_S], kTileB);
+          tma_load_3d(sV, &tm_s_bf, &bars[P_S], 0, 0, slab);
+          tma_load_3d(sV + kHalfB, &tm_s_bf, &bars[P_S], 64, 0, slab);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t ka = smem_u32(sK), va = smem_u32(sV), pka = smem_u32(sPk), pva = smem_u32(sPv);
+      const uint32_t ka = smem_u32(sK), va = smem_u32(sV), pa = smem_u32(sP);
       const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
       bool ok = mbar_wait(&bars[P_IN], 0, w);
-      if (ok) {
+      if (ok) {  // K~ = K phi_k
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // K~ = K phi_k ; V~ = V phi_v
-          const uint32_t off = (kk >> 2) * kHalfB + (kk & 3) * 32;
-          mma_ss(tA, smem_desc_sw128(ka + off, 16, 1024), smem_desc_sw128(pka + off, 16, 1024), id_kk, kk > 0);
-        }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kHalfB + (kk & 3) * 32;
-          mma_ss(tB, smem_desc_sw128(va + off, 16, 1024), smem_desc_sw128(pva + off, 16, 1024), id_kk, kk > 0);
+          mma_ss(tA, smem_desc_sw128(ka + off, 16, 1024), smem_desc_sw128(pa + off, 16, 1024), id_kk, kk > 0);
         }
-        mma_commit(&bars[P_MAPS]);
+        mma_commit(&bars[P_MK]);
+      }
+      if (ok && (ok = mbar_wait(&bars[P_PV], 0, w))) {  // V~ = V phi_v
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfB + (kk & 3) * 32;
+          mma_ss(tB, smem_desc_sw128(va + off, 16, 1024), smem_desc_sw128(pa + off, 16, 1024), id_kk, kk > 0);
+        }
+        mma_commit(&bars[P_MV]);
       }
       // K'S: A = K' (K-major), B = S_{N-1} stored [i][j]: N = j contiguous -> MN-major.
       if (ok && (ok = mbar_wait(&bars[P_KP], 0, w)) && (ok = mbar_wait(&bars[P_S], 0, w))) {
@@ -122,7 +131,7 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * kHalfB + (kk & 3) * 32;
-          mma_ss(tA, smem_desc_sw128(ka + aoff, 16, 1024), smem_desc_sw128(pka + kk * 2048, kHalfB, 1024), id_ks,
+          mma_ss(tA, smem_desc_sw128(ka + aoff, 16, 1024), smem_desc_sw128(va + kk * 2048, kHalfB, 1024), id_ks,
                  kk > 0);
         }
         mma_commit(&bars[P_KS]);
@@ -133,7 +142,7 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         const uint32_t id_d = idesc_bf16(128, 128, 1, 1);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tB, smem_desc_sw128(ka + kk * 2048, kHalfB, 1024), smem_desc_sw128(va + kk * 2048, kHalfB, 1024),
+          mma_ss(tB, smem_desc_sw128(ka + kk * 2048, kHalfB, 1024), smem_desc_sw128(pa + kk * 2048, kHalfB, 1024),
                  id_d, kk > 0);
         mma_commit(&bars[P_DS]);
       }
@@ -144,10 +153,10 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const int token = chunk * 128 + row;
     const bool valid = token < p.L;
-    bool ok = warp_wait_s(&bars[P_MAPS], 0, w);
+    bool ok = warp_wait_s(&bars[P_MK], 0, w);
     if (ok) {
       tc_fence_after();
-      // K' = K~ / max(|K~|, 1e-12), written over the K tile.
+      // K' = K~ / max(|K~|, 1e-12), written over the K tile (the K~ MMA has read it).
       float ss = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -181,7 +190,8 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[P_KP]);
     }
-    // R = beta (V~ - K'S), written over the V tile; zero for tokens past L.
+    // R = beta (V~ - K'S), written over phi_v^T (the V~ MMA, complete with
+    // the K'S one, has read it); zero for tokens past L.
     if (ok) ok = warp_wait_s(&bars[P_KS], 0, w);
     if (ok) {
       tc_fence_after();
@@ -200,7 +210,7 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             rr[e] = bt * (__uint_as_float(vt[8 * g + e]) - __uint_as_float(ks[8 * g + e]));
           uint4 v = make_uint4(pack_bf16x2(rr[0], rr[1]), pack_bf16x2(rr[2], rr[3]), pack_bf16x2(rr[4], rr[5]),
                                pack_bf16x2(rr[6], rr[7]));
-          *reinterpret_cast<uint4*>(sV + sw128_offset(row, c * 32 + 8 * g)) = v;
+          *reinterpret_cast<uint4*>(sP + sw128_offset(row, c * 32 + 8 * g)) = v;
         }
       }
       fence_async_smem();
