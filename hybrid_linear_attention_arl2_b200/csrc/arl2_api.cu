@@ -153,6 +153,10 @@ struct arl2_state {
   int64_t frame;
   int64_t bytes;
   cudaStream_t last_stream;
+  // The commit's first two state-write kernels run on `side`, forked from and
+  // joined back to the caller's stream (bf16 path).
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_join;
   CUtensorMap tm_phiq, tm_phik_t, tm_phiv_t, tm_s_bf, tm_mqt;
 };
 
@@ -187,6 +191,9 @@ void free_state(arl2_state* h) {
   for (void* p : {h->phi[0], h->phi[1], h->phi[2], (void*)h->S[0], (void*)h->S[1], (void*)h->S_bf, (void*)h->mqt,
                   (void*)h->partial, (void*)h->attn_scratch, (void*)h->attn_ready, (void*)h->err})
     if (p) cudaFree(p);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->side) cudaStreamDestroy(h->side);
   h->magic = 0;
   delete h;
 }
@@ -331,6 +338,9 @@ arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const voi
     alloc(reinterpret_cast<void**>(&h->S_bf), size_t(B) * H * d * d * 2);
     alloc(reinterpret_cast<void**>(&h->mqt), size_t(B) * H * d * d * 2);
     alloc(reinterpret_cast<void**>(&h->partial), size_t(B) * H * h->n_chunks * d * d * sizeof(float));
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
   }
   if (e != cudaSuccess) {
     free_state(h);
@@ -395,6 +405,13 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
   if (!alpha || !beta || !aligned16(alpha) || !aligned16(beta)) return ARL2_ERR_INVALID_ARGUMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
+  const bool fork = h->cfg.dtype == ARL2_BF16;
+  // The state write's first two kernels need nothing from the output's
+  // attention launch and write nothing it reads: they run on the side stream,
+  // forked before that launch, so that their CTAs take the SMs the attention
+  // launch frees in its tail.  The last one replaces MqT, which the attention
+  // launch reads: it runs after the join.
+  if (fork) ARL2_TRY(cudaEventRecord(h->ev_fork, st));
   s = run_attention(h, q, k, v, o, st);  // the output reads S_{N-1}
   if (s != ARL2_OK) return s;
   const arl2_config& c = h->cfg;
@@ -433,8 +450,11 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
     sp.corr = h->corr;
     sp.err = h->err;
     sp.wait_limit_ns = h->wait_ns;
-    ARL2_TRY(launch_state_partial(tk, tv, h->tm_phik_t, h->tm_phiv_t, h->tm_s_bf, sp, c.batch, st));
-    ARL2_TRY(launch_state_finalize(sp, c.batch, st));
+    ARL2_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+    ARL2_TRY(launch_state_partial(tk, tv, h->tm_phik_t, h->tm_phiv_t, h->tm_s_bf, sp, c.batch, h->side));
+    ARL2_TRY(launch_state_finalize(sp, c.batch, h->side));  // S_N and its bf16 copy: not read by the attention
+    ARL2_TRY(cudaEventRecord(h->ev_join, h->side));
+    ARL2_TRY(cudaStreamWaitEvent(st, h->ev_join, 0));
     ARL2_TRY(launch_readout_prep(h->tm_s_bf, h->tm_phiq, sp, c.batch, st));
   }
   h->cur = nxt;
