@@ -143,7 +143,7 @@ struct arl2_state {
   float* S[2];
   int cur;
   __nv_bfloat16* S_bf;   // bf16 copy of S[cur] (bf16 path)
-  __nv_bfloat16* mqt;    // (phi_q S[cur])^T (bf16 path)
+  __nv_bfloat16* mqt;    // two slots of (phi_q S[i])^T, slot cur in use (bf16 path)
   float* partial;        // per-chunk state-write partials (bf16 path)
   int n_chunks;
   float* attn_scratch;   // partial rows of split query blocks (bf16 path)
@@ -153,11 +153,11 @@ struct arl2_state {
   int64_t frame;
   int64_t bytes;
   cudaStream_t last_stream;
-  // The commit's first two state-write kernels run on `side`, forked from and
-  // joined back to the caller's stream (bf16 path).
+  // The commit's state-write kernels run on `side`, forked from and joined
+  // back to the caller's stream (bf16 path).
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
-  CUtensorMap tm_phiq, tm_phik_t, tm_phiv_t, tm_s_bf, tm_mqt;
+  CUtensorMap tm_phiq, tm_phik_t, tm_phiv_t, tm_s_bf, tm_mqt[2];
 };
 
 struct arl2_kv {
@@ -211,10 +211,14 @@ void free_kv(arl2_kv* h) {
     if (e_ != cudaSuccess) return from_cuda(e_); \
   } while (0)
 
+__nv_bfloat16* mqt_slot(const arl2_state* h, int i) {
+  return h->mqt + size_t(i) * h->cfg.batch * h->cfg.heads * h->cfg.head_dim * h->cfg.head_dim;
+}
+
 arl2_status prepare_readout(arl2_state* h, cudaStream_t st) {
   // MqT = (phi_q S[cur])^T from the bf16 copy of S[cur].
   StateParams sp{};
-  sp.mqt = h->mqt;
+  sp.mqt = mqt_slot(h, h->cur);
   sp.heads = h->cfg.heads;
   sp.err = h->err;
   sp.wait_limit_ns = h->wait_ns;
@@ -257,7 +261,7 @@ arl2_status run_attention(arl2_state* h, const void* q, const void* k, const voi
   p.err = h->err;
   p.wait_limit_ns = h->wait_ns;
   if (!attn_partition(p, c.batch, h->sms)) return ARL2_ERR_UNSUPPORTED;
-  ARL2_TRY(launch_attn_bf16(tq, tk, tv, h->tm_mqt, to, p, st));
+  ARL2_TRY(launch_attn_bf16(tq, tk, tv, h->tm_mqt[h->cur], to, p, st));
   return ARL2_OK;
 }
 
@@ -336,7 +340,7 @@ arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const voi
     alloc(reinterpret_cast<void**>(&h->attn_scratch), size_t(h->sms) * 2 * kAttnSlotFloats * sizeof(float));
     alloc(reinterpret_cast<void**>(&h->attn_ready), size_t(h->sms) * 2 * sizeof(unsigned));
     alloc(reinterpret_cast<void**>(&h->S_bf), size_t(B) * H * d * d * 2);
-    alloc(reinterpret_cast<void**>(&h->mqt), size_t(B) * H * d * d * 2);
+    alloc(reinterpret_cast<void**>(&h->mqt), 2 * size_t(B) * H * d * d * 2);
     alloc(reinterpret_cast<void**>(&h->partial), size_t(B) * H * h->n_chunks * d * d * sizeof(float));
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
@@ -364,12 +368,12 @@ arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const voi
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 256, st);
   if (cfg->dtype == ARL2_BF16) {
     if (e == cudaSuccess) e = cudaMemsetAsync(h->S_bf, 0, size_t(B) * H * d * d * 2, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(h->mqt, 0, size_t(B) * H * d * d * 2, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->mqt, 0, 2 * size_t(B) * H * d * d * 2, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(h->attn_ready, 0, size_t(h->sms) * 2 * sizeof(unsigned), st);
     if (e == cudaSuccess &&
         !(make_mat_map(&h->tm_phiq, h->phi[0], H) && make_mat_map(&h->tm_phik_t, h->phi[1], H) &&
           make_mat_map(&h->tm_phiv_t, h->phi[2], H) && make_mat_map(&h->tm_s_bf, h->S_bf, B * H) &&
-          make_mat_map(&h->tm_mqt, h->mqt, B * H)))
+          make_mat_map(&h->tm_mqt[0], mqt_slot(h, 0), B * H) && make_mat_map(&h->tm_mqt[1], mqt_slot(h, 1), B * H)))
       e = cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) {
@@ -406,11 +410,11 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
   const bool fork = h->cfg.dtype == ARL2_BF16;
-  // The state write's first two kernels need nothing from the output's
-  // attention launch and write nothing it reads: they run on the side stream,
-  // forked before that launch, so that their CTAs take the SMs the attention
-  // launch frees in its tail.  The last one replaces MqT, which the attention
-  // launch reads: it runs after the join.
+  // The state write needs nothing from the output's attention launch and
+  // writes nothing it reads (S_N, its bf16 copy and MqT go to the other slots):
+  // its three kernels run on the side stream, forked before that launch, so
+  // that their CTAs take the SMs the attention launch frees in its tail; the
+  // caller's stream joins them before its next work.
   if (fork) ARL2_TRY(cudaEventRecord(h->ev_fork, st));
   s = run_attention(h, q, k, v, o, st);  // the output reads S_{N-1}
   if (s != ARL2_OK) return s;
@@ -443,7 +447,7 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
     sp.partial = h->partial;
     sp.S_next = h->S[nxt];
     sp.S_next_bf = h->S_bf;
-    sp.mqt = h->mqt;
+    sp.mqt = mqt_slot(h, nxt);
     sp.L = c.tokens_per_frame;
     sp.heads = c.heads;
     sp.n_chunks = h->n_chunks;
@@ -452,10 +456,10 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
     sp.wait_limit_ns = h->wait_ns;
     ARL2_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
     ARL2_TRY(launch_state_partial(tk, tv, h->tm_phik_t, h->tm_phiv_t, h->tm_s_bf, sp, c.batch, h->side));
-    ARL2_TRY(launch_state_finalize(sp, c.batch, h->side));  // S_N and its bf16 copy: not read by the attention
+    ARL2_TRY(launch_state_finalize(sp, c.batch, h->side));
+    ARL2_TRY(launch_readout_prep(h->tm_s_bf, h->tm_phiq, sp, c.batch, h->side));
     ARL2_TRY(cudaEventRecord(h->ev_join, h->side));
     ARL2_TRY(cudaStreamWaitEvent(st, h->ev_join, 0));
-    ARL2_TRY(launch_readout_prep(h->tm_s_bf, h->tm_phiq, sp, c.batch, st));
   }
   h->cur = nxt;
   h->frame += 1;

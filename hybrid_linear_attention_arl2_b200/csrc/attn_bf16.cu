@@ -184,7 +184,7 @@ __device__ __forceinline__ void producer(const AttnParams& p, uint64_t* bars, ui
     const int n = s.j1 - s.j0;
     const int ntiles = 2 * n + ((writer && p.has_inter) ? 1 : 0);
     const int x0 = h * 128;
-    {  // L2 prefetch of the next segment's Q tiles
+    auto prefetch_next_q = [&]() {  // L2 prefetch of the next segment's Q tiles
       unsigned u2 = u;
       Seg s2;
       if (next_seg(p, u2, u_end, s2)) {
@@ -195,7 +195,7 @@ __device__ __forceinline__ void producer(const AttnParams& p, uint64_t* bars, ui
           tma_prefetch_l2_3d(tm_q, (s2.bh % p.heads) * 128 + 64, (qt2 + sub) * 128, s2.bh / p.heads);
         }
       }
-    }
+    };
     auto put = [&](int t) -> bool {
       const uint32_t slot = ring % kRing;
       if (ring >= kRing && !wait1(&bars[B_RE + slot], ((ring / kRing) - 1) & 1, w)) return false;
@@ -213,18 +213,36 @@ __device__ __forceinline__ void producer(const AttnParams& p, uint64_t* bars, ui
       ++ring;
       return true;
     };
-    const int pre = min(2, ntiles);
-    for (int t = 0; t < pre; ++t)
-      if (!put(t)) return;
-    for (int sub = 0; sub < (has_b ? 2 : 1); ++sub) {
-      if (q_use[sub] > 0 && !wait1(&bars[B_QE + sub], (q_use[sub] - 1) & 1, w)) return;
+    auto load_q = [&](int sub) -> bool {
+      if (q_use[sub] > 0 && !wait1(&bars[B_QE + sub], (q_use[sub] - 1) & 1, w)) return false;
       uint8_t* dst = sQ + sub * kTile;
       const int row = (qt_a + sub) * 128;
       mbar_expect_tx(&bars[B_QF + sub], kTile);
       tma_load_3d(dst, tm_q, &bars[B_QF + sub], x0, row, b);
       tma_load_3d(dst + kHalf, tm_q, &bars[B_QF + sub], x0 + 64, row, b);
       ++q_use[sub];
+      return true;
+    };
+    if (q_use[0] == 0) {
+      // The launch's first segment: every CTA starts at once and its first
+      // tiles come from HBM, so only what the first MMA needs (K_j0 and Q of
+      // sub-tile A) is requested until it has landed; V_j0, Q of sub-tile B,
+      // the next tiles and the L2 prefetch follow.
+      if (!put(0) || !load_q(0)) return;
+      if (!wait1(&bars[B_QF + 0], 0, w)) return;
+      if (!put(1)) return;
+      if (has_b && !load_q(1)) return;
+      prefetch_next_q();
+      for (int t = 2; t < ntiles; ++t)
+        if (!put(t)) return;
+      continue;
     }
+    prefetch_next_q();
+    const int pre = min(2, ntiles);
+    for (int t = 0; t < pre; ++t)
+      if (!put(t)) return;
+    for (int sub = 0; sub < (has_b ? 2 : 1); ++sub)
+      if (!load_q(sub)) return;
     for (int t = pre; t < ntiles; ++t)
       if (!put(t)) return;
   }
