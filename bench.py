@@ -350,9 +350,10 @@ def run_arl2(args, rank: int, world: int):
 def run_e2e(args, cfg, ds, layer, device, stream, dist, world):
     """Same metric through the C-ABI calls with host buffers: every step copies its
     five passes' Q, K, V and its gates from pinned host memory and reads the five
-    outputs back.  Copies in, compute and copies out run on three streams with
-    two buffer sets, so a pass's inputs cross PCIe while the previous pass
-    computes and its output goes back (PCIe is full duplex)."""
+    outputs back.  Copies in (Q, K and V each on its own stream), compute and
+    copies out run on separate streams with two buffer sets, so a pass's inputs
+    cross PCIe while the previous pass computes and its output goes back (PCIe
+    is full duplex)."""
     import torch
     from hybrid_linear_attention_arl2_b200 import arl2
     B, H, L, d = cfg.batch, cfg.heads, cfg.tokens, cfg.head_dim
@@ -365,7 +366,9 @@ def run_e2e(args, cfg, ds, layer, device, stream, dist, world):
     ga = [torch.empty((B, H), dtype=torch.float32, device=device) for _ in range(nbuf)]
     gb = [torch.empty((B, H, L), dtype=torch.float32, device=device) for _ in range(nbuf)]
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    s_cp = [s_in] + [torch.cuda.Stream(device) for _ in range(2)]  # Q, K, V copies on their own streams
     loaded = [torch.cuda.Event() for _ in range(nbuf)]
+    part = [[torch.cuda.Event() for _ in range(2)] for _ in range(nbuf)]
     computed = [torch.cuda.Event() for _ in range(nbuf)]
     drained = [torch.cuda.Event() for _ in range(nbuf)]
     gates = {}
@@ -382,17 +385,24 @@ def run_e2e(args, cfg, ds, layer, device, stream, dist, world):
     e0.record(s_in)
     stream.wait_event(e0)
     s_out.wait_event(e0)
+    for sc in s_cp[1:]:
+        sc.wait_event(e0)
     i = 0
     for f in range(f0, f0 + steps):
         for p in range(cfg.passes):
             k = i % nbuf
             trip = host_pool[ds.wl.pool_index(0, f, p)]
             if i >= nbuf:
-                s_in.wait_event(computed[k])  # buffer set k is free once pass i - nbuf has computed
-            with torch.cuda.stream(s_in):
-                for dst, src in zip(dq[k], trip):
+                for sc in s_cp:
+                    sc.wait_event(computed[k])  # buffer set k is free once pass i - nbuf has computed
+            for j, (dst, src) in enumerate(zip(dq[k], trip)):
+                with torch.cuda.stream(s_cp[j]):
                     dst.copy_(src, non_blocking=True)
-                    h2d += src.numel() * 2
+                h2d += src.numel() * 2
+            for j in (1, 2):
+                part[k][j - 1].record(s_cp[j])
+                s_in.wait_event(part[k][j - 1])
+            with torch.cuda.stream(s_in):
                 if p >= cfg.queries:
                     a, b = gates[f]
                     ga[k].copy_(a, non_blocking=True)
