@@ -600,7 +600,7 @@ def cpu_oracle_rate(cfg: W.Config, budget_s: float = 12.0, sample_note=True):
 # launch on the single-hybrid-layer-bf16 workload, from one ncu capture of
 # `bench.py --profile-small --no-graphs`; reported only while the kernel sources
 # hash to the value the capture was taken on.
-ATTN_TRAFFIC = {"bytes": 15400704 + 1024, "sources_sha256": "3318e8fc9ead76d6580b6902b599b97d49e7086bab9a490bab115b9abc25811a",
+ATTN_TRAFFIC = {"bytes": 15408128 + 512, "sources_sha256": "1338d0ad68e85518eab263f946646a789e09e516479508343aa1599b31758f38",
                 "capture": "profiles/attn_bf16_kernel_single-hybrid-layer-bf16.md"}
 ATTN_SOURCES = ("hybrid_linear_attention_arl2_b200/csrc/attn_bf16.cu",
                 "hybrid_linear_attention_arl2_b200/csrc/sm100.cuh",
