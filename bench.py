@@ -46,6 +46,9 @@ def _args():
     ap.add_argument("--no-graphs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", action="store_true",
+                    help="the hybrid attention block (QKV and output projections, gates from the tokens) on the "
+                         "single-layer shape (its own JSON line)")
     ap.add_argument("--profile-small", action="store_true",
                     help="a few steps, no extras: for ncu captures of the kernels")
     return ap.parse_args()
@@ -477,6 +480,76 @@ def long_stream_flatness(cfg, ds, device, rank) -> dict:
             "handle_device_bytes": int(handle_bytes)}
 
 
+# ------------------------------------------------------------------ attention block
+def run_block(args, rank: int, world: int) -> dict:
+    """The hybrid attention block on the single-layer shape (B=1, H=12, d=128,
+    L=1560, hidden 1536): per pass X -> Q, K, V (cuBLAS) -> hybrid layer -> O W_o;
+    the commit also forms its gates from X.  Inputs cycle through 40 seeded
+    token matrices (192 MB > L2); CUDA graphs of four frames, as the layer's run."""
+    import dataclasses
+    import torch
+    from hybrid_linear_attention_arl2_b200 import arl2
+    cfg = dataclasses.replace(W.CONFIGS[1], pool=40)
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    arl2.load_library()
+    wl = W.Workload(cfg, seed=cfg.seed + 100 * rank)
+    to = lambda x: torch.from_numpy(x).to(torch.bfloat16).to(device)
+    weights = [to(w) for w in wl.block_weights(0)]
+    phi = [to(p) for p in wl.phi(0)]
+    B, H, L, d = cfg.batch, cfg.heads, cfg.tokens, cfg.head_dim
+    # pool entry i is the tokens of pass i % 5 of frame i // 5
+    xs = [to(wl.block_input(0, i // cfg.passes, i % cfg.passes)) for i in range(cfg.pool)]
+    stream = torch.cuda.Stream(device)
+    period = 4
+    with torch.cuda.stream(stream):
+        blk = arl2.HybridBlock(B, H, L, *weights, *phi, corr_scale=cfg.corr_scale, stream=stream)
+        Y = torch.empty_like(xs[0])
+
+        def frame(f):
+            for p in range(cfg.passes):
+                x = xs[wl.pool_index(0, f, p)]
+                if p < cfg.queries:
+                    arl2.arl2_block_query(blk.handle, x, Y, stream)
+                else:
+                    arl2.arl2_block_commit(blk.handle, x, Y, stream)
+
+        for f in range(args.warmup):
+            frame(f)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for f in range(period):
+                frame(f)
+        stream.synchronize()
+        clocks = ClockSampler(local)
+        torch.cuda.synchronize()
+        clocks.start()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        steps = 0
+        while steps < args.steps:
+            graph.replay()
+            steps += period
+        t1.record(stream)
+        t1.synchronize()
+        clk = clocks.stop()
+        err = blk.last_error()
+        ms = t0.elapsed_time(t1)
+        del graph
+        blk.close()
+    if err:
+        raise RuntimeError(f"device error in the block run: {arl2.STATUS.get(err)}")
+    D = H * d
+    proj = 4 * 2.0 * B * L * D * D
+    fl = frame_flops(cfg)
+    frame_fl = cfg.passes * proj + fl["frame"] + 2.0 * B * L * D * 2 * H
+    value, ms_max = whole_job_rate(ms, steps, world, None, device)
+    return {"frames": steps, "ms": ms_max, "value": value, "clocks": clk, "flops_per_frame": frame_fl,
+            "projection_flops_per_frame": cfg.passes * proj}
+
+
 # ------------------------------------------------------------------ attention stack
 def run_stack(args, rank: int, world: int) -> dict:
     """The 30-layer attention stack: layers [0, 22) hybrid, [22, 30) softmax over a
@@ -665,6 +738,28 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
+    if args.block and args.impl != "reference":
+        res = run_block(args, rank, world)
+        if rank != 0:
+            return
+        pk = peaks()
+        peak_sus, src = (pk["bf16_tflops_sustained"], "of measured") if pk else (1400.0, "of fallback")
+        tf = res["flops_per_frame"] * res["value"] / 1e12
+        line = {
+            "metric": "frames/s per hybrid attention block (1560-token frames, hidden 1536, QKV/out projections "
+                      "+ hybrid layer, 4 query passes + 1 commit)",
+            "value": res["value"], "unit": "frames/s", "n_gpus": world, "steps": res["frames"],
+            "warmup": args.warmup, "ms_per_step": res["ms"] / res["frames"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic, random-init weights",
+            "config": {"workload": "hybrid-attention-block-bf16", "batch": 1, "heads": 12, "head_dim": 128,
+                       "hidden": 1536, "tokens_per_frame": 1560, "passes_per_frame": 5,
+                       "l2": "tokens cycle through 40 seeded 1560 x 1536 matrices (192 MB > 126 MB L2)",
+                       "projections": "cuBLAS GEMMs (bf16, fp32 accumulate)"},
+            "tflops": tf, "pct_bf16_peak": {"value": 100.0 * tf / peak_sus, "basis": f"sustained bf16 {src}"},
+            "clocks": res["clocks"],
+        }
+        print(json.dumps(line), flush=True)
+        return
     if args.config == 3:
         if args.impl == "reference":
             pass  # falls through to the oracle arm below with the single-layer metric

@@ -60,6 +60,11 @@ _SIGS = {
     "arl2_kv_device_bytes": (_I64, [_VP]),
     "arl2_kv_last_error": (_I32, [_VP]),
     "arl2_kv_destroy": (_I32, [_VP]),
+    "arl2_block_init": (_I32, [ctypes.POINTER(arl2_config), _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(_VP)]),
+    "arl2_block_query": (_I32, [_VP, _VP, _VP, _VP]),
+    "arl2_block_commit": (_I32, [_VP, _VP, _VP, _VP]),
+    "arl2_block_layer": (_VP, [_VP]),
+    "arl2_block_destroy": (_I32, [_VP]),
     "arl2_state_write_noalloc": (_I32, [ctypes.POINTER(arl2_config), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                         _VP]),
     "arl2_selftest_wait_timeout": (_I32, [_U64, _VP]),
@@ -196,6 +201,30 @@ def arl2_kv_destroy(h) -> None:
     _check(load_library().arl2_kv_destroy(h), "arl2_kv_destroy")
 
 
+def arl2_block_init(cfg: arl2_config, w_qkv, w_o, w_gate, phi_q, phi_k, phi_v, stream=None) -> int:
+    h = _VP()
+    _check(load_library().arl2_block_init(ctypes.byref(cfg), _ptr(w_qkv), _ptr(w_o), _ptr(w_gate), _ptr(phi_q),
+                                          _ptr(phi_k), _ptr(phi_v), _stream(stream), ctypes.byref(h)),
+           "arl2_block_init")
+    return h.value
+
+
+def arl2_block_query(h, x, y, stream=None) -> None:
+    _check(load_library().arl2_block_query(h, _ptr(x), _ptr(y), _stream(stream)), "arl2_block_query")
+
+
+def arl2_block_commit(h, x, y, stream=None) -> None:
+    _check(load_library().arl2_block_commit(h, _ptr(x), _ptr(y), _stream(stream)), "arl2_block_commit")
+
+
+def arl2_block_layer(h) -> int | None:
+    return load_library().arl2_block_layer(h)
+
+
+def arl2_block_destroy(h) -> None:
+    _check(load_library().arl2_block_destroy(h), "arl2_block_destroy")
+
+
 def arl2_state_write_noalloc(cfg: arl2_config, k, v, phi_k, phi_v, S_prev, alpha, beta, S_next, dev_error,
                              stream=None) -> None:
     """One frame's state write with no handle and no device allocation (its
@@ -323,6 +352,51 @@ class KVLayer:
     def close(self):
         if self.handle:
             arl2_kv_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class HybridBlock:
+    """A hybrid attention block: X W_qkv -> hybrid layer -> O W_o, with the
+    commit's gates from X W_gate (a handle of the C ABI; bf16, head_dim 128)."""
+
+    def __init__(self, batch, heads, tokens, w_qkv, w_o, w_gate, phi_q, phi_k, phi_v, *, softmax_scale=0.0,
+                 corr_scale=-1.0, stream=None):
+        self.cfg = make_config(batch, heads, 128, tokens, ARL2_BF16, softmax_scale, corr_scale, 0)
+        self.handle = arl2_block_init(self.cfg, w_qkv, w_o, w_gate, phi_q, phi_k, phi_v, stream)
+
+    def _out(self, like):
+        import torch
+        return torch.empty_like(like)
+
+    def query(self, x, y=None, stream=None):
+        y = self._out(x) if y is None else y
+        arl2_block_query(self.handle, x, y, stream)
+        return y
+
+    def commit(self, x, y=None, stream=None):
+        y = self._out(x) if y is None else y
+        arl2_block_commit(self.handle, x, y, stream)
+        return y
+
+    def state(self, stream=None):
+        import torch
+        c = self.cfg
+        dst = torch.empty((c.batch, c.heads, c.head_dim, c.head_dim), dtype=torch.float32, device="cuda")
+        arl2_state_get(arl2_block_layer(self.handle), dst, stream)
+        return dst
+
+    def last_error(self) -> int:
+        return arl2_last_error(arl2_block_layer(self.handle))
+
+    def close(self):
+        if self.handle:
+            arl2_block_destroy(self.handle)
             self.handle = None
 
     def __del__(self):

@@ -133,7 +133,7 @@ class Workload:
     Q' = Q @ phi, alpha [B, H], beta [B, H, L].
     """
 
-    _PHI, _GATE_A, _GATE_B, _QKV, _POOL = 1, 2, 3, 4, 5
+    _PHI, _GATE_A, _GATE_B, _QKV, _POOL, _WBLK, _XBLK = 1, 2, 3, 4, 5, 6, 7
 
     def __init__(self, cfg: Config | int, *, seed: int | None = None):
         self.cfg = CONFIGS[cfg] if isinstance(cfg, int) else cfg
@@ -201,3 +201,36 @@ class Workload:
             else:
                 per_stream.append(self._draw_triple(self.seed + b, self._QKV, layer, frame, pas))
         return tuple(np.stack([t[i] for t in per_stream]) for i in range(3))
+
+    # -- hybrid attention block (projections around the layer) ---------------
+    def block_weights(self, layer: int = 0):
+        """(W_qkv [D, 3D], W_o [D, D], W_gate [D, 2H]) of one block, D = H * d,
+        entries N(0, 1/D): unit-variance tokens give unit-variance Q, K, V."""
+        c = self.cfg
+        D = c.heads * c.head_dim
+        rng = _rng(self.seed, self._WBLK, layer)
+        s = np.float32(1.0 / np.sqrt(D))
+        w_qkv = self._store(rng.standard_normal((D, 3 * D), dtype=np.float32) * s)
+        w_o = self._store(rng.standard_normal((D, D), dtype=np.float32) * s)
+        w_gate = self._store(rng.standard_normal((D, 2 * c.heads), dtype=np.float32) * s)
+        return w_qkv, w_o, w_gate
+
+    def _draw_x(self, *words: int) -> np.ndarray:
+        c = self.cfg
+        rng = _rng(*words)
+        return self._store(rng.standard_normal((c.tokens, c.heads * c.head_dim), dtype=np.float32))
+
+    def block_input(self, layer: int, frame: int, pas: int) -> np.ndarray:
+        """X [B, L, D] of one pass of a block: N(0, 1) tokens (pool entries, as
+        for Q/K/V, when the configuration has a pool)."""
+        c = self.cfg
+        rows = []
+        for b in range(c.batch):
+            if c.pool:
+                key = ("x", b, self.pool_index(layer, frame, pas))
+                if key not in self._pool:
+                    self._pool[key] = self._draw_x(self.seed + b, self._XBLK, key[2])
+                rows.append(self._pool[key])
+            else:
+                rows.append(self._draw_x(self.seed + b, self._XBLK, layer, frame, pas))
+        return np.stack(rows)

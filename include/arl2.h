@@ -144,6 +144,43 @@ int64_t arl2_kv_device_bytes(arl2_kv_t kv);
 arl2_status arl2_kv_last_error(arl2_kv_t kv);
 arl2_status arl2_kv_destroy(arl2_kv_t kv);
 
+/* ---- Hybrid attention block (the layer around the hot path) ----------------
+ * One hybrid layer with the projections a DiT attention block puts around it
+ * (ARL2 summary, section 2.1: the frozen pretrained Q/K/V projections feed
+ * both branches; alpha and beta are per-token learned projections), bf16 with
+ * fp32 accumulation, for a hidden size D = H * 128:
+ *   Q = X W_qkv[:, 0:D],  K = X W_qkv[:, D:2D],  V = X W_qkv[:, 2D:3D]
+ *   O = the hybrid layer's output on (Q, K, V)  (arl2_frame_query / commit)
+ *   Y = O W_o
+ * and, on the commit (clean) pass, the gates from the tokens:
+ *   alpha[b][h]   = sigmoid( mean over t of (X W_gate)[b][t][h] )
+ *   beta[b][h][t] = sigmoid( (X W_gate)[b][t][H + h] )
+ * (the pages fix neither the gates' inputs nor their pooling; a head-wise
+ * alpha from the frame's mean token and a per-token beta are this build's
+ * reading).  No position encoding is applied: Q and K enter the layer as
+ * projected.  The four projections are plain GEMMs (cuBLAS, fp32 accumulate,
+ * bf16 results; W_gate's result is kept in fp32).
+ *   cfg     : bf16 configuration with head_dim 128 (hidden D = heads * 128).
+ *   w_qkv   : device bf16 [D, 3D] row-major (X W: y_j = sum_i x_i W[i][j]);
+ *   w_o     : device bf16 [D, D];  w_gate : device bf16 [D, 2H] (alpha columns
+ *             first, then beta columns);  phi_q, phi_k, phi_v as for
+ *             arl2_state_init.  Every weight is copied at init.
+ *   x, y    : device bf16 [B, L, D] (token-major; y must not overlap x).
+ * The block owns one hybrid-layer handle (its state, KV-free) and its work
+ * space (Q, K, V, O, gates: about 5 * B * L * D * 2 bytes plus cuBLAS's
+ * 32 MiB workspace, fixed at init).  arl2_block_layer() returns that handle
+ * for state get/set, last_error and the device-byte count; it is destroyed
+ * with the block.  Errors: INVALID_ARGUMENT, UNSUPPORTED (not bf16 / d != 128),
+ * OUT_OF_MEMORY, CUDA. */
+typedef struct arl2_block* arl2_block_t;
+arl2_status arl2_block_init(const arl2_config* cfg, const void* w_qkv, const void* w_o, const void* w_gate,
+                            const void* phi_q, const void* phi_k, const void* phi_v, void* stream,
+                            arl2_block_t* out);
+arl2_status arl2_block_query(arl2_block_t blk, const void* x, void* y, void* stream);
+arl2_status arl2_block_commit(arl2_block_t blk, const void* x, void* y, void* stream);
+arl2_state_t arl2_block_layer(arl2_block_t blk);
+arl2_status arl2_block_destroy(arl2_block_t blk);
+
 /* ---- State write without allocation ---------------------------------------
  * The paper has no counterpart to this call; it is a deployment aid.  Some
  * callers cannot call cudaMalloc: code that runs while a CUDA graph is being

@@ -159,3 +159,51 @@ def stream_reference(inputs, frames, queries, corr_scale, phi, S0=None, scale=No
         outs.append(frame_out)
         states.append(S)
     return outs, states
+
+
+# ---------------------------------------------------------------- attention block
+def block_projections(X, w_qkv, heads):
+    """Q, K, V of a hybrid attention block: the frozen pretrained projections
+    in front of both branches (ARL2 summary, §2.1), X [B, L, D] times the
+    three column blocks of w_qkv [D, 3D], each reshaped to [B, L, H, D/H]."""
+    X, w = _f64(X), _f64(w_qkv)
+    B, L, D = X.shape
+    d = D // heads
+    QKV = X @ w
+    return tuple(QKV[..., i * D:(i + 1) * D].reshape(B, L, heads, d) for i in range(3))
+
+
+def block_gates(X, w_gate, heads):
+    """The commit's gates from the tokens (ARL2 summary, §2.1: alpha and beta
+    are learned projections of the tokens).  Reading of this build: the first
+    H columns of X w_gate give alpha from the frame's mean token, one per head
+    (head-wise gating, §4); the last H give one beta per token and head:
+        alpha[b][h] = sigmoid(mean_t (X w_gate)[b][t][h]),
+        beta[b][h][t] = sigmoid((X w_gate)[b][t][H + h])."""
+    G = _f64(X) @ _f64(w_gate)
+    sig = lambda z: 1.0 / (1.0 + np.exp(-z))
+    alpha = sig(G[..., :heads].mean(axis=1))
+    beta = np.transpose(sig(G[..., heads:]), (0, 2, 1))
+    return alpha, beta
+
+
+def block_query(S, X, weights, phi, scale=None):
+    """A denoising step of the block: Y = frame_query(Q, K, V) W_o."""
+    w_qkv, w_o, _ = weights
+    H = phi[0].shape[0]
+    Q, K, V = block_projections(X, w_qkv, H)
+    O = frame_query(S, Q, K, V, phi, scale)
+    B, L = O.shape[:2]
+    return O.reshape(B, L, -1) @ _f64(w_o)
+
+
+def block_commit(S, X, weights, phi, corr_scale=1.0, scale=None):
+    """The clean pass of the block: gates from X, the layer's commit, Y = O W_o.
+    Returns (Y [B, L, D], S_N)."""
+    w_qkv, w_o, w_gate = weights
+    H = phi[0].shape[0]
+    Q, K, V = block_projections(X, w_qkv, H)
+    alpha, beta = block_gates(X, w_gate, H)
+    O, S_new = frame_commit(S, Q, K, V, phi, alpha, beta, corr_scale, scale)
+    B, L = O.shape[:2]
+    return O.reshape(B, L, -1) @ _f64(w_o), S_new

@@ -90,3 +90,21 @@ def test_noalloc_state_write_host_checks(lib):
     assert call(arl2.make_config(1, 2, 128, 16, arl2.ARL2_BF16), same) == 1
     assert call(arl2.make_config(4, 12, 128, 1560, arl2.ARL2_BF16)) == 7    # 4 streams x 1560 tokens
     assert arl2.arl2_status_string(7).startswith("sizes exceed")
+
+
+def test_block_host_validation(lib):
+    """The block's argument checks run before any CUDA call."""
+    ok = arl2.make_config(1, 2, 128, 64, arl2.ARL2_BF16)
+    h = ctypes.c_void_p()
+    w = 16  # any 16-byte-aligned non-null address: rejected before use
+    assert lib.arl2_block_init(ctypes.byref(ok), w, w, w, w, w, w, None, None) == 1      # no out pointer
+    assert lib.arl2_block_init(ctypes.byref(ok), None, w, w, w, w, w, None, ctypes.byref(h)) == 1
+    assert lib.arl2_block_init(ctypes.byref(ok), 17, w, w, w, w, w, None, ctypes.byref(h)) == 1  # misaligned
+    f32 = arl2.make_config(1, 2, 128, 64, arl2.ARL2_F32)
+    assert lib.arl2_block_init(ctypes.byref(f32), w, w, w, w, w, w, None, ctypes.byref(h)) == 2
+    d64 = arl2.make_config(1, 2, 64, 64, arl2.ARL2_BF16)
+    assert lib.arl2_block_init(ctypes.byref(d64), w, w, w, w, w, w, None, ctypes.byref(h)) == 2
+    assert lib.arl2_block_query(None, w, w, None) == 1
+    assert lib.arl2_block_commit(12345, w, w, None) == 1
+    assert lib.arl2_block_destroy(None) == 1
+    assert lib.arl2_block_layer(None) is None
