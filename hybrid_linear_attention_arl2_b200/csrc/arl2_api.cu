@@ -87,8 +87,10 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
 
 // Token-major activations [B, tokens, H, 128] as a map over (H*128, tokens, B),
 // boxes of 64 columns x `rows` tokens.
-bool make_act_map(CUtensorMap* m, const void* base, int B, int64_t tokens, int H, uint32_t rows = 128) {
-  const uint64_t row = uint64_t(H) * 128 * 2;
+// `ld`: elements from one token's row to the next (0: H * 128, contiguous).
+bool make_act_map(CUtensorMap* m, const void* base, int B, int64_t tokens, int H, uint32_t rows = 128,
+                  int64_t ld = 0) {
+  const uint64_t row = uint64_t(ld > 0 ? ld : int64_t(H) * 128) * 2;
   return make_map(m, base, uint64_t(H) * 128, uint64_t(tokens), uint64_t(B), row, row * uint64_t(tokens), rows);
 }
 
@@ -226,7 +228,8 @@ arl2_status prepare_readout(arl2_state* h, cudaStream_t st) {
   return ARL2_OK;
 }
 
-arl2_status run_attention(arl2_state* h, const void* q, const void* k, const void* v, void* o, cudaStream_t st) {
+arl2_status run_attention(arl2_state* h, const void* q, const void* k, const void* v, void* o, cudaStream_t st,
+                          int64_t ld = 0) {
   const arl2_config& c = h->cfg;
   if (c.dtype == ARL2_F32) {
     F32AttnParams p{};
@@ -245,9 +248,9 @@ arl2_status run_attention(arl2_state* h, const void* q, const void* k, const voi
     return ARL2_OK;
   }
   CUtensorMap tq, tk, tv, to;
-  if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads) ||
-      !make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads) ||
-      !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads) ||
+  if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
+      !make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
+      !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
       !make_act_map(&to, o, c.batch, c.tokens_per_frame, c.heads, 32))
     return ARL2_ERR_CUDA;
   AttnParams p{};
@@ -270,11 +273,20 @@ bool overlaps(const void* a, const void* b, size_t n) {
   return x < y + n && y < x + n;
 }
 
-arl2_status check_io(const arl2_config& c, const void* q, const void* k, const void* v, const void* o) {
+arl2_status check_io(const arl2_config& c, const void* q, const void* k, const void* v, const void* o,
+                     int64_t ld = 0) {
   if (!q || !k || !v || !o) return ARL2_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ARL2_ERR_INVALID_ARGUMENT;
-  const size_t n = size_t(c.batch) * c.tokens_per_frame * c.heads * c.head_dim * (c.dtype == ARL2_F32 ? 4 : 2);
-  if (overlaps(o, q, n) || overlaps(o, k, n) || overlaps(o, v, n)) return ARL2_ERR_INVALID_ARGUMENT;
+  const size_t esz = c.dtype == ARL2_F32 ? 4 : 2;
+  const size_t rows = size_t(c.batch) * c.tokens_per_frame, row = size_t(c.heads) * c.head_dim;
+  const size_t n = rows * row * esz;
+  // a strided view spans (rows - 1) pitches plus one row
+  const size_t n_in = ld > 0 ? ((rows - 1) * size_t(ld) + row) * esz : n;
+  auto clash = [&](const void* in) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(o), b = reinterpret_cast<uintptr_t>(in);
+    return a < b + n_in && b < a + n;
+  };
+  if (clash(q) || clash(k) || clash(v)) return ARL2_ERR_INVALID_ARGUMENT;
   return ARL2_OK;
 }
 
@@ -393,21 +405,37 @@ arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const voi
 }
 
 arl2_status arl2_frame_query(arl2_state_t h, const void* q, const void* k, const void* v, void* o, void* stream) {
-  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
-  arl2_status s = check_io(h->cfg, q, k, v, o);
-  if (s != ARL2_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  h->last_stream = st;
-  return run_attention(h, q, k, v, o, st);
+  return arl2::layer_query_ld(h, q, k, v, 0, o, static_cast<cudaStream_t>(stream));
 }
 
 arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, const void* v, const float* alpha,
                               const float* beta, void* o, void* stream) {
+  return arl2::layer_commit_ld(h, q, k, v, 0, alpha, beta, o, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace arl2 {
+
+arl2_status layer_query_ld(arl2_state* h, const void* q, const void* k, const void* v, int64_t ld, void* o,
+                           cudaStream_t st) {
   if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
-  arl2_status s = check_io(h->cfg, q, k, v, o);
+  if (ld != 0 && (h->cfg.dtype != ARL2_BF16 || ld < int64_t(h->cfg.heads) * 128 || ld % 8 != 0))
+    return ARL2_ERR_INVALID_ARGUMENT;
+  arl2_status s = check_io(h->cfg, q, k, v, o, ld);
+  if (s != ARL2_OK) return s;
+  h->last_stream = st;
+  return run_attention(h, q, k, v, o, st, ld);
+}
+
+arl2_status layer_commit_ld(arl2_state* h, const void* q, const void* k, const void* v, int64_t ld, const float* alpha,
+                            const float* beta, void* o, cudaStream_t st) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (ld != 0 && (h->cfg.dtype != ARL2_BF16 || ld < int64_t(h->cfg.heads) * 128 || ld % 8 != 0))
+    return ARL2_ERR_INVALID_ARGUMENT;
+  arl2_status s = check_io(h->cfg, q, k, v, o, ld);
   if (s != ARL2_OK) return s;
   if (!alpha || !beta || !aligned16(alpha) || !aligned16(beta)) return ARL2_ERR_INVALID_ARGUMENT;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
   const bool fork = h->cfg.dtype == ARL2_BF16;
   // The state write needs nothing from the output's attention launch and
@@ -416,7 +444,7 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
   // that their CTAs take the SMs the attention launch frees in its tail; the
   // caller's stream joins them before its next work.
   if (fork) ARL2_TRY(cudaEventRecord(h->ev_fork, st));
-  s = run_attention(h, q, k, v, o, st);  // the output reads S_{N-1}
+  s = run_attention(h, q, k, v, o, st, ld);  // the output reads S_{N-1}
   if (s != ARL2_OK) return s;
   const arl2_config& c = h->cfg;
   const int nxt = h->cur ^ 1;
@@ -437,8 +465,8 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
     ARL2_TRY(launch_f32_commit(p, c.batch, st));
   } else {
     CUtensorMap tk, tv;
-    if (!make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads) ||
-        !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads))
+    if (!make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
+        !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads, 128, ld))
       return ARL2_ERR_CUDA;
     StateParams sp{};
     sp.S_prev = h->S[h->cur];
@@ -465,6 +493,10 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
   h->frame += 1;
   return ARL2_OK;
 }
+
+}  // namespace arl2
+
+extern "C" {
 
 arl2_status arl2_state_get(arl2_state_t h, float* dst, int64_t* frame, void* stream) {
   if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;

@@ -8,8 +8,11 @@
 // (ARL2 summary, section 2.1: the frozen pretrained Q/K/V projections feed
 // both branches; alpha and beta are per-token learned projections; the
 // pooling of alpha over the frame is this build's reading.)  The projections
-// are plain GEMMs on cuBLAS (bf16 in, fp32 accumulate); the hybrid layer is
-// this library's own handle; the gates are one small kernel here.
+// are plain GEMMs on cuBLAS (bf16 in, fp32 accumulate): one GEMM against the
+// column-concatenated [W_qkv | W_gate] gives Q, K, V and the gates' logits
+// side by side in each token's row, which the layer reads as strided views;
+// the hybrid layer is this library's own handle; the gates are one small
+// kernel here.
 
 #include <cublas_v2.h>
 
@@ -23,16 +26,18 @@
 
 namespace arl2 {
 
-// alpha[b][h] = sigmoid(mean_t g[b][t][h]); beta[b][h][t] = sigmoid(g[b][t][H + h]).
-// One CTA per (stream, head); the mean is a fixed-order reduction.
-__global__ void __launch_bounds__(256) block_gates_kernel(const float* __restrict__ g, float* __restrict__ alpha,
-                                                          float* __restrict__ beta, int L, int H) {
+// alpha[b][h] = sigmoid(mean_t g[b][t][h]); beta[b][h][t] = sigmoid(g[b][t][H + h]),
+// g bf16 with token rows `ld` elements apart.  One CTA per (stream, head); the
+// mean is a fixed-order reduction.
+__global__ void __launch_bounds__(256) block_gates_kernel(const __nv_bfloat16* __restrict__ g, int64_t ld,
+                                                          float* __restrict__ alpha, float* __restrict__ beta, int L,
+                                                          int H) {
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   float sum = 0.f;
   for (int t = threadIdx.x; t < L; t += blockDim.x) {
-    const float* row = g + (size_t(b) * L + t) * 2 * H;
-    sum += row[h];
-    beta[size_t(bh) * L + t] = 1.f / (1.f + expf(-row[H + h]));
+    const __nv_bfloat16* row = g + (size_t(b) * L + t) * ld;
+    sum += __bfloat162float(row[h]);
+    beta[size_t(bh) * L + t] = 1.f / (1.f + expf(-__bfloat162float(row[H + h])));
   }
   __shared__ float part[8];
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -64,14 +69,11 @@ struct arl2_block {
   arl2_config cfg;
   arl2_state_t layer;
   cublasHandle_t blas;
-  void* w_qkv;
+  int64_t ldw;   // columns of w_all and qkvg: 3D, then 2H gate columns, padded to a multiple of 8
+  void* w_all;   // [D, ldw] bf16: W_qkv | W_gate | 0
   void* w_o;
-  void* w_gate;
-  void* q;
-  void* k;
-  void* v;
+  void* qkvg;    // [B * L, ldw] bf16: Q | K | V | gate logits per token
   void* o;
-  float* g;
   float* alpha;
   float* beta;
   void* ws;
@@ -93,8 +95,7 @@ bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0
 void free_block(arl2_block* b) {
   if (b->layer) arl2_state_destroy(b->layer);
   if (b->blas) cublasDestroy(b->blas);
-  for (void* p : {b->w_qkv, b->w_o, b->w_gate, b->q, b->k, b->v, b->o, (void*)b->g, (void*)b->alpha,
-                  (void*)b->beta, b->ws})
+  for (void* p : {b->w_all, b->w_o, b->qkvg, b->o, (void*)b->alpha, (void*)b->beta, b->ws})
     if (p) cudaFree(p);
   b->magic = 0;
   delete b;
@@ -109,15 +110,12 @@ bool gemm(cublasHandle_t h, int M, int N, int K, const void* A, int lda, const v
                       ctype, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS;
 }
 
-// Q, K, V = X W_qkv column blocks.
-arl2_status project_qkv(arl2_block* b, const void* x, cudaStream_t st) {
+// Q | K | V | gate logits = X [W_qkv | W_gate], one token row each.
+arl2_status project_in(arl2_block* b, const void* x, cudaStream_t st) {
   const int D = b->cfg.heads * b->cfg.head_dim, M = b->cfg.batch * b->cfg.tokens_per_frame;
   if (cublasSetStream(b->blas, st) != CUBLAS_STATUS_SUCCESS) return ARL2_ERR_CUDA;
-  const auto* w = static_cast<const __nv_bfloat16*>(b->w_qkv);
-  void* out[3] = {b->q, b->k, b->v};
-  for (int i = 0; i < 3; ++i)
-    if (!gemm(b->blas, M, D, D, x, D, w + size_t(i) * D, 3 * D, out[i], D, CUDA_R_16BF)) return ARL2_ERR_CUDA;
-  return ARL2_OK;
+  const int ldw = int(b->ldw);
+  return gemm(b->blas, M, ldw, D, x, D, b->w_all, ldw, b->qkvg, ldw, CUDA_R_16BF) ? ARL2_OK : ARL2_ERR_CUDA;
 }
 
 arl2_status project_out(arl2_block* b, void* y) {
@@ -161,24 +159,26 @@ arl2_status arl2_block_init(const arl2_config* cfg, const void* w_qkv, const voi
   }
   const size_t D = size_t(cfg->heads) * cfg->head_dim, H = cfg->heads;
   const size_t M = size_t(cfg->batch) * cfg->tokens_per_frame;
+  b->ldw = int64_t(3 * D + ((2 * H + 7) / 8) * 8);
+  const size_t ldw = size_t(b->ldw);
   cudaError_t e = cudaSuccess;
   auto alloc = [&](void** p, size_t n) {
     if (e == cudaSuccess) e = cudaMalloc(p, n);
   };
-  alloc(&b->w_qkv, D * 3 * D * 2);
+  alloc(&b->w_all, D * ldw * 2);
   alloc(&b->w_o, D * D * 2);
-  alloc(&b->w_gate, D * 2 * H * 2);
-  alloc(&b->q, M * D * 2);
-  alloc(&b->k, M * D * 2);
-  alloc(&b->v, M * D * 2);
+  alloc(&b->qkvg, M * ldw * 2);
   alloc(&b->o, M * D * 2);
-  alloc(reinterpret_cast<void**>(&b->g), M * 2 * H * sizeof(float));
   alloc(reinterpret_cast<void**>(&b->alpha), size_t(cfg->batch) * H * sizeof(float));
   alloc(reinterpret_cast<void**>(&b->beta), M * H * sizeof(float));
   alloc(&b->ws, kBlasWorkspace);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(b->w_qkv, w_qkv, D * 3 * D * 2, cudaMemcpyDeviceToDevice, st);
+  auto* wa = static_cast<__nv_bfloat16*>(b->w_all);
+  if (e == cudaSuccess) e = cudaMemsetAsync(b->w_all, 0, D * ldw * 2, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpy2DAsync(wa, ldw * 2, w_qkv, 3 * D * 2, 3 * D * 2, D, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpy2DAsync(wa + 3 * D, ldw * 2, w_gate, 2 * H * 2, 2 * H * 2, D, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(b->w_o, w_o, D * D * 2, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(b->w_gate, w_gate, D * 2 * H * 2, cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) {
     free_block(b);
     return from_cuda_e(e);
@@ -209,8 +209,10 @@ arl2_status arl2_block_query(arl2_block_t b, const void* x, void* y, void* strea
   arl2_status s = check_xy(b, x, y);
   if (s != ARL2_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = project_qkv(b, x, st)) != ARL2_OK) return s;
-  if ((s = arl2_frame_query(b->layer, b->q, b->k, b->v, b->o, stream)) != ARL2_OK) return s;
+  if ((s = project_in(b, x, st)) != ARL2_OK) return s;
+  const int D = b->cfg.heads * b->cfg.head_dim;
+  const auto* in = static_cast<const __nv_bfloat16*>(b->qkvg);
+  if ((s = arl2::layer_query_ld(b->layer, in, in + D, in + 2 * D, b->ldw, b->o, st)) != ARL2_OK) return s;
   return project_out(b, y);
 }
 
@@ -219,12 +221,14 @@ arl2_status arl2_block_commit(arl2_block_t b, const void* x, void* y, void* stre
   arl2_status s = check_xy(b, x, y);
   if (s != ARL2_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = project_qkv(b, x, st)) != ARL2_OK) return s;
-  const int D = b->cfg.heads * b->cfg.head_dim, H = b->cfg.heads, M = b->cfg.batch * b->cfg.tokens_per_frame;
-  if (!gemm(b->blas, M, 2 * H, D, x, D, b->w_gate, 2 * H, b->g, 2 * H, CUDA_R_32F)) return ARL2_ERR_CUDA;
-  arl2::block_gates_kernel<<<b->cfg.batch * H, 256, 0, st>>>(b->g, b->alpha, b->beta, b->cfg.tokens_per_frame, H);
+  if ((s = project_in(b, x, st)) != ARL2_OK) return s;
+  const int D = b->cfg.heads * b->cfg.head_dim, H = b->cfg.heads;
+  const auto* in = static_cast<const __nv_bfloat16*>(b->qkvg);
+  arl2::block_gates_kernel<<<b->cfg.batch * H, 256, 0, st>>>(in + 3 * D, b->ldw, b->alpha, b->beta,
+                                                             b->cfg.tokens_per_frame, H);
   if (cudaGetLastError() != cudaSuccess) return ARL2_ERR_CUDA;
-  if ((s = arl2_frame_commit(b->layer, b->q, b->k, b->v, b->alpha, b->beta, b->o, stream)) != ARL2_OK) return s;
+  if ((s = arl2::layer_commit_ld(b->layer, in, in + D, in + 2 * D, b->ldw, b->alpha, b->beta, b->o, st)) != ARL2_OK)
+    return s;
   return project_out(b, y);
 }
 

@@ -158,8 +158,9 @@ arl2_status arl2_kv_destroy(arl2_kv_t kv);
  * (the pages fix neither the gates' inputs nor their pooling; a head-wise
  * alpha from the frame's mean token and a per-token beta are this build's
  * reading).  No position encoding is applied: Q and K enter the layer as
- * projected.  The four projections are plain GEMMs (cuBLAS, fp32 accumulate,
- * bf16 results; W_gate's result is kept in fp32).
+ * projected.  The projections are plain GEMMs (cuBLAS, fp32 accumulate, bf16
+ * results): one against [W_qkv | W_gate] (the layer reads Q, K and V as strided
+ * views of its rows), one against W_o.
  *   cfg     : bf16 configuration with head_dim 128 (hidden D = heads * 128).
  *   w_qkv   : device bf16 [D, 3D] row-major (X W: y_j = sum_i x_i W[i][j]);
  *   w_o     : device bf16 [D, D];  w_gate : device bf16 [D, 2H] (alpha columns
