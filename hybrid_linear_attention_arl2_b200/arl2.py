@@ -47,6 +47,8 @@ _SIGS = {
     "arl2_state_init": (_I32, [ctypes.POINTER(arl2_config), _VP, _VP, _VP, _VP, ctypes.POINTER(_VP)]),
     "arl2_frame_query": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP]),
     "arl2_frame_commit": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "arl2_frame_query_strided": (_I32, [_VP, _VP, _VP, _VP, _I64, _VP, _VP]),
+    "arl2_frame_commit_strided": (_I32, [_VP, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP]),
     "arl2_state_get": (_I32, [_VP, _VP, ctypes.POINTER(_I64), _VP]),
     "arl2_state_set": (_I32, [_VP, _VP, _I64, _VP]),
     "arl2_last_error": (_I32, [_VP]),
@@ -142,6 +144,16 @@ def arl2_frame_query(h, q, k, v, o, stream=None) -> None:
 def arl2_frame_commit(h, q, k, v, alpha, beta, o, stream=None) -> None:
     _check(load_library().arl2_frame_commit(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
                                             _stream(stream)), "arl2_frame_commit")
+
+
+def arl2_frame_query_strided(h, q, k, v, ld, o, stream=None) -> None:
+    _check(load_library().arl2_frame_query_strided(h, _ptr(q), _ptr(k), _ptr(v), int(ld), _ptr(o), _stream(stream)),
+           "arl2_frame_query_strided")
+
+
+def arl2_frame_commit_strided(h, q, k, v, ld, alpha, beta, o, stream=None) -> None:
+    _check(load_library().arl2_frame_commit_strided(h, _ptr(q), _ptr(k), _ptr(v), int(ld), _ptr(alpha), _ptr(beta),
+                                                    _ptr(o), _stream(stream)), "arl2_frame_commit_strided")
 
 
 def arl2_state_get(h, dst, stream=None) -> int:

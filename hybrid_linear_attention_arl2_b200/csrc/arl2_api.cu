@@ -413,6 +413,18 @@ arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, cons
   return arl2::layer_commit_ld(h, q, k, v, 0, alpha, beta, o, static_cast<cudaStream_t>(stream));
 }
 
+arl2_status arl2_frame_query_strided(arl2_state_t h, const void* q, const void* k, const void* v, int64_t ld,
+                                     void* o, void* stream) {
+  if (ld < 0) return ARL2_ERR_INVALID_ARGUMENT;
+  return arl2::layer_query_ld(h, q, k, v, ld, o, static_cast<cudaStream_t>(stream));
+}
+
+arl2_status arl2_frame_commit_strided(arl2_state_t h, const void* q, const void* k, const void* v, int64_t ld,
+                                      const float* alpha, const float* beta, void* o, void* stream) {
+  if (ld < 0) return ARL2_ERR_INVALID_ARGUMENT;
+  return arl2::layer_commit_ld(h, q, k, v, ld, alpha, beta, o, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"
 
 namespace arl2 {

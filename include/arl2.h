@@ -106,6 +106,19 @@ arl2_status arl2_frame_query(arl2_state_t h, const void* q, const void* k, const
 arl2_status arl2_frame_commit(arl2_state_t h, const void* q, const void* k, const void* v,
                               const float* alpha, const float* beta, void* o, void* stream);
 
+/* Query and commit with Q, K and V as strided views of wider token rows, as
+ * a fused QKV projection writes them ([B, L, 3 * H * d] with K and V at column
+ * offsets H*d and 2*H*d): token rows are `ld` elements apart instead of H*d.
+ * bf16 handles only; ld >= H * d and a multiple of 8 (16-byte pitch); ld = 0
+ * means contiguous, the same as arl2_frame_query / arl2_frame_commit, which
+ * these calls equal bit for bit on the same values.  O stays contiguous and
+ * must not overlap the views' spans.  Errors: INVALID_ARGUMENT (also for an
+ * f32 handle with ld != 0), CUDA. */
+arl2_status arl2_frame_query_strided(arl2_state_t h, const void* q, const void* k, const void* v, int64_t ld,
+                                     void* o, void* stream);
+arl2_status arl2_frame_commit_strided(arl2_state_t h, const void* q, const void* k, const void* v, int64_t ld,
+                                      const float* alpha, const float* beta, void* o, void* stream);
+
 /* Copy the current state (float32 [B, H, d, d]) to device memory `dst` and the
  * frame counter to *frame (host pointer, may be null).  Synchronous with
  * respect to `stream` for *frame only; the copy is enqueued on `stream`. */

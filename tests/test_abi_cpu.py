@@ -108,3 +108,9 @@ def test_block_host_validation(lib):
     assert lib.arl2_block_commit(12345, w, w, None) == 1
     assert lib.arl2_block_destroy(None) == 1
     assert lib.arl2_block_layer(None) is None
+
+
+def test_strided_calls_host_validation(lib):
+    assert lib.arl2_frame_query_strided(None, 16, 16, 16, 0, 32, None) == 1
+    assert lib.arl2_frame_commit_strided(None, 16, 16, 16, 384, 16, 16, 32, None) == 1
+    assert lib.arl2_frame_query_strided(12345, 16, 16, 16, -8, 32, None) == 1

@@ -277,3 +277,36 @@ def test_fma_pipe_exp2_against_cuda_exp2f():
     yi = torch.empty_like(ints)
     arl2.arl2_selftest_exp2(ints, yi)
     assert torch.equal(yi / torch.exp2(ints), torch.full_like(ints, yi[125].item()))
+
+
+def test_strided_views_equal_contiguous_bitwise():
+    """Q, K, V read as strided views of [B, L, 3D] rows (a fused QKV
+    projection's layout) give the same bits as the contiguous calls."""
+    cfg = small_config(B=2, H=2, L=200, frames=1, queries=1, seed=41)
+    wl = W.Workload(cfg)
+    a_lay, _ = make_layer(cfg, wl)
+    b_lay, _ = make_layer(cfg, wl)
+    Q, K, V = (dev(x, "bf16") for x in wl.qkv(0, 0, 0))
+    B, L, H, d = Q.shape
+    D = H * d
+    fused = torch.cat([Q.reshape(B, L, D), K.reshape(B, L, D), V.reshape(B, L, D)], dim=2).contiguous()
+    alpha = torch.from_numpy(wl.alpha(0, 0)).cuda()
+    beta = torch.from_numpy(wl.beta(0, 0)).cuda()
+    o1, o2 = torch.empty_like(Q), torch.empty_like(Q)
+    for commit in (False, True):
+        if commit:
+            arl2.arl2_frame_commit(a_lay.handle, Q, K, V, alpha, beta, o1)
+            arl2.arl2_frame_commit_strided(b_lay.handle, fused, fused[..., D:], fused[..., 2 * D:], 3 * D, alpha,
+                                           beta, o2)
+        else:
+            arl2.arl2_frame_query(a_lay.handle, Q, K, V, o1)
+            arl2.arl2_frame_query_strided(b_lay.handle, fused, fused[..., D:], fused[..., 2 * D:], 3 * D, o2)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2)
+    assert torch.equal(a_lay.state(), b_lay.state())
+    with pytest.raises(arl2.Arl2Error):  # pitch below a row
+        arl2.arl2_frame_query_strided(b_lay.handle, fused, fused[..., D:], fused[..., 2 * D:], D - 8, o2)
+    with pytest.raises(arl2.Arl2Error):  # pitch not a multiple of 8 elements
+        arl2.arl2_frame_query_strided(b_lay.handle, fused, fused[..., D:], fused[..., 2 * D:], 3 * D + 4, o2)
+    a_lay.close()
+    b_lay.close()
