@@ -310,3 +310,45 @@ def test_strided_views_equal_contiguous_bitwise():
         arl2.arl2_frame_query_strided(b_lay.handle, fused, fused[..., D:], fused[..., 2 * D:], 3 * D + 4, o2)
     a_lay.close()
     b_lay.close()
+
+
+def test_update_with_zero_beta_is_pure_decay_bitwise():
+    """beta = 0: S_N = alpha S_{N-1} exactly (ARL2 summary, section 2.1 state
+    update; the fp32 product alpha * S, rounded once)."""
+    cfg = small_config(B=2, H=3, L=150, frames=1, queries=1, seed=43)
+    wl = W.Workload(cfg)
+    lay, _ = make_layer(cfg, wl)
+    rng = np.random.default_rng(43)
+    S0 = torch.from_numpy(rng.standard_normal((2, 3, 128, 128)).astype(np.float32) * 0.1).cuda()
+    lay.set_state(S0, 5)
+    Q, K, V = (dev(x, "bf16") for x in wl.qkv(0, 0, 0))
+    alpha = torch.from_numpy(wl.alpha(0, 0)).cuda()
+    beta = torch.zeros((2, 3, 150), dtype=torch.float32, device="cuda")
+    lay.commit(Q, K, V, alpha, beta)
+    torch.cuda.synchronize()
+    assert torch.equal(lay.state(), alpha[:, :, None, None] * S0)
+    lay.close()
+
+
+def test_update_with_one_unit_key_writes_its_value_bitwise():
+    """One token, k = e_i through identity maps, alpha = beta = 1, c = 1, S = 0:
+    the update writes V' into row i of S and nothing else, so k^T S_N = v'
+    (ARL2 summary, section 2.1: K'^T diag(beta)(V' - K' S_{N-1}))."""
+    H, i = 2, 37
+    eye = torch.eye(128, dtype=torch.bfloat16, device="cuda").expand(H, 128, 128).contiguous()
+    rng = np.random.default_rng(44)
+    phi_q = dev(rng.standard_normal((H, 128, 128)).astype(np.float32) * 0.1, "bf16")
+    lay = arl2.HybridLayer(1, H, 128, 1, arl2.ARL2_BF16, phi_q, eye, eye, corr_scale=1.0)
+    K = torch.zeros((1, 1, H, 128), dtype=torch.bfloat16, device="cuda")
+    K[0, 0, :, i] = 1.0
+    V = dev(rng.standard_normal((1, 1, H, 128)).astype(np.float32), "bf16")
+    Q = dev(rng.standard_normal((1, 1, H, 128)).astype(np.float32), "bf16")
+    ones_a = torch.ones((1, H), dtype=torch.float32, device="cuda")
+    ones_b = torch.ones((1, H, 1), dtype=torch.float32, device="cuda")
+    lay.commit(Q, K, V, ones_a, ones_b)
+    torch.cuda.synchronize()
+    S = lay.state()
+    want = torch.zeros_like(S)
+    want[0, :, i, :] = V[0, 0].float()
+    assert torch.equal(S, want)
+    lay.close()
