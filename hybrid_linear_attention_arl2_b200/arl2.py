@@ -58,6 +58,8 @@ _SIGS = {
     "arl2_kv_init": (_I32, [ctypes.POINTER(arl2_config), _I32, _VP, ctypes.POINTER(_VP)]),
     "arl2_kv_query": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP]),
     "arl2_kv_commit": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP]),
+    "arl2_kv_query_strided": (_I32, [_VP, _VP, _VP, _VP, _I64, _VP, _VP]),
+    "arl2_kv_commit_strided": (_I32, [_VP, _VP, _VP, _VP, _I64, _VP, _VP]),
     "arl2_kv_frames": (_I64, [_VP]),
     "arl2_kv_device_bytes": (_I64, [_VP]),
     "arl2_kv_last_error": (_I32, [_VP]),
@@ -207,6 +209,16 @@ def arl2_kv_device_bytes(h) -> int:
 
 def arl2_kv_last_error(h) -> int:
     return load_library().arl2_kv_last_error(h)
+
+
+def arl2_kv_query_strided(h, q, k, v, ld, o, stream=None) -> None:
+    _check(load_library().arl2_kv_query_strided(h, _ptr(q), _ptr(k), _ptr(v), int(ld), _ptr(o), _stream(stream)),
+           "arl2_kv_query_strided")
+
+
+def arl2_kv_commit_strided(h, q, k, v, ld, o, stream=None) -> None:
+    _check(load_library().arl2_kv_commit_strided(h, _ptr(q), _ptr(k), _ptr(v), int(ld), _ptr(o), _stream(stream)),
+           "arl2_kv_commit_strided")
 
 
 def arl2_kv_destroy(h) -> None:

@@ -625,18 +625,33 @@ namespace {
 
 // Copy this pass's K and V into cache slot `frames` (the slot after the
 // committed frames), then attend over frames 0..frames of the cache.
-arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, void* o, cudaStream_t st) {
+arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, void* o, cudaStream_t st,
+                    int64_t ld = 0) {
   const arl2_config& c = h->cfg;
   if (h->frames >= h->max_frames) return ARL2_ERR_INVALID_ARGUMENT;
   const size_t esz = c.dtype == ARL2_F32 ? 4 : 2;
-  const size_t frame_bytes = size_t(c.tokens_per_frame) * c.heads * c.head_dim * esz;
+  const size_t row_bytes = size_t(c.heads) * c.head_dim * esz;
+  const size_t frame_bytes = size_t(c.tokens_per_frame) * row_bytes;
   const size_t stream_bytes = frame_bytes * size_t(h->max_frames);
   char* kc = static_cast<char*>(h->kc);
   char* vc = static_cast<char*>(h->vc);
-  ARL2_TRY(cudaMemcpy2DAsync(kc + frame_bytes * h->frames, stream_bytes, k, frame_bytes, frame_bytes, c.batch,
-                             cudaMemcpyDeviceToDevice, st));
-  ARL2_TRY(cudaMemcpy2DAsync(vc + frame_bytes * h->frames, stream_bytes, v, frame_bytes, frame_bytes, c.batch,
-                             cudaMemcpyDeviceToDevice, st));
+  if (ld == 0) {  // one copy per tensor: B frames of contiguous rows
+    ARL2_TRY(cudaMemcpy2DAsync(kc + frame_bytes * h->frames, stream_bytes, k, frame_bytes, frame_bytes, c.batch,
+                               cudaMemcpyDeviceToDevice, st));
+    ARL2_TRY(cudaMemcpy2DAsync(vc + frame_bytes * h->frames, stream_bytes, v, frame_bytes, frame_bytes, c.batch,
+                               cudaMemcpyDeviceToDevice, st));
+  } else {  // one copy per stream and tensor: L token rows `ld` elements apart
+    const size_t pitch = size_t(ld) * esz;
+    for (int b = 0; b < c.batch; ++b) {
+      const size_t src_off = size_t(b) * c.tokens_per_frame * pitch;
+      ARL2_TRY(cudaMemcpy2DAsync(kc + stream_bytes * b + frame_bytes * h->frames, row_bytes,
+                                 static_cast<const char*>(k) + src_off, pitch, row_bytes, c.tokens_per_frame,
+                                 cudaMemcpyDeviceToDevice, st));
+      ARL2_TRY(cudaMemcpy2DAsync(vc + stream_bytes * b + frame_bytes * h->frames, row_bytes,
+                                 static_cast<const char*>(v) + src_off, pitch, row_bytes, c.tokens_per_frame,
+                                 cudaMemcpyDeviceToDevice, st));
+    }
+  }
   const int64_t kv_tokens = int64_t(h->frames + 1) * c.tokens_per_frame;
   const int64_t stride_tokens = int64_t(h->max_frames) * c.tokens_per_frame;
   if (c.dtype == ARL2_F32) {
@@ -658,7 +673,7 @@ arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, voi
     return ARL2_OK;
   }
   CUtensorMap tq, tk, tv, to;
-  if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads) ||
+  if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
       !make_act_map(&tk, h->kc, c.batch, stride_tokens, c.heads) ||
       !make_act_map(&tv, h->vc, c.batch, stride_tokens, c.heads) ||
       !make_act_map(&to, o, c.batch, c.tokens_per_frame, c.heads, 32))
@@ -697,6 +712,32 @@ arl2_status arl2_kv_commit(arl2_kv_t h, const void* q, const void* k, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
   s = kv_pass(h, q, k, v, o, st);
+  if (s == ARL2_OK) h->frames += 1;
+  return s;
+}
+
+arl2_status arl2_kv_query_strided(arl2_kv_t h, const void* q, const void* k, const void* v, int64_t ld, void* o,
+                                  void* stream) {
+  if (!live(h, kKvMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (ld < 0 || (ld != 0 && (h->cfg.dtype != ARL2_BF16 || ld < int64_t(h->cfg.heads) * h->cfg.head_dim || ld % 8 != 0)))
+    return ARL2_ERR_INVALID_ARGUMENT;
+  arl2_status s = check_io(h->cfg, q, k, v, o, ld);
+  if (s != ARL2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  return kv_pass(h, q, k, v, o, st, ld);
+}
+
+arl2_status arl2_kv_commit_strided(arl2_kv_t h, const void* q, const void* k, const void* v, int64_t ld, void* o,
+                                   void* stream) {
+  if (!live(h, kKvMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (ld < 0 || (ld != 0 && (h->cfg.dtype != ARL2_BF16 || ld < int64_t(h->cfg.heads) * h->cfg.head_dim || ld % 8 != 0)))
+    return ARL2_ERR_INVALID_ARGUMENT;
+  arl2_status s = check_io(h->cfg, q, k, v, o, ld);
+  if (s != ARL2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  s = kv_pass(h, q, k, v, o, st, ld);
   if (s == ARL2_OK) h->frames += 1;
   return s;
 }

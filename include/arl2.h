@@ -152,6 +152,14 @@ arl2_status arl2_kv_query(arl2_kv_t kv, const void* q, const void* k, const void
                           void* stream);
 arl2_status arl2_kv_commit(arl2_kv_t kv, const void* q, const void* k, const void* v, void* o,
                            void* stream);
+/* As arl2_kv_query / arl2_kv_commit with Q, K and V read as strided views
+ * (token rows `ld` elements apart; bf16 only; ld >= H * d, a multiple of 8;
+ * 0 = contiguous), bit-identical to the contiguous calls on the same values.
+ * Errors as arl2_frame_query_strided. */
+arl2_status arl2_kv_query_strided(arl2_kv_t kv, const void* q, const void* k, const void* v, int64_t ld,
+                                  void* o, void* stream);
+arl2_status arl2_kv_commit_strided(arl2_kv_t kv, const void* q, const void* k, const void* v, int64_t ld,
+                                   void* o, void* stream);
 int64_t arl2_kv_frames(arl2_kv_t kv);
 int64_t arl2_kv_device_bytes(arl2_kv_t kv);
 arl2_status arl2_kv_last_error(arl2_kv_t kv);

@@ -114,3 +114,8 @@ def test_strided_calls_host_validation(lib):
     assert lib.arl2_frame_query_strided(None, 16, 16, 16, 0, 32, None) == 1
     assert lib.arl2_frame_commit_strided(None, 16, 16, 16, 384, 16, 16, 32, None) == 1
     assert lib.arl2_frame_query_strided(12345, 16, 16, 16, -8, 32, None) == 1
+
+
+def test_kv_strided_calls_host_validation(lib):
+    assert lib.arl2_kv_query_strided(None, 16, 16, 16, 0, 32, None) == 1
+    assert lib.arl2_kv_commit_strided(12345, 16, 16, 16, 768, 32, None) == 1

@@ -352,3 +352,30 @@ def test_update_with_one_unit_key_writes_its_value_bitwise():
     want[0, :, i, :] = V[0, 0].float()
     assert torch.equal(S, want)
     lay.close()
+
+
+def test_kv_layer_strided_equals_contiguous_bitwise():
+    """The KV-cache layer with Q, K, V as strided views of fused rows gives the
+    same bits as with contiguous tensors, over frames that grow the cache."""
+    cfg = small_config(B=2, H=2, L=150, frames=3, queries=1, seed=47)
+    wl = W.Workload(cfg)
+    a = arl2.KVLayer(2, 2, 128, 150, arl2.ARL2_BF16, max_frames=3)
+    b = arl2.KVLayer(2, 2, 128, 150, arl2.ARL2_BF16, max_frames=3)
+    D = 2 * 128
+    for n in range(cfg.frames):
+        for p in range(cfg.passes):
+            Q, K, V = (dev(x, "bf16") for x in wl.qkv(0, n, p))
+            B, L = Q.shape[:2]
+            fused = torch.cat([Q.reshape(B, L, D), K.reshape(B, L, D), V.reshape(B, L, D)], dim=2).contiguous()
+            o1, o2 = torch.empty_like(Q), torch.empty_like(Q)
+            if p < cfg.queries:
+                arl2.arl2_kv_query(a.handle, Q, K, V, o1)
+                arl2.arl2_kv_query_strided(b.handle, fused, fused[..., D:], fused[..., 2 * D:], 3 * D, o2)
+            else:
+                arl2.arl2_kv_commit(a.handle, Q, K, V, o1)
+                arl2.arl2_kv_commit_strided(b.handle, fused, fused[..., D:], fused[..., 2 * D:], 3 * D, o2)
+            torch.cuda.synchronize()
+            assert torch.equal(o1, o2), (n, p)
+    assert a.frames == b.frames == cfg.frames
+    a.close()
+    b.close()
