@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libarl2.so")
 SOURCES = ["arl2_api.cu", "attn_bf16.cu", "state_bf16.cu", "f32_path.cu", "util.cu", "block.cu"]
-HEADERS = ["params.h", "sm100.cuh"]
+HEADERS = ["params.h", "layer.h", "sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

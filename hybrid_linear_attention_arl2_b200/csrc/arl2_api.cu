@@ -20,6 +20,7 @@
 
 #include "../../include/arl2.h"
 
+#include "layer.h"
 #include "params.h"
 
 using namespace arl2;

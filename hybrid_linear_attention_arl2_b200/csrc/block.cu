@@ -22,6 +22,7 @@
 #include <set>
 
 #include "arl2.h"
+#include "layer.h"
 #include "params.h"
 
 namespace arl2 {

@@ -103,18 +103,6 @@ cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaS
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
 
-// The hybrid layer's query and commit with Q, K and V read as strided views:
-// token rows `ld` elements apart (0: contiguous, H * 128), bf16 only.  The
-// C entry points arl2_frame_query / arl2_frame_commit are these with ld = 0.
-}  // namespace arl2
-struct arl2_state;
-#include "arl2.h"
-namespace arl2 {
-arl2_status layer_query_ld(arl2_state* h, const void* q, const void* k, const void* v, int64_t ld, void* o,
-                           cudaStream_t st);
-arl2_status layer_commit_ld(arl2_state* h, const void* q, const void* k, const void* v, int64_t ld, const float* alpha,
-                            const float* beta, void* o, cudaStream_t st);
-
 // Sets the dynamic shared-memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* done_mask);
 
