@@ -26,10 +26,14 @@ in the design notes of the repository):
 * O = O_intra + O_inter, with no gate or normalisation between them;
 * the delta correction carries an explicit coefficient c (``corr_scale``);
   c = 1 is the literal formula, c = 1/L the mean over the frame's tokens.
+* token-level access (``token_level_pass``, the rule the ablation rejects):
+  the same update one token at a time, with a per-token decay a_t and the
+  prediction taken before the token's own decay.
 
 Parity status: the intra branch, the read-out and the update are each pinned
 by brute force on tiny inputs, closed forms and invariants (tests marked
-"not gpu").  The values of a full frame at the benchmark shapes are pinned
+"not gpu"); the token-level pass also by an independently derived chunked
+form.  The values of a full frame at the benchmark shapes are pinned
 only through those same definitions: the pages print no worked numbers.
 """
 from __future__ import annotations
@@ -38,7 +42,7 @@ import numpy as np
 
 __all__ = [
     "feature_maps", "intra_softmax", "inter_readout", "frame_query",
-    "frame_commit", "state_update", "kv_attention", "stream_reference",
+    "frame_commit", "state_update", "kv_attention", "token_level_pass", "stream_reference",
 ]
 
 EPS_NORM = 1e-12
@@ -132,6 +136,39 @@ def kv_attention(Q, K_ctx, V_ctx, scale=None):
     keys and values, with no mask.  K_ctx and V_ctx are that concatenation,
     [B, Lk, H, d]."""
     return intra_softmax(Q, K_ctx, V_ctx, scale)
+
+
+def token_level_pass(S, Q, K, V, phi, alpha_tok, beta, corr_scale=1.0, scale=None):
+    """Token-level access: the alternative to frame-level access that the
+    pages' ablation reports as worse (ARL2 summary, §4, ablations; §2.2 names
+    frame-level access, every token reading S_{N-1}, as the chosen rule).
+    Within one pass, token t reads the state left by the tokens before it in
+    the same pass, and the update of §2.1 ("Zustandsaktualisierung") is
+    applied one token at a time:
+
+        o_t   = O_intra,t + q'_t S^(t-1),          S^(0) = S_{N-1},
+        S^(t) = a_t S^(t-1) + c beta_t k'_t^T (v'_t - k'_t S^(t-1)).
+
+    a is a decay per token (``alpha_tok`` [B, H, L]): the frame-level gate
+    alpha corresponds to a = (alpha, 1, ..., 1), and a general ``alpha_tok``
+    is the per-token gate the pages' wording also allows (§2.1).  The
+    prediction k'_t S^(t-1) reads the state before the token's own decay, as
+    the frame-level formula reads S_{N-1}.  Returns (O [B, L, H, d],
+    S^(L) [B, H, d, d]); a query pass keeps O and drops S^(L), since only the
+    clean pass writes the state (§2.2).
+
+    Token by token in order, each step vectorised over streams and heads."""
+    St = _f64(S).copy()
+    Qp, Kp, Vp = feature_maps(Q, K, V, *phi)
+    a, bt, c = _f64(alpha_tok), _f64(beta), float(corr_scale)
+    B, H, L, _ = Qp.shape
+    Oi = np.empty((B, H, L, St.shape[-1]))
+    for t in range(L):
+        Oi[:, :, t, :] = np.einsum("bhi,bhij->bhj", Qp[:, :, t, :], St)
+        pred = np.einsum("bhi,bhij->bhj", Kp[:, :, t, :], St)
+        r = bt[:, :, t, None] * (Vp[:, :, t, :] - pred)
+        St = a[:, :, t, None, None] * St + c * Kp[:, :, t, :, None] * r[:, :, None, :]
+    return intra_softmax(Q, K, V, scale) + _tokens_first(Oi), St
 
 
 def stream_reference(inputs, frames, queries, corr_scale, phi, S0=None, scale=None,

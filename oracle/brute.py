@@ -16,7 +16,7 @@ from __future__ import annotations
 
 import math
 
-__all__ = ["softmax_attention", "frame_commit", "sequential_commit"]
+__all__ = ["softmax_attention", "frame_commit", "sequential_commit", "token_scan"]
 
 
 def _dot(a, b):
@@ -115,3 +115,35 @@ def sequential_commit(S, K, V, phi, alpha, beta, corr_scale=1.0):
             S_b.append(Sp)
         S_new.append(S_b)
     return S_new
+
+
+def token_scan(S, Q, K, V, phi, alpha_tok, beta, corr_scale=1.0):
+    """Inter-frame part of a token-level pass, in scalar loops: token t reads
+    the state that tokens 1..t-1 of the same pass left, then writes its own
+    delta step (ARL2 summary, §2.1 state update applied one token at a time,
+    the access rule of the §4 ablation):
+
+        o_t[j]   = sum_i q'_t[i] S[i][j];
+        S[i][j] <- a_t S[i][j] + c beta_t k'_t[i] (v'_t[j] - sum_m k'_t[m] S[m][j]),
+
+    the prediction taken before the update of the step.  Returns (O_inter as
+    [B][L][H][d_v] lists, the final state as [B][H][d][d_v] lists)."""
+    phi_q, phi_k, phi_v = phi
+    B, L, H = len(K), len(K[0]), len(K[0][0])
+    O = [[[None] * H for _ in range(L)] for _ in range(B)]
+    S_out = []
+    for b in range(B):
+        S_b = []
+        for h in range(H):
+            St = [[float(x) for x in row] for row in S[b][h]]
+            d, dv = len(St), len(St[0])
+            for t in range(L):
+                qp = _vecmat(Q[b][t][h], phi_q[h])
+                O[b][t][h] = _vecmat(qp, St)
+                kp, vp = _mapped_token(K, V, phi_k, phi_v, b, t, h)
+                pred = _vecmat(kp, St)
+                a, w = float(alpha_tok[b][h][t]), corr_scale * float(beta[b][h][t])
+                St = [[a * St[i][j] + w * kp[i] * (vp[j] - pred[j]) for j in range(dv)] for i in range(d)]
+            S_b.append(St)
+        S_out.append(S_b)
+    return O, S_out
