@@ -7,9 +7,11 @@ t reads the state left by the earlier tokens of the same pass, and the update
 of §2.1 runs one token at a time with a per-token decay a_t.  The pins:
 
 * brute force: ``oracle.brute.token_scan`` (scalar loops);
-* an independent algorithm: the chunked (WY / UT) form below, which solves a
+* independent algorithms: the chunked (WY / UT) form below, which solves a
   unit-lower-triangular system per chunk instead of stepping token by token,
-  for chunk sizes from 1 to the whole frame with a ragged tail;
+  for chunk sizes from 1 to the whole frame with a ragged tail, and its
+  rearrangement into one state-free affine map per chunk (the decomposition
+  a chunk-parallel kernel computes);
 * reductions: one token is the frame-level commit; the first token of any
   frame reads S_{N-1} like every token of a frame-level pass;
 * closed forms: beta = 0 gives pure per-token decay; unit keys with
@@ -98,6 +100,42 @@ def chunked_scan(S0, Qp, Kp, Vp, a, beta, c, chunk):
     return O, S
 
 
+def affine_chunk_scan(S0, Qp, Kp, Vp, a, beta, c, chunk):
+    """The same pass with the entering state taken out of each chunk's work:
+    with W = A^-1 diag(c beta g_prev) K and U' = A^-1 diag(c beta) V (A as in
+    ``chunked_scan``), every chunk is the affine map
+
+        S_next = (g_C I - Kt^T W) S + Kt^T U',     Kt = diag(g_C / g_s) K,
+        O      = (diag(g_prev) Q - P W) S + P U',  P = G * (Q K^T) (strictly lower),
+
+    whose four operands need no state; only S_next = M S + N runs in
+    sequence."""
+    L, dk = Qp.shape
+    maps = []
+    for c0 in range(0, L, chunk):
+        q, k, v = Qp[c0:c0 + chunk], Kp[c0:c0 + chunk], Vp[c0:c0 + chunk]
+        ac, w = a[c0:c0 + chunk], c * beta[c0:c0 + chunk]
+        n = q.shape[0]
+        G = np.zeros((n, n))
+        for t in range(n):
+            for s in range(t):
+                G[t, s] = np.prod(ac[s + 1:t])
+        g_prev = np.array([np.prod(ac[:t]) for t in range(n)])
+        g_tail = np.array([np.prod(ac[s + 1:]) for s in range(n)])
+        Ainv = np.linalg.inv(np.eye(n) + w[:, None] * (G * (k @ k.T)))
+        W = Ainv @ ((w * g_prev)[:, None] * k)
+        Up = Ainv @ (w[:, None] * v)
+        Kt = g_tail[:, None] * k
+        P = G * (q @ k.T)
+        maps.append((np.prod(ac) * np.eye(dk) - Kt.T @ W, Kt.T @ Up, g_prev[:, None] * q - P @ W, P @ Up))
+    S = np.array(S0, dtype=np.float64)
+    outs = []
+    for M, N, Qt, Ot in maps:  # the only sequential part
+        outs.append(Qt @ S + Ot)
+        S = M @ S + N
+    return np.concatenate(outs), S
+
+
 # ---------------------------------------------------------------- pins
 def pin_token_brute(o):
     Q, K, V, phi, S, a, beta = _case(41, B=2, L=5, H=2, d=3)
@@ -119,6 +157,17 @@ def pin_token_chunked_form(o):
             Oc, Sc = chunked_scan(S[0, h], Qp[0, h], Kp[0, h], Vp[0, h], a[0, h], beta[0, h], 1.0, chunk)
             _close(Oi[0, :, h], Oc, 1e-11, f"output vs chunked form (chunk {chunk})")
             _close(Sn[0, h], Sc, 1e-11, f"state vs chunked form (chunk {chunk})")
+
+
+def pin_token_affine_chunk_maps(o):
+    Q, K, V, phi, S, a, beta = _case(48, B=1, L=10, H=1, d=6)
+    O, Sn = o.token_level_pass(S, Q, K, V, phi, a, beta, 0.8)
+    Oi = O - o.intra_softmax(Q, K, V)
+    Qp, Kp, Vp = _mapped(Q, K, V, phi)
+    for chunk in (3, 4, 10):
+        Oc, Sc = affine_chunk_scan(S[0, 0], Qp[0, 0], Kp[0, 0], Vp[0, 0], a[0, 0], beta[0, 0], 0.8, chunk)
+        _close(Oi[0, :, 0], Oc, 1e-11, f"output vs chunk affine maps (chunk {chunk})")
+        _close(Sn[0, 0], Sc, 1e-11, f"state vs chunk affine maps (chunk {chunk})")
 
 
 def pin_token_single_token_is_frame_level(o):
