@@ -49,6 +49,8 @@ _SIGS = {
     "arl2_frame_commit": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "arl2_frame_query_strided": (_I32, [_VP, _VP, _VP, _VP, _I64, _VP, _VP]),
     "arl2_frame_commit_strided": (_I32, [_VP, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP]),
+    "arl2_token_query": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "arl2_token_commit": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "arl2_state_get": (_I32, [_VP, _VP, ctypes.POINTER(_I64), _VP]),
     "arl2_state_set": (_I32, [_VP, _VP, _I64, _VP]),
     "arl2_last_error": (_I32, [_VP]),
@@ -156,6 +158,16 @@ def arl2_frame_query_strided(h, q, k, v, ld, o, stream=None) -> None:
 def arl2_frame_commit_strided(h, q, k, v, ld, alpha, beta, o, stream=None) -> None:
     _check(load_library().arl2_frame_commit_strided(h, _ptr(q), _ptr(k), _ptr(v), int(ld), _ptr(alpha), _ptr(beta),
                                                     _ptr(o), _stream(stream)), "arl2_frame_commit_strided")
+
+
+def arl2_token_query(h, q, k, v, alpha_tok, beta, o, stream=None) -> None:
+    _check(load_library().arl2_token_query(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha_tok), _ptr(beta), _ptr(o),
+                                           _stream(stream)), "arl2_token_query")
+
+
+def arl2_token_commit(h, q, k, v, alpha_tok, beta, o, stream=None) -> None:
+    _check(load_library().arl2_token_commit(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha_tok), _ptr(beta), _ptr(o),
+                                            _stream(stream)), "arl2_token_commit")
 
 
 def arl2_state_get(h, dst, stream=None) -> int:
@@ -306,6 +318,20 @@ class HybridLayer:
     def commit(self, q, k, v, alpha, beta, o=None, stream=None):
         o = self._out(q) if o is None else o
         arl2_frame_commit(self.handle, q, k, v, alpha, beta, o, stream)
+        return o
+
+    def token_query(self, q, k, v, alpha_tok, beta, o=None, stream=None):
+        """Token-level access: token t reads the state the earlier tokens of
+        this pass left; the handle's state is not written."""
+        o = self._out(q) if o is None else o
+        arl2_token_query(self.handle, q, k, v, alpha_tok, beta, o, stream)
+        return o
+
+    def token_commit(self, q, k, v, alpha_tok, beta, o=None, stream=None):
+        """Token-level access on the clean pass: the state after the frame's
+        last token becomes the handle's state."""
+        o = self._out(q) if o is None else o
+        arl2_token_commit(self.handle, q, k, v, alpha_tok, beta, o, stream)
         return o
 
     def state(self, stream=None):

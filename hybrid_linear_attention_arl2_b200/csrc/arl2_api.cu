@@ -161,6 +161,7 @@ struct arl2_state {
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
   CUtensorMap tm_phiq, tm_phik_t, tm_phiv_t, tm_s_bf, tm_mqt[2];
+  float* tok;  // scratch of the token-level calls, allocated by the first one (bf16 path)
 };
 
 struct arl2_kv {
@@ -192,7 +193,7 @@ bool live(const T* h, uint64_t magic) {
 
 void free_state(arl2_state* h) {
   for (void* p : {h->phi[0], h->phi[1], h->phi[2], (void*)h->S[0], (void*)h->S[1], (void*)h->S_bf, (void*)h->mqt,
-                  (void*)h->partial, (void*)h->attn_scratch, (void*)h->attn_ready, (void*)h->err})
+                  (void*)h->partial, (void*)h->attn_scratch, (void*)h->attn_ready, (void*)h->err, (void*)h->tok})
     if (p) cudaFree(p);
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   if (h->ev_join) cudaEventDestroy(h->ev_join);
@@ -229,8 +230,10 @@ arl2_status prepare_readout(arl2_state* h, cudaStream_t st) {
   return ARL2_OK;
 }
 
+// inter = false: the intra-frame branch alone (the token-level calls add
+// their own read-out afterwards).
 arl2_status run_attention(arl2_state* h, const void* q, const void* k, const void* v, void* o, cudaStream_t st,
-                          int64_t ld = 0) {
+                          int64_t ld = 0, bool inter = true) {
   const arl2_config& c = h->cfg;
   if (c.dtype == ARL2_F32) {
     F32AttnParams p{};
@@ -259,7 +262,7 @@ arl2_status run_attention(arl2_state* h, const void* q, const void* k, const voi
   p.heads = c.heads;
   p.scale_log2 = h->scale * 1.4426950408889634f;
   p.flags = c.flags;
-  p.has_inter = 1;
+  p.has_inter = inter ? 1 : 0;
   p.scratch = h->attn_scratch;
   p.ready = h->attn_ready;
   p.err = h->err;
@@ -426,6 +429,16 @@ arl2_status arl2_frame_commit_strided(arl2_state_t h, const void* q, const void*
   return arl2::layer_commit_ld(h, q, k, v, ld, alpha, beta, o, static_cast<cudaStream_t>(stream));
 }
 
+arl2_status arl2_token_query(arl2_state_t h, const void* q, const void* k, const void* v, const float* alpha_tok,
+                             const float* beta, void* o, void* stream) {
+  return arl2::token_pass(h, q, k, v, alpha_tok, beta, o, static_cast<cudaStream_t>(stream), false);
+}
+
+arl2_status arl2_token_commit(arl2_state_t h, const void* q, const void* k, const void* v, const float* alpha_tok,
+                              const float* beta, void* o, void* stream) {
+  return arl2::token_pass(h, q, k, v, alpha_tok, beta, o, static_cast<cudaStream_t>(stream), true);
+}
+
 }  // extern "C"
 
 namespace arl2 {
@@ -504,6 +517,57 @@ arl2_status layer_commit_ld(arl2_state* h, const void* q, const void* k, const v
   }
   h->cur = nxt;
   h->frame += 1;
+  return ARL2_OK;
+}
+
+arl2_status token_pass(arl2_state* h, const void* q, const void* k, const void* v, const float* alpha_tok,
+                       const float* beta, void* o, cudaStream_t st, bool commit) {
+  if (!live(h, kStateMagic)) return ARL2_ERR_INVALID_ARGUMENT;
+  const arl2_config& c = h->cfg;
+  if (c.dtype != ARL2_BF16) return ARL2_ERR_UNSUPPORTED;
+  arl2_status s = check_io(c, q, k, v, o);
+  if (s != ARL2_OK) return s;
+  if (!alpha_tok || !beta || !aligned16(alpha_tok) || !aligned16(beta)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (!h->tok) {
+    const size_t n = token_scratch_floats(c.batch, c.heads, c.tokens_per_frame) * sizeof(float);
+    void* mem = nullptr;
+    if (cudaMalloc(&mem, n) != cudaSuccess) {
+      cudaGetLastError();
+      return ARL2_ERR_OUT_OF_MEMORY;
+    }
+    h->tok = static_cast<float*>(mem);
+    h->bytes += int64_t(n);
+  }
+  h->last_stream = st;
+  s = run_attention(h, q, k, v, o, st, 0, false);  // the intra-frame branch into o
+  if (s != ARL2_OK) return s;
+  const int nxt = h->cur ^ 1;
+  TokenParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.phi_q = static_cast<const __nv_bfloat16*>(h->phi[0]);
+  p.phi_k_t = static_cast<const __nv_bfloat16*>(h->phi[1]);
+  p.phi_v_t = static_cast<const __nv_bfloat16*>(h->phi[2]);
+  p.alpha_tok = alpha_tok;
+  p.beta = beta;
+  p.corr = h->corr;
+  p.B = c.batch;
+  p.L = c.tokens_per_frame;
+  p.H = c.heads;
+  p.n_chunks = h->n_chunks;
+  token_bind_scratch(p, h->tok);
+  p.s_in = h->S[h->cur];
+  p.s_out = commit ? h->S[nxt] : nullptr;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  ARL2_TRY(launch_token_level(p, !(c.flags & ARL2_INTRA_ONLY), st));
+  if (commit) {  // S_N becomes the current state; its bf16 copy and read-out operand follow it
+    h->cur = nxt;
+    ARL2_TRY(launch_to_bf16(h->S[h->cur], h->S_bf, size_t(c.batch) * c.heads * 128 * 128, st));
+    s = prepare_readout(h, st);
+    if (s != ARL2_OK) return s;
+    h->frame += 1;
+  }
   return ARL2_OK;
 }
 

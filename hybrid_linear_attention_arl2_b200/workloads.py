@@ -133,7 +133,7 @@ class Workload:
     Q' = Q @ phi, alpha [B, H], beta [B, H, L].
     """
 
-    _PHI, _GATE_A, _GATE_B, _QKV, _POOL, _WBLK, _XBLK = 1, 2, 3, 4, 5, 6, 7
+    _PHI, _GATE_A, _GATE_B, _QKV, _POOL, _WBLK, _XBLK, _GATE_T = 1, 2, 3, 4, 5, 6, 7, 8
 
     def __init__(self, cfg: Config | int, *, seed: int | None = None):
         self.cfg = CONFIGS[cfg] if isinstance(cfg, int) else cfg
@@ -171,6 +171,16 @@ class Workload:
         for b in range(c.batch):
             rng = _rng(self.seed + b, self._GATE_B, layer, frame)
             rows.append(_sigmoid(rng.standard_normal((c.heads, c.tokens))))
+        return np.stack(rows).astype(np.float32)
+
+    def alpha_tok(self, layer: int, frame: int) -> np.ndarray:
+        """Per-token decays [B, H, L] for token-level passes: sigmoid(N(4, 0.5)),
+        about 0.98, so that a 128-token chunk keeps a tenth of its entering state."""
+        c = self.cfg
+        rows = []
+        for b in range(c.batch):
+            rng = _rng(self.seed + b, self._GATE_T, layer, frame)
+            rows.append(_sigmoid(4.0 + np.sqrt(0.5) * rng.standard_normal((c.heads, c.tokens))))
         return np.stack(rows).astype(np.float32)
 
     # -- per-pass activations -----------------------------------------------

@@ -119,6 +119,29 @@ arl2_status arl2_frame_query_strided(arl2_state_t h, const void* q, const void* 
 arl2_status arl2_frame_commit_strided(arl2_state_t h, const void* q, const void* k, const void* v, int64_t ld,
                                       const float* alpha, const float* beta, void* o, void* stream);
 
+/* Token-level access: the access rule that the ablation of the ARL2 summary
+ * (section 4) reports as worse than frame-level access (section 2.2).  Within
+ * the pass, token t reads the state left by the tokens before it, and the
+ * update of section 2.1 runs one token at a time with a per-token decay:
+ *   o_t   = O_intra,t + q'_t S^(t-1),   S^(0) = the handle's current state,
+ *   S^(t) = a_t S^(t-1) + c beta_t k'_t^T (v'_t - k'_t S^(t-1)),
+ * c being the handle's corr_scale.  The frame-level gate alpha corresponds to
+ * a = (alpha, 1, ..., 1).
+ * alpha_tok, beta: device float32 [B, H, L], 16-byte aligned.
+ * arl2_token_query leaves the state as it is (denoising passes never write
+ * it); arl2_token_commit makes S^(L) the current state, advances the frame
+ * counter, and refreshes what the frame-level calls read, so the two kinds of
+ * call may follow one another on one handle.
+ * bf16 handles only.  The first token-level call on a handle allocates its
+ * scratch (about 5.2 KB per token and head), so it must not be the first
+ * call captured into a CUDA graph.  The arithmetic past the intra-frame
+ * branch is float32.  Errors: INVALID_ARGUMENT, UNSUPPORTED (an f32 handle),
+ * OUT_OF_MEMORY, CUDA. */
+arl2_status arl2_token_query(arl2_state_t h, const void* q, const void* k, const void* v, const float* alpha_tok,
+                             const float* beta, void* o, void* stream);
+arl2_status arl2_token_commit(arl2_state_t h, const void* q, const void* k, const void* v, const float* alpha_tok,
+                              const float* beta, void* o, void* stream);
+
 /* Copy the current state (float32 [B, H, d, d]) to device memory `dst` and the
  * frame counter to *frame (host pointer, may be null).  Synchronous with
  * respect to `stream` for *frame only; the copy is enqueued on `stream`. */

@@ -119,3 +119,10 @@ def test_strided_calls_host_validation(lib):
 def test_kv_strided_calls_host_validation(lib):
     assert lib.arl2_kv_query_strided(None, 16, 16, 16, 0, 32, None) == 1
     assert lib.arl2_kv_commit_strided(12345, 16, 16, 16, 768, 32, None) == 1
+
+
+def test_token_level_calls_host_validation(lib):
+    # a null or unknown handle is rejected before any CUDA call
+    assert lib.arl2_token_query(None, 16, 16, 16, 16, 16, 32, None) == 1
+    assert lib.arl2_token_commit(None, 16, 16, 16, 16, 16, 32, None) == 1
+    assert lib.arl2_token_commit(12345, 16, 16, 16, 16, 16, 32, None) == 1
