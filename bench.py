@@ -49,6 +49,8 @@ def _args():
     ap.add_argument("--block", action="store_true",
                     help="the hybrid attention block (QKV and output projections, gates from the tokens) on the "
                          "single-layer shape (its own JSON line)")
+    ap.add_argument("--token", action="store_true",
+                    help="the single-layer shape with token-level access (the ablated rule; its own JSON line)")
     ap.add_argument("--profile-small", action="store_true",
                     help="a few steps, no extras: for ncu captures of the kernels")
     return ap.parse_args()
@@ -550,6 +552,62 @@ def run_block(args, rank: int, world: int) -> dict:
             "projection_flops_per_frame": cfg.passes * proj}
 
 
+# ------------------------------------------------------------------ token-level access
+def run_token(args, rank: int, world: int) -> dict:
+    """The single-layer shape (B=1, H=12, d=128, L=1560) with token-level
+    access: per frame four token-level queries and one token-level commit,
+    c = 1, per-token decays and write strengths from the seeded generators
+    (eight frames' worth on the device, cycled).  Inputs cycle through the
+    20-triple pool of the frame-level run (288 MB > L2).  Eager launches; the
+    first call allocates the handle's scratch, so it runs in the warm-up."""
+    import torch
+    from hybrid_linear_attention_arl2_b200 import arl2
+    cfg = W.CONFIGS[1]
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    arl2.load_library()
+    ds = DeviceStream(cfg, rank, device)
+    wl = ds.wl
+    gates = [(torch.from_numpy(wl.alpha_tok(0, f)).to(device), torch.from_numpy(wl.beta(0, f)).to(device))
+             for f in range(8)]
+    B, H, L, d = cfg.batch, cfg.heads, cfg.tokens, cfg.head_dim
+    frames = max(1, min(args.steps, 40))
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        layer = arl2.HybridLayer(B, H, d, L, arl2.ARL2_BF16, *ds.phi, corr_scale=1.0, stream=stream)
+        O = torch.empty_like(ds.pool[0][0])
+
+        def frame(f):
+            a, b = gates[f % len(gates)]
+            for p in range(cfg.passes):
+                q, k, v = ds.triple(f, p)
+                if p < cfg.queries:
+                    arl2.arl2_token_query(layer.handle, q, k, v, a, b, O, stream)
+                else:
+                    arl2.arl2_token_commit(layer.handle, q, k, v, a, b, O, stream)
+
+        for f in range(max(3, args.warmup)):
+            frame(f)
+        stream.synchronize()
+        clocks = ClockSampler(local)
+        clocks.start()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for f in range(frames):
+            frame(f)
+        t1.record(stream)
+        t1.synchronize()
+        clk = clocks.stop()
+        err = layer.last_error()
+        ms = t0.elapsed_time(t1)
+        layer.close()
+    if err:
+        raise RuntimeError(f"device error in the token-level run: {arl2.STATUS.get(err)}")
+    value, ms_max = whole_job_rate(ms, frames, world, None, device)
+    return {"frames": frames, "ms": ms_max, "value": value, "clocks": clk}
+
+
 # ------------------------------------------------------------------ attention stack
 def run_stack(args, rank: int, world: int) -> dict:
     """The 30-layer attention stack: layers [0, 22) hybrid, [22, 30) softmax over a
@@ -738,6 +796,25 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
+    if args.token and args.impl != "reference":
+        res = run_token(args, rank, world)
+        if rank != 0:
+            return
+        line = {
+            "metric": "frames/s per hybrid layer with token-level access (1560-token frames, 4 query passes + "
+                      "1 commit)",
+            "value": res["value"], "unit": "frames/s", "n_gpus": world, "steps": res["frames"],
+            "warmup": max(3, args.warmup), "ms_per_step": res["ms"] / res["frames"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 inputs, f32 scan", "data": "synthetic",
+            "config": {"workload": "single-hybrid-layer-token-level-bf16", "batch": 1, "heads": 12,
+                       "head_dim": 128, "tokens_per_frame": 1560, "passes_per_frame": 5, "corr_scale": 1.0,
+                       "gates": "per-token decay sigmoid(N(4, 0.5)), beta sigmoid(N(0, 1))",
+                       "l2": "inputs cycle through a 20-triple pool (288 MB > 126 MB L2)",
+                       "timing": "eager launches, CUDA events around all timed frames"},
+            "tokens_per_s": res["value"] * 1560, "clocks": res["clocks"],
+        }
+        print(json.dumps(line), flush=True)
+        return
     if args.block and args.impl != "reference":
         res = run_block(args, rank, world)
         if rank != 0:
