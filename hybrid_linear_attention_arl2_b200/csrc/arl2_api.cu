@@ -531,9 +531,10 @@ arl2_status token_pass(arl2_state* h, const void* q, const void* k, const void* 
   if (!h->tok) {
     const size_t n = token_scratch_floats(c.batch, c.heads, c.tokens_per_frame) * sizeof(float);
     void* mem = nullptr;
-    if (cudaMalloc(&mem, n) != cudaSuccess) {
+    const cudaError_t e = cudaMalloc(&mem, n);
+    if (e != cudaSuccess) {  // out of memory, or (say) an allocation inside a stream capture
       cudaGetLastError();
-      return ARL2_ERR_OUT_OF_MEMORY;
+      return from_cuda(e);
     }
     h->tok = static_cast<float*>(mem);
     h->bytes += int64_t(n);
