@@ -82,3 +82,39 @@ def test_gathered_shards_equal_the_whole_layer():
         full, S_r, (h0, h1) = out[r]
         np.testing.assert_allclose(full, O, rtol=0, atol=1e-12)
         np.testing.assert_allclose(S_r, S_new[:, h0:h1], rtol=0, atol=1e-12)
+
+
+def test_sharded_layer_passes_its_head_views_to_the_abi(monkeypatch):
+    """What rank 1 of 2 hands the C ABI for a 5-head layer: views that start 3
+    heads into each token row with the whole row's pitch, its own gate slices,
+    and a handle of 2 heads (the binding's calls are replaced by recorders)."""
+    from hybrid_linear_attention_arl2_b200 import arl2, sharding
+    made, calls = {}, []
+
+    class FakeLayer:
+        def __init__(self, batch, heads, head_dim, tokens, dtype, pq, pk, pv, **kw):
+            made.update(batch=batch, heads=heads, phi=(pq, pk, pv))
+            self.handle = 7
+
+        def _out(self, like):
+            return torch.zeros((like.shape[0], like.shape[1], made["heads"], like.shape[3]))
+
+    monkeypatch.setattr(arl2, "HybridLayer", FakeLayer)
+    monkeypatch.setattr(arl2, "arl2_frame_query_strided", lambda *a: calls.append(("q",) + a))
+    monkeypatch.setattr(arl2, "arl2_frame_commit_strided", lambda *a: calls.append(("c",) + a))
+    B, L, H, d = 1, 4, 5, 128
+    phi = [torch.arange(H, dtype=torch.float32)[:, None, None].expand(H, d, d).contiguous() for _ in range(3)]
+    layer = sharding.ShardedHybridLayer(1, 2, B, H, L, *phi)
+    assert made["heads"] == 2 and torch.equal(made["phi"][0][:, 0, 0], torch.tensor([3.0, 4.0]))
+    q, k, v = (torch.zeros((B, L, H, d)) for _ in range(3))
+    layer.query(q, k, v)
+    alpha = torch.arange(H, dtype=torch.float32)[None]
+    beta = torch.arange(H, dtype=torch.float32)[None, :, None].expand(B, H, L).contiguous()
+    layer.commit(q, k, v, alpha, beta)
+    (_, h, qv, kv, vv, ld, o, _), (_, _, qc, _, _, ldc, a, b, _, _) = calls
+    assert h == 7 and ld == ldc == H * d
+    for view, full in ((qv, q), (kv, k), (vv, v), (qc, q)):
+        assert view.data_ptr() == full.data_ptr() + 3 * d * full.element_size()
+        assert view.stride()[1] == H * d
+    assert torch.equal(a, torch.tensor([[3.0, 4.0]])) and torch.equal(b[0, :, 0], torch.tensor([3.0, 4.0]))
+    assert o.shape == (B, L, 2, d)
