@@ -71,7 +71,7 @@ def frame_flops(cfg: W.Config) -> dict:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """SM clock, power and clock-event reasons sampled every 10 ms by NVML while
+    """SM clock, power and clock-event reasons sampled every millisecond by NVML while
     the timed region runs (read-only queries; no setting of the GPU is changed).
     Falls back to `nvidia-smi -lms 50` when NVML cannot be loaded."""
 
@@ -93,7 +93,7 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             h = pynvml.nvmlDeviceGetHandleByIndex(self._nvml_index(pynvml))
-            self.source = "nvml 10 ms"
+            self.source = "nvml 1 ms"
             bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
                     "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
                     "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
@@ -109,7 +109,7 @@ class ClockSampler:
                     except pynvml.NVMLError:
                         break
                     self.samples.append((sm, smax, w, tuple(n for n, b in bits.items() if r & b)))
-                    self.stop_flag.wait(0.010)
+                    self.stop_flag.wait(0.001)
             self.thread = threading.Thread(target=poll, daemon=True)
             self.thread.start()
             return
@@ -485,7 +485,7 @@ def long_stream_flatness(cfg, ds, device, rank) -> dict:
 # ------------------------------------------------------------------ attention block
 def run_block(args, rank: int, world: int) -> dict:
     """The hybrid attention block on the single-layer shape (B=1, H=12, d=128,
-    L=1560, hidden 1536): per pass X -> Q, K, V (cuBLAS) -> hybrid layer -> O W_o;
+    L=1560, hidden 1536): per pass X -> Q, K, V (tcgen05 GEMM) -> hybrid layer -> O W_o;
     the commit also forms its gates from X.  Inputs cycle through 40 seeded
     token matrices (192 MB > L2); CUDA graphs of four frames, as the layer's run."""
     import dataclasses
@@ -760,6 +760,16 @@ def peaks():
         return None
 
 
+def peak_pair(pk):
+    """(burst, sustained) dense bf16 TFLOP/s and their source.  The burst figure
+    is the headline denominator: the kernels are timed in regions of a few
+    milliseconds at the clocks sampled alongside; the sustained figure (a
+    seconds-long loop under the power cap) is reported as a second ratio."""
+    if pk:
+        return pk["bf16_tflops"], pk["bf16_tflops_sustained"], "of measured"
+    return 1590.0, 1400.0, "of fallback"
+
+
 def main():
     args = _args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -819,8 +829,7 @@ def main():
         res = run_block(args, rank, world)
         if rank != 0:
             return
-        pk = peaks()
-        peak_sus, src = (pk["bf16_tflops_sustained"], "of measured") if pk else (1400.0, "of fallback")
+        peak_burst, peak_sus, src = peak_pair(peaks())
         tf = res["flops_per_frame"] * res["value"] / 1e12
         line = {
             "metric": "frames/s per hybrid attention block (1560-token frames, hidden 1536, QKV/out projections "
@@ -831,8 +840,9 @@ def main():
             "config": {"workload": "hybrid-attention-block-bf16", "batch": 1, "heads": 12, "head_dim": 128,
                        "hidden": 1536, "tokens_per_frame": 1560, "passes_per_frame": 5,
                        "l2": "tokens cycle through 40 seeded 1560 x 1536 matrices (192 MB > 126 MB L2)",
-                       "projections": "cuBLAS GEMMs (bf16, fp32 accumulate)"},
-            "tflops": tf, "pct_bf16_peak": {"value": 100.0 * tf / peak_sus, "basis": f"sustained bf16 {src}"},
+                       "projections": "tcgen05 GEMMs of this library (bf16, fp32 accumulate)"},
+            "tflops": tf, "pct_bf16_peak": {"value": 100.0 * tf / peak_burst, "basis": f"burst bf16 {src}",
+                                            "sustained_basis": 100.0 * tf / peak_sus},
             "clocks": res["clocks"],
         }
         print(json.dumps(line), flush=True)
@@ -844,8 +854,7 @@ def main():
             res = run_stack(args, rank, world)
             if rank != 0:
                 return
-            pk = peaks()
-            peak_sus, src = (pk["bf16_tflops_sustained"], "of measured") if pk else (1400.0, "of fallback")
+            peak_burst, peak_sus, src = peak_pair(peaks())
             line = {
                 "metric": "stack frames/s (30 attention layers: 22 hybrid + 8 KV-cache softmax, 1560-token frames)",
                 "value": res["frames"] * world / (res["ms_total"] / 1e3), "unit": "frames/s", "n_gpus": world,
@@ -860,12 +869,14 @@ def main():
                 "split_ms": {"hybrid": res["ms_hybrid"], "kv_softmax": res["ms_kv"]},
                 "tflops": {"stack": res["stack_tflops"], "hybrid_layers": res["hybrid_tflops"],
                            "kv_softmax_layers": res["kv_tflops"]},
-                "pct_bf16_peak": {"value": 100.0 * res["stack_tflops"] / peak_sus,
-                                  "basis": f"sustained bf16 {src}"},
+                "pct_bf16_peak": {"value": 100.0 * res["stack_tflops"] / peak_burst,
+                                  "basis": f"burst bf16 {src}",
+                                  "sustained_basis": 100.0 * res["stack_tflops"] / peak_sus},
                 "roofline": {"bound": "tensor", "kernel": "attn_bf16_kernel (KV-cache softmax layers)",
-                             "achieved": res["kv_tflops"], "peak": peak_sus, "unit": "TFLOP/s",
-                             "frac": res["kv_tflops"] / peak_sus, "traffic": None,
-                             "peak_basis": f"bf16_tflops_sustained {src}"},
+                             "achieved": res["kv_tflops"], "peak": peak_burst, "unit": "TFLOP/s",
+                             "frac": res["kv_tflops"] / peak_burst, "traffic": None,
+                             "peak_basis": f"bf16_tflops (burst) {src}",
+                             "frac_vs_sustained": res["kv_tflops"] / peak_sus},
                 "clocks": res["clocks"], "gpu_launches": res["launches"],
             }
             print(json.dumps(line), flush=True)
@@ -877,20 +888,18 @@ def main():
     fl = res["flops"]
     frame_tflops = fl["frame"] * res["value"] / max(1, world) / 1e12  # per GPU
     attn_tflops = fl["attn_per_pass"] / (res["attn_avg_ms"] / 1e3) / 1e12
-    if pk:
-        peak_sus, peak_burst, src = pk["bf16_tflops_sustained"], pk["bf16_tflops"], "of measured"
-    else:
-        peak_sus, peak_burst, src = 1400.0, 1590.0, "of fallback"
+    peak_burst, peak_sus, src = peak_pair(pk)
     line = {
         "metric": metric, "value": res["value"], "unit": "frames/s", "n_gpus": world, "steps": res["steps"],
         "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
         "tokens_per_s": res["value"] * cfg.tokens * cfg.batch,
-        "pct_bf16_peak": {"value": 100.0 * frame_tflops / peak_sus, "basis": f"sustained bf16 {src}",
-                          "burst_basis": 100.0 * frame_tflops / peak_burst},
-        "roofline": {"bound": "tensor", "kernel": "attn_bf16_kernel", "achieved": attn_tflops, "peak": peak_sus,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak_sus, "traffic": attn_traffic(),
-                     "peak_basis": f"bf16_tflops_sustained {src}"},
+        "pct_bf16_peak": {"value": 100.0 * frame_tflops / peak_burst, "basis": f"burst bf16 {src}",
+                          "sustained_basis": 100.0 * frame_tflops / peak_sus},
+        "roofline": {"bound": "tensor", "kernel": "attn_bf16_kernel", "achieved": attn_tflops, "peak": peak_burst,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak_burst, "traffic": attn_traffic(),
+                     "peak_basis": f"bf16_tflops (burst) {src}",
+                     "frac_vs_sustained": attn_tflops / peak_sus},
         "clocks": res["clocks"],
         "gpu_launches": res["launches_per_step"] * res["steps"],
     }

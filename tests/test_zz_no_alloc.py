@@ -7,8 +7,11 @@ serves them: it computes the same state write as ``arl2_frame_commit`` with
 its work space in the library's static scratch array.  This test calls it
 through the C ABI for two frames in a row -- the second call reuses the array
 the first one left behind -- and checks each new state against the state the
-handle's commit wrote from the same inputs, within the bf16 state tolerance of
-the parity tests (||S - S_ref||_F / ||S_ref||_F <= 1e-2).
+handle's commit wrote from the same inputs.  Both run the same kernels in the
+same order on bit-identical inputs, so the states must be equal bit for bit; a
+scratch-layout or aliasing mistake that shifts a few values would pass a
+tolerance but not this.  The Frobenius-relative error against the bf16 state
+tolerance of the parity tests (1e-2) is reported when they differ.
 
 The file name sorts last so that a run which stops at the first failure has
 run every other test before this one.
@@ -58,8 +61,11 @@ def test_noalloc_state_write_matches_commit_twice(B, H, L, corr):
         got = host(S_next)
         assert np.isfinite(got).all(), f"frame {n}: non-finite state"
         assert np.linalg.norm(S_ref) > 0
-        e = frob_rel(got, S_ref)
-        assert e <= BF16_STATE_TOL, f"frame {n}: {e:.3e} > {BF16_STATE_TOL}"
+        if not torch.equal(S_next, layer.state()):
+            e = frob_rel(got, S_ref)
+            diff = int((S_next != layer.state()).sum().item())
+            pytest.fail(f"frame {n}: {diff} state values differ from the commit's (Frobenius-relative "
+                        f"{e:.3e}, tolerance of the parity tests {BF16_STATE_TOL})")
         S_prev, S_next = S_next, S_prev
     assert layer.last_error() == 0
     layer.close()
