@@ -75,6 +75,7 @@ _SIGS = {
                                         _VP]),
     "arl2_selftest_wait_timeout": (_I32, [_U64, _VP]),
     "arl2_selftest_exp2": (_I32, [_VP, _VP, _I64, _VP]),
+    "arl2_gemm_bf16": (_I32, [_VP, _I64, _VP, _I64, _VP, _I64, _I64, _I64, _I64, _VP]),
     "arl2_status_string": (ctypes.c_char_p, [_I32]),
     "arl2_abi_version": (_I32, []),
 }
@@ -273,6 +274,13 @@ def arl2_state_write_noalloc(cfg: arl2_config, k, v, phi_k, phi_v, S_prev, alpha
 
 def arl2_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     return load_library().arl2_selftest_wait_timeout(limit_ns, _stream(stream))
+
+
+def arl2_gemm_bf16(a, b, c, m, n, k, lda=None, ldb=None, ldc=None, stream=None) -> None:
+    """C[m, n] = A[m, k] B[k, n] on bf16 device tensors (row-major; leading
+    dimensions default to k, n and n)."""
+    _check(load_library().arl2_gemm_bf16(_ptr(a), lda or k, _ptr(b), ldb or n, _ptr(c), ldc or n, m, n, k,
+                                         _stream(stream)), "arl2_gemm_bf16")
 
 
 def arl2_selftest_exp2(x, y, stream=None) -> None:

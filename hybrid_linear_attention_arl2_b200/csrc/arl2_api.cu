@@ -11,6 +11,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -96,8 +97,8 @@ bool make_act_map(CUtensorMap* m, const void* base, int B, int64_t tokens, int H
 }
 
 // Stacked 128 x 128 bf16 matrices [slabs, 128, 128] as a map over (128, 128, slabs).
-bool make_mat_map(CUtensorMap* m, const void* base, int slabs) {
-  return make_map(m, base, 128, 128, uint64_t(slabs), 256, 256 * 128, 128);
+bool make_mat_map(CUtensorMap* m, const void* base, int slabs, uint32_t rows = 128) {
+  return make_map(m, base, 128, 128, uint64_t(slabs), 256, 256 * 128, rows);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -152,6 +153,8 @@ struct arl2_state {
   float* attn_scratch;   // partial rows of split query blocks (bf16 path)
   unsigned* attn_ready;  // their ready flags, zero between launches
   int sms;
+  int pairs;             // CTA pairs of the attention kernel resident at once
+  bool state_fused;      // the state write runs as one cluster launch (<= 16 chunks)
   uint32_t* err;
   int64_t frame;
   int64_t bytes;
@@ -161,6 +164,7 @@ struct arl2_state {
   cudaStream_t side;
   cudaEvent_t ev_fork, ev_join;
   CUtensorMap tm_phiq, tm_phik_t, tm_phiv_t, tm_s_bf, tm_mqt[2];
+  CUtensorMap tm_mqt64[2];  // the same MqT slots in 64-row boxes (a CTA's half for the pair kernel)
   float* tok;  // scratch of the token-level calls, allocated by the first one (bf16 path)
 };
 
@@ -177,6 +181,7 @@ struct arl2_kv {
   float* attn_scratch;
   unsigned* attn_ready;
   int sms;
+  int pairs;  // CTA pairs of the attention kernel resident at once
   uint32_t* err;
   int64_t bytes;
   cudaStream_t last_stream;
@@ -253,7 +258,7 @@ arl2_status run_attention(arl2_state* h, const void* q, const void* k, const voi
   }
   CUtensorMap tq, tk, tv, to;
   if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
-      !make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
+      !make_act_map(&tk, k, c.batch, c.tokens_per_frame, c.heads, 64, ld) ||
       !make_act_map(&tv, v, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
       !make_act_map(&to, o, c.batch, c.tokens_per_frame, c.heads, 32))
     return ARL2_ERR_CUDA;
@@ -267,14 +272,15 @@ arl2_status run_attention(arl2_state* h, const void* q, const void* k, const voi
   p.ready = h->attn_ready;
   p.err = h->err;
   p.wait_limit_ns = h->wait_ns;
-  if (!attn_partition(p, c.batch, h->sms)) return ARL2_ERR_UNSUPPORTED;
-  ARL2_TRY(launch_attn_bf16(tq, tk, tv, h->tm_mqt[h->cur], to, p, st));
+  if (!attn_pair_partition(p, c.batch, h->pairs)) return ARL2_ERR_UNSUPPORTED;
+  ARL2_TRY(launch_attn_pair(tq, tk, tv, h->tm_mqt64[h->cur], to, p, st));
   return ARL2_OK;
 }
 
-bool overlaps(const void* a, const void* b, size_t n) {
+// [a, a + na) and [b, b + nb) share a byte.
+bool overlaps2(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x < y + n && y < x + n;
+  return x < y + nb && y < x + na;
 }
 
 arl2_status check_io(const arl2_config& c, const void* q, const void* k, const void* v, const void* o,
@@ -353,8 +359,10 @@ arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const voi
   alloc(reinterpret_cast<void**>(&h->err), 256);
   if (cfg->dtype == ARL2_BF16) {
     if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || h->sms < 1) h->sms = 1;
-    alloc(reinterpret_cast<void**>(&h->attn_scratch), size_t(h->sms) * 2 * kAttnSlotFloats * sizeof(float));
-    alloc(reinterpret_cast<void**>(&h->attn_ready), size_t(h->sms) * 2 * sizeof(unsigned));
+    h->pairs = std::min(h->sms / 2, attn_pair_capacity());
+    h->state_fused = state_fused_supported(h->n_chunks, H, B);
+    alloc(reinterpret_cast<void**>(&h->attn_scratch), attn_scratch_floats(h->sms) * sizeof(float));
+    alloc(reinterpret_cast<void**>(&h->attn_ready), attn_ready_words(h->sms) * sizeof(unsigned));
     alloc(reinterpret_cast<void**>(&h->S_bf), size_t(B) * H * d * d * 2);
     alloc(reinterpret_cast<void**>(&h->mqt), 2 * size_t(B) * H * d * d * 2);
     alloc(reinterpret_cast<void**>(&h->partial), size_t(B) * H * h->n_chunks * d * d * sizeof(float));
@@ -385,11 +393,13 @@ arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const voi
   if (cfg->dtype == ARL2_BF16) {
     if (e == cudaSuccess) e = cudaMemsetAsync(h->S_bf, 0, size_t(B) * H * d * d * 2, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(h->mqt, 0, 2 * size_t(B) * H * d * d * 2, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(h->attn_ready, 0, size_t(h->sms) * 2 * sizeof(unsigned), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->attn_ready, 0, attn_ready_words(h->sms) * sizeof(unsigned), st);
     if (e == cudaSuccess &&
         !(make_mat_map(&h->tm_phiq, h->phi[0], H) && make_mat_map(&h->tm_phik_t, h->phi[1], H) &&
           make_mat_map(&h->tm_phiv_t, h->phi[2], H) && make_mat_map(&h->tm_s_bf, h->S_bf, B * H) &&
-          make_mat_map(&h->tm_mqt[0], mqt_slot(h, 0), B * H) && make_mat_map(&h->tm_mqt[1], mqt_slot(h, 1), B * H)))
+          make_mat_map(&h->tm_mqt[0], mqt_slot(h, 0), B * H) && make_mat_map(&h->tm_mqt[1], mqt_slot(h, 1), B * H) &&
+          make_mat_map(&h->tm_mqt64[0], mqt_slot(h, 0), B * H, 64) &&
+          make_mat_map(&h->tm_mqt64[1], mqt_slot(h, 1), B * H, 64)))
       e = cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) {
@@ -509,9 +519,14 @@ arl2_status layer_commit_ld(arl2_state* h, const void* q, const void* k, const v
     sp.err = h->err;
     sp.wait_limit_ns = h->wait_ns;
     ARL2_TRY(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-    ARL2_TRY(launch_state_partial(tk, tv, h->tm_phik_t, h->tm_phiv_t, h->tm_s_bf, sp, c.batch, h->side));
-    ARL2_TRY(launch_state_finalize(sp, c.batch, h->side));
-    ARL2_TRY(launch_readout_prep(h->tm_s_bf, h->tm_phiq, sp, c.batch, h->side));
+    if (h->state_fused) {  // one launch: partials reduced on chip, MqT formed by each cluster's rank 0
+      ARL2_TRY(launch_state_fused(tk, tv, h->tm_phik_t, h->tm_phiv_t, h->tm_s_bf, h->tm_phiq, sp, c.batch,
+                                  h->side));
+    } else {
+      ARL2_TRY(launch_state_partial(tk, tv, h->tm_phik_t, h->tm_phiv_t, h->tm_s_bf, sp, c.batch, h->side));
+      ARL2_TRY(launch_state_finalize(sp, c.batch, h->side));
+      ARL2_TRY(launch_readout_prep(h->tm_s_bf, h->tm_phiq, sp, c.batch, h->side));
+    }
     ARL2_TRY(cudaEventRecord(h->ev_join, h->side));
     ARL2_TRY(cudaStreamWaitEvent(st, h->ev_join, 0));
   }
@@ -519,6 +534,9 @@ arl2_status layer_commit_ld(arl2_state* h, const void* q, const void* k, const v
   h->frame += 1;
   return ARL2_OK;
 }
+
+uint32_t* layer_error_word(arl2_state* h) { return h->err; }
+uint64_t layer_wait_limit(arl2_state* h) { return h->wait_ns; }
 
 arl2_status token_pass(arl2_state* h, const void* q, const void* k, const void* v, const float* alpha_tok,
                        const float* beta, void* o, cudaStream_t st, bool commit) {
@@ -613,7 +631,7 @@ arl2_status arl2_last_error(arl2_state_t h) {
   if (w) {
     // a kernel that gave up may have left partial-ready flags raised
     ARL2_TRY(cudaMemset(h->err, 0, sizeof(w)));
-    if (h->attn_ready) ARL2_TRY(cudaMemset(h->attn_ready, 0, size_t(h->sms) * 2 * sizeof(unsigned)));
+    if (h->attn_ready) ARL2_TRY(cudaMemset(h->attn_ready, 0, attn_ready_words(h->sms) * sizeof(unsigned)));
   }
   return static_cast<arl2_status>(w);
 }
@@ -662,8 +680,9 @@ arl2_status arl2_kv_init(const arl2_config* cfg, int32_t max_frames, void* strea
   const size_t esz = cfg->dtype == ARL2_F32 ? 4 : 2;
   const size_t bytes = size_t(cfg->batch) * size_t(tokens) * cfg->heads * cfg->head_dim * esz;
   if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || h->sms < 1) h->sms = 1;
-  const size_t scratch_bytes = size_t(h->sms) * 2 * kAttnSlotFloats * sizeof(float);
-  const size_t ready_bytes = size_t(h->sms) * 2 * sizeof(unsigned);
+  h->pairs = cfg->dtype == ARL2_BF16 ? std::min(h->sms / 2, attn_pair_capacity()) : 0;
+  const size_t scratch_bytes = attn_scratch_floats(h->sms) * sizeof(float);
+  const size_t ready_bytes = attn_ready_words(h->sms) * sizeof(unsigned);
   cudaError_t e = dev_alloc(&h->kc, bytes);
   if (e == cudaSuccess) e = dev_alloc(&h->vc, bytes);
   if (e == cudaSuccess && cfg->dtype == ARL2_BF16) e = dev_alloc(reinterpret_cast<void**>(&h->attn_scratch), scratch_bytes);
@@ -740,8 +759,8 @@ arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, voi
   }
   CUtensorMap tq, tk, tv, to;
   if (!make_act_map(&tq, q, c.batch, c.tokens_per_frame, c.heads, 128, ld) ||
-      !make_act_map(&tk, h->kc, c.batch, stride_tokens, c.heads) ||
-      !make_act_map(&tv, h->vc, c.batch, stride_tokens, c.heads) ||
+      !make_act_map(&tk, h->kc, c.batch, stride_tokens, c.heads, 64) ||
+      !make_act_map(&tv, h->vc, c.batch, stride_tokens, c.heads, 128) ||
       !make_act_map(&to, o, c.batch, c.tokens_per_frame, c.heads, 32))
     return ARL2_ERR_CUDA;
   AttnParams p{};
@@ -755,8 +774,8 @@ arl2_status kv_pass(arl2_kv* h, const void* q, const void* k, const void* v, voi
   p.ready = h->attn_ready;
   p.err = h->err;
   p.wait_limit_ns = h->wait_ns;
-  if (!attn_partition(p, c.batch, h->sms)) return ARL2_ERR_UNSUPPORTED;
-  ARL2_TRY(launch_attn_bf16(tq, tk, tv, tq, to, p, st));
+  if (!attn_pair_partition(p, c.batch, h->pairs)) return ARL2_ERR_UNSUPPORTED;
+  ARL2_TRY(launch_attn_pair(tq, tk, tv, tq, to, p, st));
   return ARL2_OK;
 }
 
@@ -819,7 +838,7 @@ arl2_status arl2_kv_last_error(arl2_kv_t h) {
   if (w) {
     // a kernel that gave up may have left partial-ready flags raised
     ARL2_TRY(cudaMemset(h->err, 0, sizeof(w)));
-    if (h->attn_ready) ARL2_TRY(cudaMemset(h->attn_ready, 0, size_t(h->sms) * 2 * sizeof(unsigned)));
+    if (h->attn_ready) ARL2_TRY(cudaMemset(h->attn_ready, 0, attn_ready_words(h->sms) * sizeof(unsigned)));
   }
   return static_cast<arl2_status>(w);
 }
@@ -848,6 +867,30 @@ arl2_status arl2_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   cudaFree(err);
   if (e != cudaSuccess) return from_cuda(e);
   return static_cast<arl2_status>(w);
+}
+
+arl2_status arl2_gemm_bf16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c, int64_t ldc, int64_t m,
+                           int64_t n, int64_t k, void* stream) {
+  if (!a || !b || !c || !aligned16(a) || !aligned16(b) || !aligned16(c)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (m < 0 || n < 0 || k < 0 || m > (1 << 30) || n > (1 << 30) || k > (1 << 30)) return ARL2_ERR_INVALID_ARGUMENT;
+  if (lda < k || ldb < n || ldc < n || lda % 8 || ldb % 8 || ldc % 8) return ARL2_ERR_INVALID_ARGUMENT;
+  if (m == 0 || n == 0) return ARL2_OK;
+  const size_t nc = (size_t(m - 1) * size_t(ldc) + size_t(n)) * 2;
+  if (overlaps2(c, nc, a, (size_t(m - 1) * size_t(lda) + size_t(k)) * 2) ||
+      overlaps2(c, nc, b, (size_t(k > 0 ? k - 1 : 0) * size_t(ldb) + size_t(n)) * 2))
+    return ARL2_ERR_INVALID_ARGUMENT;
+  if (!encode_fn()) return ARL2_ERR_NO_DEVICE;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ARL2_ERR_NO_DEVICE;
+  GemmParams p{};
+  p.M = int(m);
+  p.N = int(n);
+  p.K = int(k);
+  p.err = nullptr;
+  p.wait_limit_ns = kDefaultWaitNs;
+  ARL2_TRY(gemm_bf16(a, lda, b, ldb, c, ldc, p, sms, static_cast<cudaStream_t>(stream)));
+  return ARL2_OK;
 }
 
 arl2_status arl2_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
@@ -907,7 +950,19 @@ extern "C" arl2_status arl2_state_write_noalloc(const arl2_config* cfg, const vo
   const int B = cfg->batch, H = cfg->heads, L = cfg->tokens_per_frame;
   const size_t mat_bf = size_t(128) * 128 * 2;
   const size_t state_bytes = size_t(B) * H * 128 * 128 * sizeof(float);
-  if (overlaps(S_prev, S_next, state_bytes)) return ARL2_ERR_INVALID_ARGUMENT;
+  // The outputs (S_next, dev_error) may share no byte with any input or with
+  // each other: the kernels read every input after the first output byte is
+  // written.
+  {
+    const size_t act = size_t(B) * L * H * 128 * 2, phi = size_t(H) * 128 * 128 * 2;
+    const struct { const void* p; size_t n; } in[] = {
+        {k, act}, {v, act}, {phi_k, phi}, {phi_v, phi}, {S_prev, state_bytes},
+        {alpha, size_t(B) * H * sizeof(float)}, {beta, size_t(B) * H * L * sizeof(float)}};
+    for (const auto& r : in)
+      if (overlaps2(S_next, state_bytes, r.p, r.n) || overlaps2(dev_error, sizeof(uint32_t), r.p, r.n))
+        return ARL2_ERR_INVALID_ARGUMENT;
+    if (overlaps2(S_next, state_bytes, dev_error, sizeof(uint32_t))) return ARL2_ERR_INVALID_ARGUMENT;
+  }
   const int n_chunks = (L + 127) / 128;
   // Scratch layout: phi_k^T, phi_v^T [H,128,128] bf16; S_prev and S_next in
   // bf16 [B,H,128,128]; per-chunk partials [B,H,n_chunks,128,128] fp32.

@@ -1,0 +1,766 @@
+// Intra-frame softmax attention with the inter-frame read-out fused into its
+// epilogue, on CTA pairs (tcgen05 cta_group::2), bf16 operands, fp32
+// accumulation in tensor memory (sm_100a).
+//
+//   O = softmax(Q K^T * scale) V  +  Q MqT^T        (MqT = (phi_q S_{N-1})^T)
+//
+// The first term is the intra-frame branch (ARL2 summary, section 2.1: the
+// original bidirectional softmax attention within each frame).  The second is
+// the inter-frame read-out O_inter = Q' S_{N-1} = (Q phi_q) S_{N-1}, computed
+// as Q (phi_q S_{N-1}), one extra 256 x 128 x 128 MMA per 256 query rows.
+//
+// Work decomposition.  A cluster of two CTAs owns a block of 256 query rows of
+// one (stream, head): query tile 2b in rank 0, tile 2b + 1 in rank 1.  Every
+// MMA covers both CTAs' rows (M = 256): rank 0 issues it, each CTA supplies
+// its own 128 rows of the A operand and half of the B operand (64 keys of a K
+// tile, 64 head dimensions of a V tile) and keeps its 128 rows of the
+// accumulator in its own tensor memory.  The key tiles of a block alternate
+// between two chains with their own S buffer, softmax warpgroup, running
+// statistics (m, l) and O accumulator, so that one chain's softmax overlaps
+// the other chain's MMAs; the epilogue merges the two chains.  The sequence
+// of (block, key tile) units over all (stream, head) pairs is cut into
+// contiguous equal ranges, one per CTA pair ("stream-K").  A block whose key
+// range is split across pairs is finished by the pair holding its key tile 0
+// (always that pair's last segment); the pairs continuing it store their
+// normalised partial output and (m, l) in fp32 and raise ready flags, and the
+// finishing pair combines the pieces in key order (deterministic).
+//
+// Roles per CTA (512 threads, four warpgroups):
+//   warp 0       TMA producer: per segment the CTA's Q tile (two slots, so the
+//                next segment's Q loads during the current one), then its
+//                halves of K_j, V_j (and of MqT for blocks it finishes)
+//                through a ring of 16 KB slots; the loads of both CTAs count
+//                on rank 0's barriers;
+//   warp 1       (rank 0 only) tcgen05 issuer: S(i) = Q K^T, O_c += P V, X = Q MqT^T;
+//   warp 2       tensor-memory allocator (both CTAs, cta_group::2);
+//   warps 4..7   softmax of chain 0 (one query row per thread);
+//   warps 8..11  softmax of chain 1;
+//   warps 12..15 epilogue: at the end of a segment reads O_0, O_1 (and X)
+//                from tensor memory, hands it back at once, merges the chains
+//                (and, for a split block, the other pairs' pieces) and writes
+//                the output with TMA tile stores, or stores the partial.
+// Tensor memory (512 columns per CTA): S_0 [0,128), S_1 [128,256) (P written
+// in place as bf16 pairs; X goes into S_1 at the end of a segment),
+// O_0 [256,384), O_1 [384,512).
+//
+// Every wait is bounded (mbarriers and peer flags): on expiry the CTA raises
+// its abort flag and records a timeout; there is no named barrier, so a role
+// that leaves early never strands another.  The same kernel without the
+// read-out serves the softmax layers that keep a growing KV cache.
+
+#include "params.h"
+#include "sm100.cuh"
+
+namespace arl2 {
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kRing = 7;
+constexpr uint32_t kQTile = 32768;  // 128 rows x 128 bf16
+constexpr uint32_t kBox = 16384;    // 128 rows x 64 bf16
+constexpr uint32_t kSlot = 16384;   // a half tile: 64 keys x 128 dims, 128 keys x 64 dims, or 64 rows of MqT
+constexpr uint32_t kTilesBytes = 2 * kQTile + kRing * kSlot + kQTile;  // Q x2, ring, output staging
+constexpr uint32_t kBarBytes = 256;
+constexpr uint32_t kStatsBytes = 2 * 2 * 128 * 4;  // (m, l) of both chains
+constexpr int kSmem = 232448;
+static_assert(kTilesBytes + kBarBytes + kStatsBytes + 1024 <= uint32_t(kSmem), "shared memory layout too large");
+constexpr int kMaxContrib = 8;
+constexpr int kLaunchRegs = 128;
+constexpr int kCtlRegs = 56;
+constexpr int kSoftmaxRegs = 176;
+constexpr int kEpiRegs = 104;
+static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs + 128 * kEpiRegs <= kThreads * kLaunchRegs,
+              "register split too large");
+
+enum {
+  B_QF = 0,              // [2] Q slot loaded (rank 0: both CTAs' bytes)
+  B_QE = 2,              // [2] Q slot free (commit, both CTAs)
+  B_RF = 4,              // [kRing] ring slot loaded (rank 0: both CTAs' bytes)
+  B_RE = 4 + kRing,      // [kRing] ring slot free (commit, both CTAs)
+  B_SF = 4 + 2 * kRing,  // [2] S of chain c in tensor memory (commit, both CTAs)
+  B_PF = B_SF + 2,       // [2] P of chain c written (rank 0: 4 warps x 2 CTAs)
+  B_SD = B_PF + 2,       // every MMA of the segment completed (commit, both CTAs)
+  B_ST = B_SD + 1,       // both chains' statistics in shared memory (local: 8 warps)
+  B_EO = B_ST + 1,       // epilogues done with O_0, O_1 and X (rank 0: 4 warps x 2 CTAs)
+  B_SC = B_EO + 1,       // statistics read by the epilogue (local: 4 warps)
+  B_DRAIN = B_SC + 1,
+  B_COUNT
+};
+static_assert(B_COUNT * 8 + 8 <= int(kBarBytes), "barrier area too small");
+
+struct Seg {
+  int bh, blk, j0, j1;
+};
+
+__device__ __forceinline__ bool next_seg(const AttnParams& p, unsigned& u, unsigned u_end, Seg& s) {
+  if (u >= u_end) return false;
+  const unsigned per = unsigned(p.n_blk) * unsigned(p.nkv);
+  s.bh = int(u / per);
+  const unsigned r = u - unsigned(s.bh) * per;
+  s.blk = int(r / unsigned(p.nkv));
+  s.j0 = int(r - unsigned(s.blk) * unsigned(p.nkv));
+  s.j1 = int(min(unsigned(p.nkv), unsigned(s.j0) + (u_end - u)));
+  u += unsigned(s.j1 - s.j0);
+  return true;
+}
+
+// Ring positions within a segment of n key tiles, in the order the issuer
+// consumes them: K_0, K_1, V_0, K_2, V_1, ..., K_{n-1}, V_{n-2}, V_{n-1}, MqT.
+__device__ __forceinline__ int pos_k(int i) { return i == 0 ? 0 : 2 * i - 1; }
+__device__ __forceinline__ int pos_v(int i, int n) { return i + 1 < n ? 2 * i + 2 : 2 * i + 1; }
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  const bool ok = mbar_wait(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Pairs after `pair` whose first segment continues block (bh, blk); every
+// pair's range is non-empty, so they are pairs pair + 1 .. pair + n.  -1 if
+// more than kMaxContrib (the host partition rules that out).
+__device__ __forceinline__ int contributors(const AttnParams& p, int pair, const Seg& s) {
+  const unsigned block_end = (unsigned(s.bh) * unsigned(p.n_blk) + unsigned(s.blk) + 1u) * unsigned(p.nkv);
+  const int pairs = p.grid / 2;
+  int n = 0;
+  while (pair + 1 + n < pairs && p.range[pair + 1 + n] < block_end) ++n;
+  return n <= kMaxContrib ? n : -1;
+}
+
+__device__ __forceinline__ float* slot_of(const AttnParams& p, int cta) {
+  return p.scratch + size_t(cta) * kAttnPairSlotFloats;
+}
+
+// ------------------------------------------------------------------ producer
+// One thread per CTA.  Rank 0 announces the bytes of both CTAs on its own
+// barriers; each CTA loads its own halves with rank 0's barrier as the target.
+__device__ __forceinline__ void producer(const AttnParams& p, uint64_t* bars, uint8_t* sQ, uint8_t* sR,
+                                         const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                         const CUtensorMap* tm_mq, const int rank, const unsigned u_begin,
+                                         const unsigned u_end, const WaitCtl& w) {
+  uint32_t ring = 0, k = 0;
+  unsigned u = u_begin;
+  Seg s;
+  const bool lead = rank == 0;
+  while (next_seg(p, u, u_end, s)) {
+    const int b = s.bh / p.heads, h = s.bh % p.heads;
+    const int n = s.j1 - s.j0;
+    const bool writer = s.j0 == 0;
+    const int ntiles = 2 * n + ((writer && p.has_inter) ? 1 : 0);
+    const int x0 = h * 128;
+    const uint32_t qs = k & 1;
+    // Q of this segment, once the MMAs of segment k - 2 have released the slot
+    if (k >= 2 && !mbar_wait(&bars[B_QE + qs], ((k >> 1) - 1) & 1, w)) return;
+    if (lead) mbar_expect_tx(&bars[B_QF + qs], 2 * kQTile);
+    const int qrow = (2 * s.blk + rank) * 128;
+    tma_load_3d_pair(sQ + qs * kQTile, tm_q, &bars[B_QF + qs], x0, qrow, b);
+    tma_load_3d_pair(sQ + qs * kQTile + kBox, tm_q, &bars[B_QF + qs], x0 + 64, qrow, b);
+    for (int t = 0; t < ntiles; ++t) {
+      const uint32_t slot = ring % kRing;
+      if (ring >= kRing && !mbar_wait(&bars[B_RE + slot], ((ring / kRing) - 1) & 1, w)) return;
+      uint8_t* dst = sR + slot * kSlot;
+      if (lead) mbar_expect_tx(&bars[B_RF + slot], 2 * kSlot);
+      if (t < 2 * n) {
+        // position t holds K_i or V_i (see pos_k / pos_v)
+        int i, is_v;
+        if (t == 0) {
+          i = 0, is_v = 0;
+        } else if (t == 2 * n - 1) {
+          i = n - 1, is_v = 1;
+        } else if (t & 1) {
+          i = (t + 1) >> 1, is_v = 0;
+        } else {
+          i = (t - 2) >> 1, is_v = 1;
+        }
+        const int j = s.j0 + i;
+        if (is_v) {  // all 128 keys, this CTA's 64 head dimensions
+          tma_load_3d_pair(dst, tm_v, &bars[B_RF + slot], x0 + 64 * rank, j * 128, b);
+        } else {     // this CTA's 64 keys, all 128 head dimensions
+          tma_load_3d_pair(dst, tm_k, &bars[B_RF + slot], x0, j * 128 + 64 * rank, b);
+          tma_load_3d_pair(dst + kSlot / 2, tm_k, &bars[B_RF + slot], x0 + 64, j * 128 + 64 * rank, b);
+        }
+      } else {  // this CTA's 64 rows of MqT
+        tma_load_3d_pair(dst, tm_mq, &bars[B_RF + slot], 0, 64 * rank, s.bh);
+        tma_load_3d_pair(dst + kSlot / 2, tm_mq, &bars[B_RF + slot], 64, 64 * rank, s.bh);
+      }
+      ++ring;
+    }
+    ++k;
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+// S (or X) over K = 128: A = the CTA's 128 query rows (two 64-column boxes
+// 16 KB apart), B = its half of a K tile or of MqT (64 rows, boxes 8 KB apart).
+__device__ __forceinline__ void mma_s_group(const uint32_t d, const uint32_t a_lo, const uint32_t b_lo,
+                                            const uint32_t hi, const uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_pair_ss(d, a_lo + (kk >> 2) * (kBox >> 4) + (kk & 3) * 2, b_lo + (kk >> 2) * ((kSlot / 2) >> 4) + (kk & 3) * 2,
+                hi, idesc, kk > 0);
+}
+
+// O (+)= P V over nk 16-key steps: P from tensor memory, V MN-major (the
+// CTA's 64 head dimensions, one 128-byte row per key).
+__device__ __forceinline__ void mma_pv_group(const uint32_t d, const uint32_t p_tmem, const uint32_t v_lo,
+                                             const uint32_t hi, const uint32_t idesc, const int nk, const bool acc0) {
+  if (nk == 8) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) mma_pair_ts(d, p_tmem + kk * 8, v_lo + kk * 128, hi, idesc, kk > 0 || acc0);
+  } else {
+    for (int kk = 0; kk < nk; ++kk) mma_pair_ts(d, p_tmem + kk * 8, v_lo + kk * 128, hi, idesc, kk > 0 || acc0);
+  }
+}
+
+// One thread of rank 0.  Per segment (n key tiles, chain c = i & 1 of tile i):
+//   S(0);  for i: S(i+1) (into the buffer PV(i-1) has just read: tcgen05.mma
+//   operations of one thread run in issue order), then PV(i) once both CTAs'
+//   softmax has written P(i);  X = Q MqT^T into S_1 for blocks finished here.
+// Before a segment's S(1) and PV(0) the epilogues must be done with the
+// previous segment's X and O (B_EO).
+__device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, const uint32_t tmem,
+                                           const uint32_t q_addr, const uint32_t r_addr, const unsigned u_begin,
+                                           const unsigned u_end, const WaitCtl& w) {
+  constexpr uint32_t kQ16 = kQTile >> 4, kSlot16 = kSlot >> 4;
+  const uint32_t id_s = idesc_bf16(256, 128, 0, 0);
+  const uint32_t id_o = idesc_bf16(256, 128, 0, 1);
+  const uint64_t dq64 = smem_desc_sw128(q_addr, 16, 1024);
+  const uint32_t hi = uint32_t(dq64 >> 32);
+  const uint32_t dq0 = uint32_t(dq64);
+  const uint32_t dk0 = uint32_t(smem_desc_sw128(r_addr, 16, 1024));     // K-major ring slot
+  const uint32_t dv0 = uint32_t(smem_desc_sw128(r_addr, kBox, 1024));   // MN-major ring slot
+  uint32_t ring = 0, k = 0, g[2] = {0, 0};
+  unsigned u = u_begin;
+  Seg s;
+  while (next_seg(p, u, u_end, s)) {
+    const int n = s.j1 - s.j0;
+    const uint32_t qs = k & 1;
+    const uint32_t dq = dq0 + qs * kQ16;
+    if (!mbar_wait(&bars[B_QF + qs], (k >> 1) & 1, w)) return;
+    const uint32_t r0 = ring;
+    if (!mbar_wait(&bars[B_RF + r0 % kRing], (r0 / kRing) & 1, w)) return;
+    mma_s_group(tmem, dq, dk0 + (r0 % kRing) * kSlot16, hi, id_s);
+    mma_commit_pair(&bars[B_SF + 0]);
+    mma_commit_pair(&bars[B_RE + r0 % kRing]);
+    for (int i = 0; i < n; ++i) {
+      const int c = i & 1;
+      if (i + 1 < n) {
+        const uint32_t rk = r0 + pos_k(i + 1);
+        if (!mbar_wait(&bars[B_RF + rk % kRing], (rk / kRing) & 1, w)) return;
+        if (i == 0 && k > 0) {  // S_1 may hold the previous segment's X
+          if (!mbar_wait(&bars[B_EO], (k - 1) & 1, w)) return;
+          tc_fence_after();
+        }
+        mma_s_group(tmem + ((i + 1) & 1) * 128, dq, dk0 + (rk % kRing) * kSlot16, hi, id_s);
+        mma_commit_pair(&bars[B_SF + ((i + 1) & 1)]);
+        mma_commit_pair(&bars[B_RE + rk % kRing]);
+      }
+      const uint32_t rv = r0 + pos_v(i, n);
+      if (!mbar_wait(&bars[B_RF + rv % kRing], (rv / kRing) & 1, w)) return;
+      if (!mbar_wait(&bars[B_PF + c], g[c] & 1, w)) return;
+      ++g[c];
+      if (i == 0 && n == 1 && k > 0 && !mbar_wait(&bars[B_EO], (k - 1) & 1, w)) return;
+      tc_fence_after();
+      const int valid = min(128, p.kv_len - (s.j0 + i) * 128);
+      mma_pv_group(tmem + 256 + c * 128, tmem + c * 128, dv0 + (rv % kRing) * kSlot16, hi, id_o, (valid + 15) >> 4,
+                   i >= 2);
+      mma_commit_pair(&bars[B_RE + rv % kRing]);
+    }
+    ring = r0 + 2 * n;
+    if (s.j0 == 0 && p.has_inter) {  // X = Q MqT^T for the rows this pair finishes
+      const uint32_t rm = ring;
+      if (!mbar_wait(&bars[B_RF + rm % kRing], (rm / kRing) & 1, w)) return;
+      mma_s_group(tmem + 128, dq, dk0 + (rm % kRing) * kSlot16, hi, id_s);
+      mma_commit_pair(&bars[B_RE + rm % kRing]);
+      ++ring;
+    }
+    mma_commit_pair(&bars[B_SD]);
+    mma_commit_pair(&bars[B_QE + qs]);
+    ++k;
+  }
+}
+
+// ------------------------------------------------------------------ softmax
+// One warpgroup per chain, one query row per thread.  Per key tile of the
+// chain: the 128-column row of S from tensor memory; its maximum; lazy
+// rescaling (the running max m moves only when the tile's max exceeds it by
+// more than 8, a factor 256, and then O_c is rescaled in tensor memory --
+// stable there, since the commit that announced S tracks the chain's previous
+// PV); P = 2^(S * scale * log2(e) - m) packed to bf16 pairs over S's first 64
+// columns; the running row sum l.  At the end of a segment (m, l) go to shared
+// memory for the epilogue.
+__device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars, float* stats, const uint32_t tmem,
+                                             const int c, const int quarter, const int lane, const unsigned u_begin,
+                                             const unsigned u_end, const WaitCtl& w) {
+  const int row = quarter * 32 + lane;
+  const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+  const uint32_t tS = tmem + c * 128, tO = tmem + 256 + c * 128;
+  const uint32_t pf_leader = cluster_map(smem_u32(&bars[B_PF + c]), 0);
+  const float sl2 = p.scale_log2;
+  uint32_t g = 0, k = 0;
+  unsigned u = u_begin;
+  Seg s;
+  while (next_seg(p, u, u_end, s)) {
+    const int n = s.j1 - s.j0;
+    float m = -INFINITY, l = 0.f;
+    for (int i = c; i < n; i += 2) {
+      if (!warp_wait(&bars[B_SF + c], g & 1, w)) return;
+      ++g;
+      tc_fence_after();
+      const int valid = min(128, p.kv_len - (s.j0 + i) * 128);
+      uint32_t r[128];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(tS + lane_off + q * 32, slice32(r, q));
+      tmem_wait_ld();
+      if (valid < 128) {
+#pragma unroll
+        for (int x = 0; x < 128; ++x)
+          if (x >= valid) r[x] = __float_as_uint(-INFINITY);
+      }
+      float m4[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        m4[q] = fmax3(__uint_as_float(r[q]), __uint_as_float(r[4 + q]), __uint_as_float(r[8 + q]));
+#pragma unroll
+      for (int x = 12; x < 124; x += 8)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], __uint_as_float(r[x + q]), __uint_as_float(r[x + 4 + q]));
+#pragma unroll
+      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], __uint_as_float(r[124 + q]));
+      const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl2;
+      float f = 1.f;
+      bool any_rescale = false;
+      if (i == c) {
+        m = mx;
+      } else {
+        const bool need = mx > m + 8.f;
+        any_rescale = __any_sync(0xffffffffu, need);
+        if (need) {
+          f = fast_exp2(m - mx);
+          m = mx;
+        }
+      }
+      const float2 sc = make_float2(sl2, sl2), nm = make_float2(-m, -m);
+      float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float2 y = __ffma2_rn(
+              make_float2(__uint_as_float(r[q * 32 + 2 * x]), __uint_as_float(r[q * 32 + 2 * x + 1])), sc, nm);
+          const float2 e = make_float2(fast_exp2(y.x), fast_exp2(y.y));
+          s2[x & 3] = __fadd2_rn(s2[x & 3], e);
+          pk[x] = pack_bf16x2(e.x, e.y);
+        }
+        tmem_st16(tS + lane_off + q * 16, pk);
+      }
+      const float2 s01 = __fadd2_rn(s2[0], s2[1]), s23 = __fadd2_rn(s2[2], s2[3]);
+      const float2 sa = __fadd2_rn(s01, s23);
+      l = fmaf(l, f, sa.x + sa.y);
+      tmem_wait_st();
+      if (any_rescale) {  // rare: O_c is rescaled before P is announced, so the PV sees a consistent O_c
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + q * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
+          tmem_st32(tO + lane_off + q * 32, o);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(pf_leader);
+    }
+    // the epilogue has read the previous segment's statistics
+    if (k > 0 && !warp_wait(&bars[B_SC], (k - 1) & 1, w)) return;
+    stats[(c * 2 + 0) * 128 + row] = m;
+    stats[(c * 2 + 1) * 128 + row] = l;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[B_ST]);
+    ++k;
+  }
+}
+
+// ------------------------------------------------------------------ epilogue
+// 16-byte chunk i (four floats, columns 4i..4i+3) of row r of an fp32 partial
+// slot lies at float index (i * 128 + r) * 4, so a warp's chunk is one
+// contiguous 512-byte span; (m, l) follow at kPartStats.
+constexpr int kPartStats = 128 * 128;
+
+// One warpgroup, one query row per thread.  At the end of a segment (its MMAs
+// done, both chains' statistics in shared memory):
+//  * own piece: m = max(m_0, m_1), l = l_0 a_0 + l_1 a_1, O = (O_0 a_0 + O_1 a_1) / l
+//    with a_c = 2^(m_c - m);
+//  * a segment that does not start at key tile 0 (a contributor) stores its
+//    piece (O normalised, m, l) in fp32 and raises this warp's ready flag;
+//  * a segment holding a whole block writes O (+ X) through per-warp staging
+//    boxes and TMA tile stores;
+//  * a segment that starts a block continued by the next pairs (always the
+//    pair's last segment) also waits for those pairs' flags and merges their
+//    pieces in key order before adding X.
+// Tensor memory is handed back (B_EO on rank 0) as soon as it has been read.
+__device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bars, const float* stats, uint8_t* stage,
+                                              const CUtensorMap* tm_o, const uint32_t tmem, const int cta,
+                                              const int rank, const int quarter, const int lane,
+                                              const unsigned u_begin, const unsigned u_end, volatile int* abort_flag,
+                                              const WaitCtl& w) {
+  const int row = quarter * 32 + lane;
+  const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+  const uint32_t eo_leader = cluster_map(smem_u32(&bars[B_EO]), 0);
+  const bool use_intra = !(p.flags & 2u);
+  const bool use_inter = p.has_inter && !(p.flags & 1u);
+  const int pair = cta >> 1;
+  uint32_t k = 0;
+  bool staged = false;
+  uint8_t* wst = stage + quarter * 8192;
+  unsigned u = u_begin;
+  Seg s;
+  while (next_seg(p, u, u_end, s)) {
+    const int n = s.j1 - s.j0;
+    const int b = s.bh / p.heads, h = s.bh % p.heads;
+    const bool writer = s.j0 == 0, full = writer && s.j1 == p.nkv;
+    const int qt = 2 * s.blk + rank;
+    const bool row_ok = qt * 128 + row < p.q_len;
+    const bool warp_on = qt * 128 + quarter * 32 < p.q_len;  // warp-uniform
+    int n_contrib = 0;
+    if (writer && !full && (n_contrib = contributors(p, pair, s)) < 0) {
+      record_error(p.err, kDevBadShape);  // the host partition rules this out
+      *abort_flag = 1;
+      return false;
+    }
+    if (!warp_wait(&bars[B_SD], k & 1, w)) return false;
+    if (!warp_wait(&bars[B_ST], k & 1, w)) return false;
+    tc_fence_after();
+    const float m0 = stats[0 * 128 + row], l0 = stats[1 * 128 + row];
+    const float m1 = n > 1 ? stats[2 * 128 + row] : -INFINITY, l1 = n > 1 ? stats[3 * 128 + row] : 0.f;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[B_SC]);
+    const float M = fmaxf(m0, m1);
+    const float e0 = fast_exp2(m0 - M), e1 = n > 1 ? fast_exp2(m1 - M) : 0.f;
+    const float L = l0 * e0 + l1 * e1;
+    // weights of this pair's own piece and of the contributors' pieces
+    float a0 = 0.f, a1 = 0.f, wk[kMaxContrib];
+#pragma unroll
+    for (int q = 0; q < kMaxContrib; ++q) wk[q] = 0.f;
+    if (!writer) {
+      const float inv = 1.f / L;
+      a0 = e0 * inv;
+      a1 = e1 * inv;
+    } else if (n_contrib == 0) {
+      const float inv = row_ok ? 1.f / L : 0.f;
+      a0 = e0 * inv;
+      a1 = e1 * inv;
+    } else {
+      // the contributors' flags (one per warp of their epilogue), then their statistics
+      if (lane == 0) {
+        for (int q = 0; q < n_contrib && !*abort_flag; ++q) {
+          const unsigned* f = p.ready + (size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter;
+          const uint64_t t0 = global_timer_ns();
+          while (ld_acquire(f) == 0u) {
+            if (*abort_flag || global_timer_ns() - t0 > p.wait_limit_ns) {
+              *abort_flag = 1;
+              record_error(p.err, kDevTimeout);
+              break;
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (*abort_flag) return false;
+      for (int q = 0; q < n_contrib; ++q)  // every lane acquires what the contributors released
+        (void)ld_acquire(p.ready + (size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter);
+      float mk[kMaxContrib], lk[kMaxContrib];
+      float Mx = M;
+#pragma unroll
+      for (int q = 0; q < kMaxContrib; ++q) {
+        mk[q] = -INFINITY;
+        lk[q] = 0.f;
+        if (q < n_contrib) {
+          const float* st = slot_of(p, 2 * (pair + 1 + q) + rank) + kPartStats;
+          mk[q] = st[row];
+          lk[q] = st[128 + row];
+        }
+        Mx = fmaxf(Mx, mk[q]);
+      }
+      const float es = fast_exp2(M - Mx);
+      float Lx = L * es;
+#pragma unroll
+      for (int q = 0; q < kMaxContrib; ++q) {
+        wk[q] = q < n_contrib ? lk[q] * fast_exp2(mk[q] - Mx) : 0.f;
+        Lx += wk[q];
+      }
+      const float inv = row_ok ? 1.f / Lx : 0.f;
+      a0 = e0 * es * inv;
+      a1 = e1 * es * inv;
+#pragma unroll
+      for (int q = 0; q < kMaxContrib; ++q) wk[q] *= inv;
+    }
+    if (!use_intra) a0 = a1 = 0.f;
+    const float2 A0 = make_float2(a0, a0), A1 = make_float2(a1, a1);
+    if (!writer) {  // ------------------------------------------------------ contributor
+      float* slot = slot_of(p, cta);
+      float4* d4 = reinterpret_cast<float4*>(slot) + row;
+#pragma unroll 1
+      for (int q = 0; q < 8; ++q) {  // 16 columns at a time
+        uint32_t o0[16], o1[16];
+        tmem_ld16(tmem + 256 + lane_off + q * 16, o0);
+        if (n > 1) tmem_ld16(tmem + 384 + lane_off + q * 16, o1);
+        tmem_wait_ld();
+        float2* v = reinterpret_cast<float2*>(o0);
+        const float2* v1 = reinterpret_cast<const float2*>(o1);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) v[x] = n > 1 ? __ffma2_rn(v1[x], A1, __fmul2_rn(v[x], A0)) : __fmul2_rn(v[x], A0);
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+          d4[(4 * q + x) * 128] = make_float4(v[2 * x].x, v[2 * x].y, v[2 * x + 1].x, v[2 * x + 1].y);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(eo_leader);
+      slot[kPartStats + row] = M;
+      slot[kPartStats + 128 + row] = L;
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) st_release(p.ready + size_t(cta) * 4 + quarter, 1u);
+      ++k;
+      continue;
+    }
+    // ------------------------------------------------------------------ writer
+    if (lane == 0 && staged) bulk_wait_read0();  // this warp's previous tile store has read its boxes
+    __syncwarp();
+#pragma unroll 1
+    for (int q = 0; q < 8; ++q) {  // 16 columns at a time
+      uint32_t o0[16], o1[16], rx[16];
+      tmem_ld16(tmem + 256 + lane_off + q * 16, o0);
+      if (n > 1) tmem_ld16(tmem + 384 + lane_off + q * 16, o1);
+      if (use_inter) tmem_ld16(tmem + 128 + lane_off + q * 16, rx);
+      tmem_wait_ld();
+      float2* v = reinterpret_cast<float2*>(o0);
+      const float2* v1 = reinterpret_cast<const float2*>(o1);
+#pragma unroll
+      for (int x = 0; x < 8; ++x) v[x] = n > 1 ? __ffma2_rn(v1[x], A1, __fmul2_rn(v[x], A0)) : __fmul2_rn(v[x], A0);
+      if (n_contrib > 0 && use_intra) {
+#pragma unroll 1
+        for (int c2 = 0; c2 < n_contrib; ++c2) {
+          const float4* src = reinterpret_cast<const float4*>(slot_of(p, 2 * (pair + 1 + c2) + rank)) + row;
+          const float2 W = make_float2(wk[c2], wk[c2]);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float4 t4 = src[(4 * q + x) * 128];
+            v[2 * x] = __ffma2_rn(make_float2(t4.x, t4.y), W, v[2 * x]);
+            v[2 * x + 1] = __ffma2_rn(make_float2(t4.z, t4.w), W, v[2 * x + 1]);
+          }
+        }
+      }
+      if (use_inter) {
+        const float2* x2 = reinterpret_cast<const float2*>(rx);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) v[x] = __fadd2_rn(v[x], x2[x]);
+      }
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int ch = 2 * q + x;  // 16-byte chunk of the row: box ch / 8, chunk ch % 8 swizzled by row
+        *reinterpret_cast<uint4*>(wst + (ch >> 3) * 4096 + lane * 128 + (((ch & 7) ^ (lane & 7)) << 4)) =
+            make_uint4(pack_bf16x2(v[4 * x].x, v[4 * x].y), pack_bf16x2(v[4 * x + 1].x, v[4 * x + 1].y),
+                       pack_bf16x2(v[4 * x + 2].x, v[4 * x + 2].y), pack_bf16x2(v[4 * x + 3].x, v[4 * x + 3].y));
+      }
+    }
+    tc_fence_before();
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_cluster(eo_leader);
+      if (warp_on) {
+        tma_store_3d(tm_o, wst, h * 128, qt * 128 + quarter * 32, b);
+        tma_store_3d(tm_o, wst + 4096, h * 128 + 64, qt * 128 + quarter * 32, b);
+        bulk_commit();
+      }
+    }
+    staged = true;
+    if (n_contrib > 0 && lane == 0) {  // the pieces are read: their flags go back to zero for the next launch
+      for (int q = 0; q < n_contrib; ++q) p.ready[(size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter] = 0u;
+    }
+    ++k;
+  }
+  if (lane == 0) bulk_wait0();
+  return true;
+}
+
+// ------------------------------------------------------------------ kernel
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_mq,
+                 const __grid_constant__ CUtensorMap tm_o, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                               // [2] Q slots
+  uint8_t* sR = smem + 2 * kQTile;                  // [kRing] half tiles
+  uint8_t* sStage = sR + kRing * kSlot;             // output staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTilesBytes);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* stats = reinterpret_cast<float*>(smem + kTilesBytes + kBarBytes);  // [2 chains][m, l][128]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  const int rank = int(cluster_ctarank());
+  const int pair = cta >> 1;
+  const unsigned u_begin = p.range[pair], u_end = p.range[pair + 1];
+  // The same offset in both CTAs (the launch gives both the same dynamic
+  // shared memory); a layout that does not fit is refused by both.
+  const bool fits = size_t(smem - smem_raw) + kTilesBytes + kBarBytes + kStatsBytes <= size_t(kSmem);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_COUNT; ++i) {
+      uint32_t count = 1;
+      if (i == B_PF || i == B_PF + 1 || i == B_EO) count = 8;  // 4 warps x 2 CTAs (rank 0's copies)
+      if (i == B_ST) count = 8;                                // 4 warps x 2 chains (local)
+      if (i == B_SC) count = 4;                                // the epilogue's 4 warps (local)
+      mbar_init(&bars[i], count);
+    }
+    *abort_flag = fits ? 0 : 1;
+    if (!fits) record_error(p.err, kDevBadShape);
+    fence_barrier_init();
+  }
+  if (warp == 2) tmem_alloc_pair(tmem_holder, 512);
+  tc_fence_before();
+  __syncthreads();
+  cluster_barrier();  // both CTAs' barriers initialised before any remote arrive or load
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtl w{abort_flag, p.err, p.wait_limit_ns};
+  const int wg = warp >> 2;
+  if (!*abort_flag) {
+    if (wg == 0) {
+      regs_dec<kCtlRegs>();
+      if (warp == 0 && lane == 0) {
+        tma_prefetch(&tm_q);
+        tma_prefetch(&tm_k);
+        tma_prefetch(&tm_v);
+        producer(p, bars, sQ, sR, &tm_q, &tm_k, &tm_v, &tm_mq, rank, u_begin, u_end, w);
+      } else if (warp == 1 && lane == 0 && rank == 0) {
+        mma_issuer(p, bars, tmem, smem_u32(sQ), smem_u32(sR), u_begin, u_end, w);
+      }
+      __syncwarp();
+    } else if (wg == 3) {
+      regs_dec<kEpiRegs>();
+      epilogue_role(p, bars, stats, sStage, &tm_o, tmem, cta, rank, warp & 3, lane, u_begin, u_end, abort_flag, w);
+    } else {
+      regs_inc<kSoftmaxRegs>();
+      softmax_role(p, bars, stats, tmem, wg - 1, warp & 3, lane, u_begin, u_end, w);
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  // Every MMA issued by rank 0 has completed and every commit it made has
+  // arrived in both CTAs once the drain commit (the last one) has arrived:
+  // only then may either CTA release its shared and tensor memory.
+  if (warp == 1 && lane == 0) {
+    if (rank == 0) mma_commit_pair(&bars[B_DRAIN]);
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(&bars[B_DRAIN], 0) && global_timer_ns() - t0 < 10000000ull) {
+    }
+  }
+  if (*abort_flag) {
+    // A wait ran out (here or, through a barrier that never completed, in the
+    // other CTA): let this CTA's own copies land before its shared memory is
+    // released.
+    if (warp == 0 && lane == 0) {
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 2000000ull) {
+      }
+    }
+    if (wg == 3 && lane == 0) bulk_wait0();
+  }
+  __syncthreads();
+  cluster_barrier();  // neither CTA leaves while the other may still signal its barriers
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tmq, const CUtensorMap& tmo, const AttnParams& p,
+                             cudaStream_t stream) {
+  static unsigned done = 0;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(attn_pair_kernel), kSmem, &done);
+  if (e != cudaSuccess) return e;
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attn_pair_kernel);
+    if (e != cudaSuccess) return e;
+    regs = fa.numRegs;
+  }
+  if (regs != kLaunchRegs) return cudaErrorInvalidConfiguration;  // the register split needs this count
+  if (p.grid < 2 || (p.grid & 1)) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = stream;
+  // Every pair must be resident at once (a finishing pair waits for the
+  // pieces of the pairs after it): the grid may not exceed the number of
+  // clusters the device can hold.
+  static int capacity = -1;
+  if (capacity < 0) {
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, attn_pair_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    capacity = n;
+  }
+  if (p.grid / 2 > capacity) return cudaErrorCooperativeLaunchTooLarge;
+  return cudaLaunchKernelEx(&cfg, attn_pair_kernel, tq, tk, tv, tmq, tmo, p);
+}
+
+int attn_pair_capacity() {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  static unsigned done = 0;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(attn_pair_kernel), kSmem, &done) != cudaSuccess) return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, attn_pair_kernel, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+bool attn_pair_partition(AttnParams& p, int batch, int max_pairs) {
+  p.n_qt = (p.q_len + 127) / 128;
+  p.n_pair = p.n_qt / 2;
+  p.n_blk = (p.n_qt + 1) / 2;
+  p.nkv = (p.kv_len + 127) / 128;
+  const long long bh = (long long)batch * p.heads;
+  const long long units = bh * p.n_blk * p.nkv;
+  if (units >= (1LL << 31)) return false;
+  p.total_units = units;
+  // Each pair takes at least an eighth of a block, so a block is split across
+  // at most nine pairs (the finishing pair reads at most eight pieces).
+  const long long u_min = (p.nkv + kMaxContrib - 1) / kMaxContrib;
+  long long pairs = units / (u_min > 0 ? u_min : 1);
+  if (pairs > max_pairs) pairs = max_pairs;
+  if (pairs > kAttnMaxGrid / 2) pairs = kAttnMaxGrid / 2;
+  if (pairs < 1) return false;
+  p.grid = int(2 * pairs);
+  for (int c = 0; c <= int(pairs); ++c) p.range[c] = unsigned(units * c / pairs);
+  return true;
+}
+
+}  // namespace arl2

@@ -8,13 +8,11 @@
 // (ARL2 summary, section 2.1: the frozen pretrained Q/K/V projections feed
 // both branches; alpha and beta are per-token learned projections; the
 // pooling of alpha over the frame is this build's reading.)  The projections
-// are plain GEMMs on cuBLAS (bf16 in, fp32 accumulate): one GEMM against the
-// column-concatenated [W_qkv | W_gate] gives Q, K, V and the gates' logits
-// side by side in each token's row, which the layer reads as strided views;
-// the hybrid layer is this library's own handle; the gates are one small
-// kernel here.
-
-#include <cublas_v2.h>
+// run on this library's tcgen05 GEMM (gemm_bf16.cu; bf16 in, fp32
+// accumulate): one GEMM against the column-concatenated [W_qkv | W_gate]
+// gives Q, K, V and the gates' logits side by side in each token's row, which
+// the layer reads as strided views; the hybrid layer is this library's own
+// handle; the gates are one small kernel here.
 
 #include <cstdint>
 #include <mutex>
@@ -56,7 +54,6 @@ __global__ void __launch_bounds__(256) block_gates_kernel(const __nv_bfloat16* _
 namespace {
 
 constexpr uint64_t kBlockMagic = 0x41524c32424c4b31ull;  // "ARL2BLK1"
-constexpr size_t kBlasWorkspace = size_t(32) << 20;
 
 std::mutex g_block_mu;
 std::set<const void*> g_blocks;
@@ -69,7 +66,7 @@ struct arl2_block {
   uint64_t magic;
   arl2_config cfg;
   arl2_state_t layer;
-  cublasHandle_t blas;
+  int sms;       // persistent GEMM grid
   int64_t ldw;   // columns of w_all and qkvg: 3D, then 2H gate columns, padded to a multiple of 8
   void* w_all;   // [D, ldw] bf16: W_qkv | W_gate | 0
   void* w_o;
@@ -77,7 +74,6 @@ struct arl2_block {
   void* o;
   float* alpha;
   float* beta;
-  void* ws;
 };
 
 namespace {
@@ -95,33 +91,34 @@ bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0
 
 void free_block(arl2_block* b) {
   if (b->layer) arl2_state_destroy(b->layer);
-  if (b->blas) cublasDestroy(b->blas);
-  for (void* p : {b->w_all, b->w_o, b->qkvg, b->o, (void*)b->alpha, (void*)b->beta, b->ws})
+  for (void* p : {b->w_all, b->w_o, b->qkvg, b->o, (void*)b->alpha, (void*)b->beta})
     if (p) cudaFree(p);
   b->magic = 0;
   delete b;
 }
 
-// Row-major C[M][N] (ldc) = A[M][K] (lda) * B[K][N] (ldb): the column-major
-// product C^T = B^T A^T.  bf16 operands, fp32 accumulation, C in `ctype`.
-bool gemm(cublasHandle_t h, int M, int N, int K, const void* A, int lda, const void* B, int ldb, void* C, int ldc,
-          cudaDataType_t ctype) {
-  const float one = 1.f, zero = 0.f;
-  return cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, N, M, K, &one, B, CUDA_R_16BF, ldb, A, CUDA_R_16BF, lda, &zero, C,
-                      ctype, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS;
+// Row-major C[M][N] (ldc) = A[M][K] (lda) * B[K][N] (ldb) on the library's
+// GEMM; a wait that runs out is recorded in the layer's error word.
+arl2_status gemm(const arl2_block* b, int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t ldb,
+                 void* C, int64_t ldc, cudaStream_t st) {
+  arl2::GemmParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.err = arl2::layer_error_word(b->layer);
+  p.wait_limit_ns = arl2::layer_wait_limit(b->layer);
+  return arl2::gemm_bf16(A, lda, B, ldb, C, ldc, p, b->sms, st) == cudaSuccess ? ARL2_OK : ARL2_ERR_CUDA;
 }
 
 // Q | K | V | gate logits = X [W_qkv | W_gate], one token row each.
 arl2_status project_in(arl2_block* b, const void* x, cudaStream_t st) {
   const int D = b->cfg.heads * b->cfg.head_dim, M = b->cfg.batch * b->cfg.tokens_per_frame;
-  if (cublasSetStream(b->blas, st) != CUBLAS_STATUS_SUCCESS) return ARL2_ERR_CUDA;
-  const int ldw = int(b->ldw);
-  return gemm(b->blas, M, ldw, D, x, D, b->w_all, ldw, b->qkvg, ldw, CUDA_R_16BF) ? ARL2_OK : ARL2_ERR_CUDA;
+  return gemm(b, M, int(b->ldw), D, x, D, b->w_all, b->ldw, b->qkvg, b->ldw, st);
 }
 
-arl2_status project_out(arl2_block* b, void* y) {
+arl2_status project_out(arl2_block* b, void* y, cudaStream_t st) {
   const int D = b->cfg.heads * b->cfg.head_dim, M = b->cfg.batch * b->cfg.tokens_per_frame;
-  return gemm(b->blas, M, D, D, b->o, D, b->w_o, D, y, D, CUDA_R_16BF) ? ARL2_OK : ARL2_ERR_CUDA;
+  return gemm(b, M, D, D, b->o, D, b->w_o, D, y, D, st);
 }
 
 bool overlap(const void* a, const void* c, size_t n) {
@@ -172,7 +169,6 @@ arl2_status arl2_block_init(const arl2_config* cfg, const void* w_qkv, const voi
   alloc(&b->o, M * D * 2);
   alloc(reinterpret_cast<void**>(&b->alpha), size_t(cfg->batch) * H * sizeof(float));
   alloc(reinterpret_cast<void**>(&b->beta), M * H * sizeof(float));
-  alloc(&b->ws, kBlasWorkspace);
   auto* wa = static_cast<__nv_bfloat16*>(b->w_all);
   if (e == cudaSuccess) e = cudaMemsetAsync(b->w_all, 0, D * ldw * 2, st);
   if (e == cudaSuccess)
@@ -184,15 +180,9 @@ arl2_status arl2_block_init(const arl2_config* cfg, const void* w_qkv, const voi
     free_block(b);
     return from_cuda_e(e);
   }
-  // cuBLAS with a fixed workspace allocates nothing per call (so calls may be
-  // captured into CUDA graphs)
-  if (cublasCreate(&b->blas) != CUBLAS_STATUS_SUCCESS) {
-    b->blas = nullptr;
-    free_block(b);
-    return ARL2_ERR_CUDA;
-  }
-  if (cublasSetWorkspace(b->blas, b->ws, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS ||
-      cublasSetMathMode(b->blas, CUBLAS_DEFAULT_MATH) != CUBLAS_STATUS_SUCCESS) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&b->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || b->sms < 1) {
     free_block(b);
     return ARL2_ERR_CUDA;
   }
@@ -214,7 +204,7 @@ arl2_status arl2_block_query(arl2_block_t b, const void* x, void* y, void* strea
   const int D = b->cfg.heads * b->cfg.head_dim;
   const auto* in = static_cast<const __nv_bfloat16*>(b->qkvg);
   if ((s = arl2::layer_query_ld(b->layer, in, in + D, in + 2 * D, b->ldw, b->o, st)) != ARL2_OK) return s;
-  return project_out(b, y);
+  return project_out(b, y, st);
 }
 
 arl2_status arl2_block_commit(arl2_block_t b, const void* x, void* y, void* stream) {
@@ -230,7 +220,7 @@ arl2_status arl2_block_commit(arl2_block_t b, const void* x, void* y, void* stre
   if (cudaGetLastError() != cudaSuccess) return ARL2_ERR_CUDA;
   if ((s = arl2::layer_commit_ld(b->layer, in, in + D, in + 2 * D, b->ldw, b->alpha, b->beta, b->o, st)) != ARL2_OK)
     return s;
-  return project_out(b, y);
+  return project_out(b, y, st);
 }
 
 arl2_state_t arl2_block_layer(arl2_block_t b) { return live_block(b) ? b->layer : nullptr; }

@@ -20,6 +20,11 @@ arl2_status layer_query_ld(::arl2_state* h, const void* q, const void* k, const 
 arl2_status layer_commit_ld(::arl2_state* h, const void* q, const void* k, const void* v, int64_t ld, const float* alpha,
                             const float* beta, void* o, cudaStream_t st);
 
+// The layer handle's device error word and its wait limit, for kernels the
+// attention block launches beside the layer (its GEMMs).
+uint32_t* layer_error_word(::arl2_state* h);
+uint64_t layer_wait_limit(::arl2_state* h);
+
 // The token-level query (commit = false) and commit of a bf16 hybrid-layer
 // handle: arl2_token_query and arl2_token_commit.
 arl2_status token_pass(::arl2_state* h, const void* q, const void* k, const void* v, const float* alpha_tok,

@@ -38,6 +38,19 @@ struct AttnParams {
 // then m[128] and l[128] in fp32
 constexpr int kAttnSlotFloats = 128 * 64 + 256;
 
+// floats of one CTA's partial slot of the CTA-pair kernel (attn_pair.cu): its
+// 128 x 128 piece of O in fp32, normalised by its own l, chunk-major (16-byte
+// chunk i of row r at float (i * 128 + r) * 4), then m[128] and l[128]
+constexpr int kAttnPairSlotFloats = 128 * 128 + 256;
+// ready flags per CTA of the pair kernel (one per epilogue warp)
+constexpr int kAttnPairFlags = 4;
+// device words of the attention scratch and flags a handle allocates for `sms` SMs
+constexpr size_t attn_scratch_floats(int sms) {
+  return size_t(sms) * (2 * size_t(kAttnSlotFloats) > size_t(kAttnPairSlotFloats) ? 2 * size_t(kAttnSlotFloats)
+                                                                                  : size_t(kAttnPairSlotFloats));
+}
+constexpr size_t attn_ready_words(int sms) { return size_t(sms) * kAttnPairFlags; }
+
 // State write and read-out preparation (state_bf16.cu).
 struct StateParams {
   const float* S_prev;      // [B, H, 128, 128]
@@ -90,10 +103,28 @@ cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const
 // Fills the partition fields of `p` for B streams on a device with `sms` SMs;
 // false if the problem is too large for 32-bit unit indices.
 bool attn_partition(AttnParams& p, int batch, int sms);
+// The same on CTA pairs (attn_pair.cu): tk holds 64-row boxes (a CTA's half of
+// a key tile), tv 128-row boxes, tmq 64-row boxes of the [B*H, 128, 128] MqT
+// slabs; p.grid is the CTA count (even), p.range is per pair.
+cudaError_t launch_attn_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tmq, const CUtensorMap& tmo, const AttnParams& p,
+                             cudaStream_t stream);
+// max_pairs: the clusters of two the device holds at once (attn_pair_capacity).
+bool attn_pair_partition(AttnParams& p, int batch, int max_pairs);
+// Clusters of the pair kernel resident at once on the current device (0 on error).
+int attn_pair_capacity();
 cudaError_t launch_state_partial(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tpk,
                                  const CUtensorMap& tpv, const CUtensorMap& ts, const StateParams& p, int batch,
                                  cudaStream_t stream);
 cudaError_t launch_state_finalize(const StateParams& p, int batch, cudaStream_t stream);
+// The whole state write in one launch (state_bf16.cu): one cluster of
+// n_chunks CTAs per (stream, head), reducing the chunks' partials on chip in
+// chunk order (bit-identical to partial + finalize) and forming MqT into p.mqt.
+// Needs n_chunks <= 16 and a device that schedules such clusters.
+bool state_fused_supported(int n_chunks, int heads, int batch);
+cudaError_t launch_state_fused(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tpk,
+                               const CUtensorMap& tpv, const CUtensorMap& ts, const CUtensorMap& tphiq,
+                               const StateParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_readout_prep(const CUtensorMap& ts, const CUtensorMap& tphiq, const StateParams& p, int batch,
                                 cudaStream_t stream);
 cudaError_t launch_f32_attn(const F32AttnParams& p, int batch, cudaStream_t stream);
@@ -102,6 +133,17 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16* src, __nv_bfloat16* dst, 
 cudaError_t launch_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
+
+// Projection GEMM of the attention block (gemm_bf16.cu): C[M][N] = A[M][K] B[K][N],
+// bf16 row-major operands with leading dimensions lda, ldb, ldc (elements,
+// multiples of 8), fp32 accumulation, bf16 C.
+struct GemmParams {
+  int M, N, K;
+  uint32_t* err;
+  uint64_t wait_limit_ns;
+};
+cudaError_t gemm_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc, const GemmParams& p,
+                      int sms, cudaStream_t stream);
 
 // Sets the dynamic shared-memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* done_mask);

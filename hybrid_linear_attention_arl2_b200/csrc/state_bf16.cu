@@ -48,12 +48,49 @@ __device__ __forceinline__ bool warp_wait_s(uint64_t* bar, uint32_t parity, cons
   return __all_sync(0xffffffffu, ok);
 }
 
-enum { P_IN, P_MK, P_PV, P_MV, P_KP, P_S, P_KS, P_R, P_DS, P_DRAIN, P_COUNT };
+enum { P_IN, P_MK, P_PV, P_MV, P_KP, P_S, P_KS, P_R, P_DS, P_PQ, P_MQ, P_DRAIN, P_COUNT };
 
+__device__ __forceinline__ uint32_t cluster_rank_s() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nrank_s() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_dsmem_b16(uint32_t cluster_addr, uint16_t v) {
+  asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(cluster_addr), "h"(v) : "memory");
+}
+
+// Float offset of 16-byte chunk c (columns 4c..4c+3) of row i of a chunk's
+// fp32 partial held in shared memory for the cluster's reduction: chunks are
+// XOR-swizzled by row so that a warp writing one chunk of 32 rows spreads over
+// every bank.
+__device__ __forceinline__ uint32_t part_off(int i, int c) { return uint32_t(i) * 128 + uint32_t((c ^ (i & 31)) << 2); }
+
+// kFused = false: one CTA per 128-token chunk writes its partial delta to
+// global memory (state_finalize_kernel then reduces).  kFused = true: the
+// CTAs of one (stream, head) form a cluster, one per chunk; they reduce their
+// partials through distributed shared memory in chunk order (the same sums,
+// in the same order, as state_finalize_kernel), apply the decay, write S_N and
+// its bf16 copy, and the cluster's rank 0 forms MqT = (phi_q S_N)^T: the whole
+// state write in one launch, with no partial leaving the chip.
+template <bool kFused>
 __global__ void __launch_bounds__(kStateThreads, 2)
 state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_phik_t, const __grid_constant__ CUtensorMap tm_phiv_t,
-                     const __grid_constant__ CUtensorMap tm_s_bf, const StateParams p) {
+                     const __grid_constant__ CUtensorMap tm_s_bf, const __grid_constant__ CUtensorMap tm_phiq,
+                     const StateParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;               // K tile, then K' (bf16)
@@ -66,6 +103,7 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int slab = b * p.heads + h;
+  const int rank = kFused ? int(cluster_rank_s()) : 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < P_COUNT; ++i) mbar_init(&bars[i], (i == P_KP || i == P_R) ? 4u : 1u);
@@ -218,21 +256,126 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[P_R]);
     }
-    // Store this chunk's delta rows (row = state row i).
+    // This chunk's delta rows (row = state row i): to global memory, or (fused)
+    // to this CTA's shared memory for the cluster's reduction (the K and V
+    // tiles are free once the last MMA has completed).
     if (ok) ok = warp_wait_s(&bars[P_DS], 0, w);
     if (ok) {
       tc_fence_after();
-      float* dst = p.partial + ((size_t(slab) * p.n_chunks + chunk) * 128 + row) * 128;
+      float* dst = kFused ? reinterpret_cast<float*>(sK) : p.partial + ((size_t(slab) * p.n_chunks + chunk) * 128 + row) * 128;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(tB + lane_off + c * 32, r);
         tmem_wait_ld();
-        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
-                              __uint_as_float(r[4 * i + 3]));
+        for (int i = 0; i < 8; ++i) {
+          const float4 v4 = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                        __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          if (kFused)
+            *reinterpret_cast<float4*>(dst + part_off(row, c * 8 + i)) = v4;
+          else
+            reinterpret_cast<float4*>(dst + c * 32)[i] = v4;
+        }
+      }
+    }
+  }
+  if (kFused) {
+    // Every CTA of the cluster reaches these barriers, also after a timeout
+    // (ok = false): the cluster's reduction is skipped then, not its barriers.
+    __syncthreads();
+    const int nrank = int(cluster_nrank_s());
+    const bool ok_all = !*abort_flag;
+    // rank 0: phi_q into the tile R occupied (the last MMA has read it)
+    if (rank == 0 && warp == 0 && lane == 0 && ok_all) {
+      mbar_expect_tx(&bars[P_PQ], kTileB);
+      tma_load_3d(sP, &tm_phiq, &bars[P_PQ], 0, 0, h);
+      tma_load_3d(sP + kHalfB, &tm_phiq, &bars[P_PQ], 64, 0, h);
+    }
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    // This rank's rows of S_N: sum the chunks' partials in chunk order (rank
+    // q holds chunk q), then S_N = alpha S_{N-1} + c * sum.
+    const int rpc = (128 + nrank - 1) / nrank;
+    const int i0 = rank * rpc, i1 = min(128, i0 + rpc);
+    const int nchunks16 = max(0, i1 - i0) * 32;  // 16-byte chunks of this rank's rows
+    const uint32_t part_base = smem_u32(sK);
+    const float a = p.alpha[slab];
+    for (int q16 = threadIdx.x; ok_all && q16 < nchunks16; q16 += kStateThreads) {
+      {
+        const int i = i0 + q16 / 32, c = q16 % 32;
+        const uint32_t off = part_base + part_off(i, c) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < nrank; ++q) {
+          const float4 v = ld_dsmem_f4(cluster_map(off, uint32_t(q)));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const size_t e = size_t(slab) * 16384 + size_t(i) * 128 + c * 4;
+        const float4 sp4 = *reinterpret_cast<const float4*>(p.S_prev + e);
+        float4 r;
+        r.x = fmaf(a, sp4.x, p.corr * acc.x);
+        r.y = fmaf(a, sp4.y, p.corr * acc.y);
+        r.z = fmaf(a, sp4.z, p.corr * acc.z);
+        r.w = fmaf(a, sp4.w, p.corr * acc.w);
+        *reinterpret_cast<float4*>(p.S_next + e) = r;
+        const uint2 bf = make_uint2(pack_bf16x2(r.x, r.y), pack_bf16x2(r.z, r.w));
+        *reinterpret_cast<uint2*>(p.S_next_bf + e) = bf;
+      }
+    }
+    // every partial is read: rank 0's K/V tiles take the bf16 S_N for the
+    // read-out MMA (row k = state row, 64-column boxes, 128-byte swizzle: the
+    // layout the tensor cores read as an MN-major operand)
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    // (each thread re-reads the bf16 values it wrote itself)
+    for (int q16 = threadIdx.x; ok_all && q16 < nchunks16; q16 += kStateThreads) {
+      const int i = i0 + q16 / 32, c = q16 % 32;
+      const uint2 bf = *reinterpret_cast<const uint2*>(p.S_next_bf + size_t(slab) * 16384 + size_t(i) * 128 + c * 4);
+      const uint16_t v4[4] = {uint16_t(bf.x & 0xFFFFu), uint16_t(bf.x >> 16), uint16_t(bf.y & 0xFFFFu),
+                              uint16_t(bf.y >> 16)};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) st_dsmem_b16(cluster_map(smem_u32(sK) + sw128_offset(i, 4 * c + x), 0u), v4[x]);
+    }
+    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (rank == 0 && ok_all) {
+      // MqT[j][i] = sum_k S_N[k][j] phi_q[i][k]: M = j, N = i, K = k (as in readout_prep_kernel)
+      if (warp == 1) {
+        if (lane == 0 && mbar_wait(&bars[P_PQ], 0, w)) {
+          tc_fence_after();
+          const uint32_t sa = smem_u32(sK), pa = smem_u32(sP);
+          const uint32_t id = idesc_bf16(128, 128, 1, 0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t boff = (kk >> 2) * kHalfB + (kk & 3) * 32;
+            mma_ss(tA, smem_desc_sw128(sa + kk * 2048, kHalfB, 1024), smem_desc_sw128(pa + boff, 16, 1024), id,
+                   kk > 0);
+          }
+          mma_commit(&bars[P_MQ]);
+        }
+        __syncwarp();
+      } else if (warp >= 2) {
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;  // j
+        const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+        if (warp_wait_s(&bars[P_MQ], 0, w)) {
+          tc_fence_after();
+          __nv_bfloat16* dst = p.mqt + (size_t(slab) * 128 + row) * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tA + lane_off + c * 32, r);
+            tmem_wait_ld();
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              d4[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                                 pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                                 pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                                 pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7])));
+          }
+        }
       }
     }
   }
@@ -378,11 +521,60 @@ cudaError_t launch_state_partial(const CUtensorMap& tk, const CUtensorMap& tv, c
                                  const CUtensorMap& tpv, const CUtensorMap& ts, const StateParams& p, int batch,
                                  cudaStream_t stream) {
   static unsigned done = 0;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(state_partial_kernel), kPartialSmem, &done);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(state_partial_kernel<false>), kPartialSmem, &done);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_chunks, p.heads, batch);
-  state_partial_kernel<<<grid, kStateThreads, kPartialSmem, stream>>>(tk, tv, tpk, tpv, ts, p);
+  state_partial_kernel<false><<<grid, kStateThreads, kPartialSmem, stream>>>(tk, tv, tpk, tpv, ts, ts, p);
   return cudaGetLastError();
+}
+
+namespace {
+cudaLaunchConfig_t fused_config(int n_chunks, int heads, int batch, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_chunks, heads, batch);
+  cfg.blockDim = dim3(kStateThreads);
+  cfg.dynamicSmemBytes = kPartialSmem;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = n_chunks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+cudaError_t fused_attrs() {
+  static unsigned done = 0;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(state_partial_kernel<true>), kPartialSmem, &done);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(state_partial_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+}
+}  // namespace
+
+bool state_fused_supported(int n_chunks, int heads, int batch) {
+  if (n_chunks < 1 || n_chunks > 16) return false;
+  if (fused_attrs() != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = fused_config(n_chunks, heads, batch, attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, state_partial_kernel<true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return n >= 1;
+}
+
+cudaError_t launch_state_fused(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tpk,
+                               const CUtensorMap& tpv, const CUtensorMap& ts, const CUtensorMap& tphiq,
+                               const StateParams& p, int batch, cudaStream_t stream) {
+  cudaError_t e = fused_attrs();
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = fused_config(p.n_chunks, p.heads, batch, attr);
+  cfg.stream = stream;
+  return cudaLaunchKernelEx(&cfg, state_partial_kernel<true>, tk, tv, tpk, tpv, ts, tphiq, p);
 }
 
 cudaError_t launch_state_finalize(const StateParams& p, int batch, cudaStream_t stream) {

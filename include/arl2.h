@@ -133,8 +133,10 @@ arl2_status arl2_frame_commit_strided(arl2_state_t h, const void* q, const void*
  * counter, and refreshes what the frame-level calls read, so the two kinds of
  * call may follow one another on one handle.
  * bf16 handles only.  The first token-level call on a handle allocates its
- * scratch (about 5.2 KB per token and head), so it must not be the first
- * call captured into a CUDA graph.  The arithmetic past the intra-frame
+ * scratch (about 5.2 KB per token and head) with cudaMalloc and adds it to
+ * arl2_state_device_bytes, so that first call must not be made while a
+ * stream is being captured into a CUDA graph (it fails there with
+ * OUT_OF_MEMORY or CUDA); later calls allocate nothing.  The arithmetic past the intra-frame
  * branch is float32.  Errors: INVALID_ARGUMENT, UNSUPPORTED (an f32 handle),
  * OUT_OF_MEMORY, CUDA. */
 arl2_status arl2_token_query(arl2_state_t h, const void* q, const void* k, const void* v, const float* alpha_tok,
@@ -155,7 +157,10 @@ arl2_status arl2_state_set(arl2_state_t h, const float* src, int64_t frame, void
  * recorded by its kernels, ARL2_OK if none. */
 arl2_status arl2_last_error(arl2_state_t h);
 
-/* Device bytes held by the handle (constant over the stream's life). */
+/* Device bytes held by the handle.  Fixed at init and independent of the
+ * frame index, with one exception: the first token-level call
+ * (arl2_token_query / arl2_token_commit) allocates that call's scratch and
+ * adds it to the count, which then stays constant again. */
 int64_t arl2_state_device_bytes(arl2_state_t h);
 
 /* Wall-clock limit of one device-side wait in the handle's kernels (default
@@ -226,6 +231,20 @@ arl2_status arl2_block_commit(arl2_block_t blk, const void* x, void* y, void* st
 arl2_state_t arl2_block_layer(arl2_block_t blk);
 arl2_status arl2_block_destroy(arl2_block_t blk);
 
+/* The attention block's projection GEMM on its own: C = A B with A [M, K],
+ * B [K, N] and C [M, N] row-major bf16 device matrices (leading dimensions
+ * lda >= K, ldb >= N, ldc >= N elements, each a multiple of 8; pointers
+ * 16-byte aligned), fp32 accumulation, C rounded to bf16.  This is the
+ * token-by-weight product that turns the block's input X into Q | K | V | gate
+ * logits and the layer's output O into Y (ARL2 summary, section 2.1: the frozen
+ * Q/K/V projections feed both branches).  C must not overlap A or B.
+ * Errors: INVALID_ARGUMENT (null or misaligned pointers, bad sizes or leading
+ * dimensions, overlap), NO_DEVICE, CUDA.  A device-side wait that runs out is
+ * not reported here: the call has no handle; the block reports it through its
+ * layer (arl2_last_error of arl2_block_layer). */
+arl2_status arl2_gemm_bf16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c, int64_t ldc, int64_t m,
+                           int64_t n, int64_t k, void* stream);
+
 /* ---- State write without allocation ---------------------------------------
  * The paper has no counterpart to this call; it is a deployment aid.  Some
  * callers cannot call cudaMalloc: code that runs while a CUDA graph is being
@@ -245,16 +264,21 @@ arl2_status arl2_block_destroy(arl2_block_t blk);
  *   k, v      : device bf16 [B, L, H, 128];  phi_k, phi_v : device bf16 [H, 128, 128]
  *               as given to arl2_state_init;
  *   S_prev    : device float32 [B, H, 128, 128];  alpha : float32 [B, H];
- *   beta      : float32 [B, H, L];  S_next : device float32 [B, H, 128, 128],
- *               must not overlap S_prev;
+ *   beta      : float32 [B, H, L];  S_next : device float32 [B, H, 128, 128];
  *   dev_error : device uint32, set to 0 by the call and to an arl2_status by a
  *               kernel whose bounded wait ran out (read it after a sync).
+ * S_next and dev_error may share no byte with any input or with each other
+ * (INVALID_ARGUMENT otherwise).
  * All pointers are caller-owned and 16-byte aligned.  The scratch needed is
  *   2 * H * 32768 + 2 * B * H * 32768 + B * H * ceil(L / 128) * 65536 bytes
  * (each part rounded up to 1 KiB); more than ARL2_NOALLOC_SCRATCH_BYTES returns
  * ARL2_ERR_SCRATCH_LIMIT before any CUDA call.  The first call on a device
  * looks up the array's device address (once per device, with that device
- * current); make that first call before any stream capture begins.  Every
+ * current); make that first call before any stream capture begins.  The
+ * library keeps that address for the life of the process, so it must not
+ * outlive the device context it was looked up in: after cudaDeviceReset (or
+ * any other teardown of the device's primary context) do not call this entry
+ * point again in the same process.  Every
  * call shares the one array and leaves its contents behind, so calls whose
  * kernels overlap on the GPU (other streams, other host threads) race:
  * serialise them.  Errors: INVALID_ARGUMENT, UNSUPPORTED, SCRATCH_LIMIT, CUDA. */

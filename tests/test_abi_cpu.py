@@ -73,10 +73,13 @@ def test_kv_validation(lib):
 
 def test_noalloc_state_write_host_checks(lib):
     """The allocation-free state write rejects, before any CUDA call, what it
-    cannot run: a float32 config, null or misaligned pointers, overlapping
-    states, and sizes whose work space exceeds its fixed static array."""
+    cannot run: a float32 config, null or misaligned pointers, an output
+    (S_next or the error word) that shares a byte with an input or with the
+    other output, and sizes whose work space exceeds its fixed static array."""
     L = arl2.load_library()
-    ptrs = [16, 32, 48, 64, 1 << 20, 96, 112, 64 << 20, 144]
+    G = 1 << 30  # fake, never dereferenced addresses 1 GiB apart
+    # k, v, phi_k, phi_v, S_prev, alpha, beta, S_next, dev_error
+    ptrs = [1 * G, 2 * G, 3 * G, 4 * G, 5 * G, 6 * G, 7 * G, 8 * G, 9 * G]
     call = lambda cfg, p=ptrs: L.arl2_state_write_noalloc(ctypes.byref(cfg), *p, None)
     assert call(arl2.make_config(1, 2, 32, 16, arl2.ARL2_F32)) == 2
     assert call(arl2.make_config(1, 2, 64, 16, arl2.ARL2_BF16)) == 2
@@ -85,9 +88,17 @@ def test_noalloc_state_write_host_checks(lib):
     assert call(arl2.make_config(1, 2, 128, 16, arl2.ARL2_BF16), bad) == 1
     bad[0] = 17
     assert call(arl2.make_config(1, 2, 128, 16, arl2.ARL2_BF16), bad) == 1
-    same = list(ptrs)
-    same[7] = same[4]                                                       # S_next over S_prev
-    assert call(arl2.make_config(1, 2, 128, 16, arl2.ARL2_BF16), same) == 1
+    small = arl2.make_config(1, 2, 128, 16, arl2.ARL2_BF16)  # k, v: 8 KiB; states 128 KiB; beta 128 B
+    for out, target, offset in [(7, 4, 0),            # S_next over S_prev
+                                (7, 0, 8192 - 16),    # S_next starts inside the last 16 bytes of k
+                                (7, 1, -128 * 1024 + 16),  # S_next ends inside v
+                                (7, 5, 0), (7, 6, 64),     # over alpha, over beta
+                                (7, 2, 4096),              # over phi_k
+                                (8, 0, 4096), (8, 6, 0),   # the error word inside k, inside beta
+                                (8, 7, 1024)]:             # the error word inside S_next
+        bad = list(ptrs)
+        bad[out] = ptrs[target] + offset
+        assert call(small, bad) == 1, (out, target, offset)
     assert call(arl2.make_config(4, 12, 128, 1560, arl2.ARL2_BF16)) == 7    # 4 streams x 1560 tokens
     assert arl2.arl2_status_string(7).startswith("sizes exceed")
 

@@ -168,3 +168,20 @@ def test_attention_stack_sample():
     for x in list(hyb.values()) + list(kvl.values()):
         assert x.last_error() == 0
         x.close()
+
+
+@pytest.mark.parametrize("index", [1, 4])
+def test_every_query_row_of_a_full_size_pass(index):
+    """Every query row (all 1560, every head and stream) of one query pass and
+    of the commit pass of the second frame, against the oracle: the rows the
+    sampled tests skip include the interior of every query tile and the rows
+    of blocks whose key range the launch splits between CTA pairs."""
+    cfg = W.CONFIGS[index]
+    wl = W.Workload(cfg)
+    keep = lambda n, p: n == 1 and p in (0, cfg.queries)
+    g_out, g_S = run_gpu_stream(cfg, wl, frames=2, keep=keep)
+    r_out, r_S = run_oracle_stream(cfg, wl, frames=2, keep=keep)
+    for key, r in r_out.items():
+        e = max_rel(g_out[key], r)
+        assert e <= OUT_TOL, (key, e)
+    assert frob_rel(g_S[-1], r_S[-1]) <= STATE_TOL
