@@ -14,16 +14,20 @@
 // MMA covers both CTAs' rows (M = 256): rank 0 issues it, each CTA supplies
 // its own 128 rows of the A operand and half of the B operand (64 keys of a K
 // tile, 64 head dimensions of a V tile) and keeps its 128 rows of the
-// accumulator in its own tensor memory.  The key tiles of a block alternate
-// between two chains with their own S buffer, softmax warpgroup, running
-// statistics (m, l) and O accumulator, so that one chain's softmax overlaps
-// the other chain's MMAs; the epilogue merges the two chains.  The sequence
-// of (block, key tile) units over all (stream, head) pairs is cut into
-// contiguous equal ranges, one per CTA pair ("stream-K").  A block whose key
-// range is split across pairs is finished by the pair holding its key tile 0
-// (always that pair's last segment); the pairs continuing it store their
-// normalised partial output and (m, l) in fp32 and raise ready flags, and the
-// finishing pair combines the pieces in key order (deterministic).
+// accumulator in its own tensor memory.  S and P are double-buffered in tensor
+// memory and S is issued two key tiles ahead of the PV that consumes the
+// matching P, so the softmax of tile i finds S(i) ready as soon as it is done
+// with tile i - 1: it never waits for a PV, and the tensor core never waits
+// for the softmax of the tile it is about to compute.  The softmax of one tile
+// is split by columns between two warpgroups (keys 0..63 and 64..127 of the
+// same 128 rows), which exchange their partial row maxima through shared
+// memory.  The sequence of (block, key tile) units over all (stream, head)
+// pairs is cut into contiguous equal ranges, one per CTA pair ("stream-K").  A
+// block whose key range is split across pairs is finished by the pair holding
+// its key tile 0 (always that pair's last segment); the pairs continuing it
+// store their normalised partial output and (m, l) in fp32 and raise ready
+// flags, and the finishing pair combines the pieces in key order
+// (deterministic).
 //
 // Roles per CTA (512 threads, four warpgroups):
 //   warp 0       TMA producer: per segment the CTA's Q tile (two slots, so the
@@ -31,17 +35,20 @@
 //                halves of K_j, V_j (and of MqT for blocks it finishes)
 //                through a ring of 16 KB slots; the loads of both CTAs count
 //                on rank 0's barriers;
-//   warp 1       (rank 0 only) tcgen05 issuer: S(i) = Q K^T, O_c += P V, X = Q MqT^T;
+//   warp 1       (rank 0 only) tcgen05 issuer: S(i) = Q K_i^T, O += P(i) V_i,
+//                X = Q MqT^T;
 //   warp 2       tensor-memory allocator (both CTAs, cta_group::2);
-//   warps 4..7   softmax of chain 0 (one query row per thread);
-//   warps 8..11  softmax of chain 1;
-//   warps 12..15 epilogue: at the end of a segment reads O_0, O_1 (and X)
-//                from tensor memory, hands it back at once, merges the chains
-//                (and, for a split block, the other pairs' pieces) and writes
-//                the output with TMA tile stores, or stores the partial.
-// Tensor memory (512 columns per CTA): S_0 [0,128), S_1 [128,256) (P written
-// in place as bf16 pairs; X goes into S_1 at the end of a segment),
-// O_0 [256,384), O_1 [384,512).
+//   warp 3       (rank 1 only) forwards its softmax warps' per-tile signals to
+//                rank 0's barriers, one cluster-scope arrive per signal;
+//   warps 4..7   softmax, keys 0..63 of every tile (one query row per thread);
+//   warps 8..11  softmax, keys 64..127;
+//   warps 12..15 epilogue: at the end of a segment reads O (and X) from
+//                tensor memory, hands it back at once, merges the other pairs'
+//                pieces of a split block and writes the output with TMA tile
+//                stores, or stores the partial.
+// Tensor memory (512 columns per CTA): S[0] [0,128), S[1] [128,256) (fp32);
+// P[0] [256,320), P[1] [320,384) (bf16 pairs; X = Q MqT^T overlays [256,384)
+// at the end of a segment); O [384,512).
 //
 // Every wait is bounded (mbarriers and peer flags): on expiry the CTA raises
 // its abort flag and records a timeout; there is no named barrier, so a role
@@ -61,15 +68,15 @@ constexpr uint32_t kQTile = 32768;  // 128 rows x 128 bf16
 constexpr uint32_t kBox = 16384;    // 128 rows x 64 bf16
 constexpr uint32_t kSlot = 16384;   // a half tile: 64 keys x 128 dims, 128 keys x 64 dims, or 64 rows of MqT
 constexpr uint32_t kTilesBytes = 2 * kQTile + kRing * kSlot + kQTile;  // Q x2, ring, output staging
-constexpr uint32_t kBarBytes = 256;
-constexpr uint32_t kStatsBytes = 2 * 2 * 128 * 4;  // (m, l) of both chains
+constexpr uint32_t kBarBytes = 512;
+constexpr uint32_t kStatsBytes = 3 * 128 * 4 + 2 * 2 * 128 * 4;  // (m, l_lo, l_hi); partial maxima [2 halves][2 tiles]
 constexpr int kSmem = 232448;
 static_assert(kTilesBytes + kBarBytes + kStatsBytes + 1024 <= uint32_t(kSmem), "shared memory layout too large");
 constexpr int kMaxContrib = 8;
 constexpr int kLaunchRegs = 128;
-constexpr int kCtlRegs = 56;
-constexpr int kSoftmaxRegs = 176;
-constexpr int kEpiRegs = 104;
+constexpr int kCtlRegs = 64;
+constexpr int kSoftmaxRegs = 160;
+constexpr int kEpiRegs = 128;
 static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs + 128 * kEpiRegs <= kThreads * kLaunchRegs,
               "register split too large");
 
@@ -78,13 +85,20 @@ enum {
   B_QE = 2,              // [2] Q slot free (commit, both CTAs)
   B_RF = 4,              // [kRing] ring slot loaded (rank 0: both CTAs' bytes)
   B_RE = 4 + kRing,      // [kRing] ring slot free (commit, both CTAs)
-  B_SF = 4 + 2 * kRing,  // [2] S of chain c in tensor memory (commit, both CTAs)
-  B_PF = B_SF + 2,       // [2] P of chain c written (rank 0: 4 warps x 2 CTAs)
-  B_SD = B_PF + 2,       // every MMA of the segment completed (commit, both CTAs)
-  B_ST = B_SD + 1,       // both chains' statistics in shared memory (local: 8 warps)
-  B_EO = B_ST + 1,       // epilogues done with O_0, O_1 and X (rank 0: 4 warps x 2 CTAs)
-  B_SC = B_EO + 1,       // statistics read by the epilogue (local: 4 warps)
-  B_DRAIN = B_SC + 1,
+  B_SF = 4 + 2 * kRing,  // [2] S(i) in S[i & 1] (commit, both CTAs)
+  B_SC = B_SF + 2,       // [2] S[i & 1] read by the softmax (rank 0: its 8 warps + 1 forwarded from rank 1)
+  B_PF = B_SC + 2,       // [2] P(i) in P[i & 1] (rank 0: its 8 warps + 1 forwarded from rank 1)
+  B_PD = B_PF + 2,       // [2] PV(i) completed: P[i & 1] free, O current (commit, both CTAs)
+  B_XQ = B_PD + 2,       // [2 tiles][4 quarters] partial row maxima exchanged (local: 2 warps)
+  B_SD = B_XQ + 8,       // every MMA of the segment completed (commit, both CTAs)
+  B_ST = B_SD + 1,       // the segment's statistics in shared memory (local: 8 warps)
+  B_STC = B_ST + 1,      // statistics read by the epilogue (local: 4 warps)
+  B_EO = B_STC + 1,      // epilogues done with O and X (rank 0: 4 warps x 2 CTAs)
+  B_EL = B_EO + 1,       // this CTA's epilogue done with O and X (local: 4 warps)
+  B_PQ = B_EL + 1,       // [4] a contributor's piece of this warp's rows in shared memory (local: bytes)
+  B_SCL = B_PQ + 4,      // [2] rank 1: its 8 softmax warps have read S[i & 1] (local)
+  B_PFL = B_SCL + 2,     // [2] rank 1: its 8 softmax warps have written P(i) (local)
+  B_DRAIN = B_PFL + 2,
   B_COUNT
 };
 static_assert(B_COUNT * 8 + 8 <= int(kBarBytes), "barrier area too small");
@@ -106,9 +120,13 @@ __device__ __forceinline__ bool next_seg(const AttnParams& p, unsigned& u, unsig
 }
 
 // Ring positions within a segment of n key tiles, in the order the issuer
-// consumes them: K_0, K_1, V_0, K_2, V_1, ..., K_{n-1}, V_{n-2}, V_{n-1}, MqT.
-__device__ __forceinline__ int pos_k(int i) { return i == 0 ? 0 : 2 * i - 1; }
-__device__ __forceinline__ int pos_v(int i, int n) { return i + 1 < n ? 2 * i + 2 : 2 * i + 1; }
+// consumes them (S two tiles ahead of PV): K_0, K_1, K_2, V_0, K_3, V_1, ...,
+// K_{n-1}, V_{n-3}, V_{n-2}, V_{n-1}, then MqT.
+__device__ __forceinline__ int pos_k(int i) { return i < 2 ? i : 2 * i - 2; }
+__device__ __forceinline__ int pos_v(int i, int n) {
+  if (n == 1) return 1;
+  return i + 2 < n ? 2 * i + 3 : 2 * n - 2 + (i - (n - 2));
+}
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   unsigned v;
@@ -169,16 +187,18 @@ __device__ __forceinline__ void producer(const AttnParams& p, uint64_t* bars, ui
       uint8_t* dst = sR + slot * kSlot;
       if (lead) mbar_expect_tx(&bars[B_RF + slot], 2 * kSlot);
       if (t < 2 * n) {
-        // position t holds K_i or V_i (see pos_k / pos_v)
+        // position t holds K_i or V_i (the inverse of pos_k / pos_v)
         int i, is_v;
-        if (t == 0) {
-          i = 0, is_v = 0;
-        } else if (t == 2 * n - 1) {
-          i = n - 1, is_v = 1;
-        } else if (t & 1) {
-          i = (t + 1) >> 1, is_v = 0;
+        if (n == 1) {
+          i = 0, is_v = t;
+        } else if (t < 2) {
+          i = t, is_v = 0;
+        } else if (t >= 2 * n - 2) {
+          i = t - n, is_v = 1;
+        } else if ((t & 1) == 0) {
+          i = t / 2 + 1, is_v = 0;
         } else {
-          i = (t - 2) >> 1, is_v = 1;
+          i = (t + 1) / 2 - 2, is_v = 1;
         }
         const int j = s.j0 + i;
         if (is_v) {  // all 128 keys, this CTA's 64 head dimensions
@@ -220,12 +240,14 @@ __device__ __forceinline__ void mma_pv_group(const uint32_t d, const uint32_t p_
   }
 }
 
-// One thread of rank 0.  Per segment (n key tiles, chain c = i & 1 of tile i):
-//   S(0);  for i: S(i+1) (into the buffer PV(i-1) has just read: tcgen05.mma
-//   operations of one thread run in issue order), then PV(i) once both CTAs'
-//   softmax has written P(i);  X = Q MqT^T into S_1 for blocks finished here.
-// Before a segment's S(1) and PV(0) the epilogues must be done with the
-// previous segment's X and O (B_EO).
+// One thread of rank 0.  Tiles are counted over the whole launch (g): S(g)
+// goes to S[g & 1] once the softmax of both CTAs has read S(g - 2) out of it
+// (B_SC); PV(g) reads P[g & 1] once both CTAs' softmax has written P(g)
+// (B_PF).  Per segment of n key tiles the order is
+//     S(0), S(1), S(2), PV(0), S(3), PV(1), ..., S(n-1), PV(n-3), PV(n-2), PV(n-1)
+// then, for blocks finished here, X = Q MqT^T over [256, 384) (both P
+// buffers are consumed by then).  A segment's first PV, which overwrites O,
+// waits until the epilogues have read the previous segment's O and X (B_EO).
 __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, const uint32_t tmem,
                                            const uint32_t q_addr, const uint32_t r_addr, const unsigned u_begin,
                                            const unsigned u_end, const WaitCtl& w) {
@@ -237,7 +259,7 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, 
   const uint32_t dq0 = uint32_t(dq64);
   const uint32_t dk0 = uint32_t(smem_desc_sw128(r_addr, 16, 1024));     // K-major ring slot
   const uint32_t dv0 = uint32_t(smem_desc_sw128(r_addr, kBox, 1024));   // MN-major ring slot
-  uint32_t ring = 0, k = 0, g[2] = {0, 0};
+  uint32_t ring = 0, k = 0, gs = 0, gp = 0;
   unsigned u = u_begin;
   Seg s;
   while (next_seg(p, u, u_end, s)) {
@@ -246,39 +268,41 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, 
     const uint32_t dq = dq0 + qs * kQ16;
     if (!mbar_wait(&bars[B_QF + qs], (k >> 1) & 1, w)) return;
     const uint32_t r0 = ring;
-    if (!mbar_wait(&bars[B_RF + r0 % kRing], (r0 / kRing) & 1, w)) return;
-    mma_s_group(tmem, dq, dk0 + (r0 % kRing) * kSlot16, hi, id_s);
-    mma_commit_pair(&bars[B_SF + 0]);
-    mma_commit_pair(&bars[B_RE + r0 % kRing]);
-    for (int i = 0; i < n; ++i) {
-      const int c = i & 1;
-      if (i + 1 < n) {
-        const uint32_t rk = r0 + pos_k(i + 1);
+    for (int i = 0; i < n + 2; ++i) {
+      if (i < n) {  // S(i)
+        const uint32_t rk = r0 + pos_k(i), buf = gs & 1;
         if (!mbar_wait(&bars[B_RF + rk % kRing], (rk / kRing) & 1, w)) return;
-        if (i == 0 && k > 0) {  // S_1 may hold the previous segment's X
-          if (!mbar_wait(&bars[B_EO], (k - 1) & 1, w)) return;
+        if (gs >= 2) {
+          if (!mbar_wait(&bars[B_SC + buf], ((gs - 2) >> 1) & 1, w)) return;
           tc_fence_after();
         }
-        mma_s_group(tmem + ((i + 1) & 1) * 128, dq, dk0 + (rk % kRing) * kSlot16, hi, id_s);
-        mma_commit_pair(&bars[B_SF + ((i + 1) & 1)]);
+        mma_s_group(tmem + buf * 128, dq, dk0 + (rk % kRing) * kSlot16, hi, id_s);
+        mma_commit_pair(&bars[B_SF + buf]);
         mma_commit_pair(&bars[B_RE + rk % kRing]);
+        ++gs;
       }
-      const uint32_t rv = r0 + pos_v(i, n);
-      if (!mbar_wait(&bars[B_RF + rv % kRing], (rv / kRing) & 1, w)) return;
-      if (!mbar_wait(&bars[B_PF + c], g[c] & 1, w)) return;
-      ++g[c];
-      if (i == 0 && n == 1 && k > 0 && !mbar_wait(&bars[B_EO], (k - 1) & 1, w)) return;
-      tc_fence_after();
-      const int valid = min(128, p.kv_len - (s.j0 + i) * 128);
-      mma_pv_group(tmem + 256 + c * 128, tmem + c * 128, dv0 + (rv % kRing) * kSlot16, hi, id_o, (valid + 15) >> 4,
-                   i >= 2);
-      mma_commit_pair(&bars[B_RE + rv % kRing]);
+      if (i >= 2 || (n == 1 && i == 1)) {  // PV(j)
+        const int j = n == 1 ? 0 : i - 2;
+        if (j >= n) continue;
+        const uint32_t rv = r0 + pos_v(j, n), buf = gp & 1;
+        if (!mbar_wait(&bars[B_RF + rv % kRing], (rv / kRing) & 1, w)) return;
+        if (!mbar_wait(&bars[B_PF + buf], (gp >> 1) & 1, w)) return;
+        if (j == 0 && k > 0 && !mbar_wait(&bars[B_EO], (k - 1) & 1, w)) return;
+        tc_fence_after();
+        const int valid = min(128, p.kv_len - (s.j0 + j) * 128);
+        mma_pv_group(tmem + 384, tmem + 256 + buf * 64, dv0 + (rv % kRing) * kSlot16, hi, id_o, (valid + 15) >> 4,
+                     j > 0);
+        mma_commit_pair(&bars[B_PD + buf]);
+        mma_commit_pair(&bars[B_RE + rv % kRing]);
+        ++gp;
+        if (n == 1) break;
+      }
     }
     ring = r0 + 2 * n;
     if (s.j0 == 0 && p.has_inter) {  // X = Q MqT^T for the rows this pair finishes
       const uint32_t rm = ring;
       if (!mbar_wait(&bars[B_RF + rm % kRing], (rm / kRing) & 1, w)) return;
-      mma_s_group(tmem + 128, dq, dk0 + (rm % kRing) * kSlot16, hi, id_s);
+      mma_s_group(tmem + 256, dq, dk0 + (rm % kRing) * kSlot16, hi, id_s);
       mma_commit_pair(&bars[B_RE + rm % kRing]);
       ++ring;
     }
@@ -289,21 +313,26 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, 
 }
 
 // ------------------------------------------------------------------ softmax
-// One warpgroup per chain, one query row per thread.  Per key tile of the
-// chain: the 128-column row of S from tensor memory; its maximum; lazy
-// rescaling (the running max m moves only when the tile's max exceeds it by
-// more than 8, a factor 256, and then O_c is rescaled in tensor memory --
-// stable there, since the commit that announced S tracks the chain's previous
-// PV); P = 2^(S * scale * log2(e) - m) packed to bf16 pairs over S's first 64
-// columns; the running row sum l.  At the end of a segment (m, l) go to shared
-// memory for the epilogue.
-__device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars, float* stats, const uint32_t tmem,
-                                             const int c, const int quarter, const int lane, const unsigned u_begin,
-                                             const unsigned u_end, const WaitCtl& w) {
+// Two warpgroups share every tile: half h takes keys 64h .. 64h + 63 of the
+// 128 rows (one row per thread).  Per tile g: its 64 columns of S from S[g & 1]
+// (then S[g & 1] is handed back to the issuer); the half's row maximum,
+// exchanged with the other half through shared memory; lazy rescaling (the
+// running max m moves only when the tile's max exceeds it by more than 8, a
+// factor 256; then O is rescaled in tensor memory, each half its 64 columns,
+// once the previous PV has completed); P = 2^(S * scale * log2(e) - m) packed
+// to bf16 pairs into P[g & 1] (free once PV(g - 2) has completed); the half's
+// running row sum l.  Both halves take the same decisions from the same row
+// maxima.  At the end of a segment (m, l) go to shared memory for the epilogue.
+__device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars, float* stats, float* xmax,
+                                             const uint32_t tmem, const int rank, const int half, const int quarter,
+                                             const int lane, const unsigned u_begin, const unsigned u_end,
+                                             const WaitCtl& w) {
   const int row = quarter * 32 + lane;
   const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-  const uint32_t tS = tmem + c * 128, tO = tmem + 256 + c * 128;
-  const uint32_t pf_leader = cluster_map(smem_u32(&bars[B_PF + c]), 0);
+  // rank 0 arrives on its own barriers; rank 1 on local ones that its
+  // forwarder relays (a cluster-scope arrive costs each warp ~10^3 cycles)
+  const int sc_bar = rank == 0 ? B_SC : B_SCL, pf_bar = rank == 0 ? B_PF : B_PFL;
+  const uint32_t tO = tmem + 384 + half * 64;
   const float sl2 = p.scale_log2;
   uint32_t g = 0, k = 0;
   unsigned u = u_begin;
@@ -311,18 +340,21 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars
   while (next_seg(p, u, u_end, s)) {
     const int n = s.j1 - s.j0;
     float m = -INFINITY, l = 0.f;
-    for (int i = c; i < n; i += 2) {
-      if (!warp_wait(&bars[B_SF + c], g & 1, w)) return;
-      ++g;
+    for (int i = 0; i < n; ++i, ++g) {
+      const uint32_t buf = g & 1, ph = (g >> 1) & 1;
+      if (!warp_wait(&bars[B_SF + buf], ph, w)) return;
       tc_fence_after();
-      const int valid = min(128, p.kv_len - (s.j0 + i) * 128);
-      uint32_t r[128];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tS + lane_off + q * 32, slice32(r, q));
+      const int valid = min(128, p.kv_len - (s.j0 + i) * 128) - half * 64;  // valid columns of this half
+      uint32_t r[64];
+      tmem_ld32(tmem + buf * 128 + half * 64 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(tmem + buf * 128 + half * 64 + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_wait_ld();
-      if (valid < 128) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[sc_bar + buf]);  // S[buf] may take the next S
+      if (valid < 64) {
 #pragma unroll
-        for (int x = 0; x < 128; ++x)
+        for (int x = 0; x < 64; ++x)
           if (x >= valid) r[x] = __float_as_uint(-INFINITY);
       }
       float m4[4];
@@ -330,15 +362,20 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars
       for (int q = 0; q < 4; ++q)
         m4[q] = fmax3(__uint_as_float(r[q]), __uint_as_float(r[4 + q]), __uint_as_float(r[8 + q]));
 #pragma unroll
-      for (int x = 12; x < 124; x += 8)
+      for (int x = 12; x < 60; x += 8)
 #pragma unroll
         for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], __uint_as_float(r[x + q]), __uint_as_float(r[x + 4 + q]));
 #pragma unroll
-      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], __uint_as_float(r[124 + q]));
-      const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl2;
+      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], __uint_as_float(r[60 + q]));
+      const float pm = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+      xmax[(half * 2 + buf) * 128 + row] = pm;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_XQ + buf * 4 + quarter]);
+      if (!warp_wait(&bars[B_XQ + buf * 4 + quarter], ph, w)) return;
+      const float mx = fmaxf(pm, xmax[((1 - half) * 2 + buf) * 128 + row]) * sl2;
       float f = 1.f;
       bool any_rescale = false;
-      if (i == c) {
+      if (i == 0) {
         m = mx;
       } else {
         const bool need = mx > m + 8.f;
@@ -350,26 +387,24 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars
       }
       const float2 sc = make_float2(sl2, sl2), nm = make_float2(-m, -m);
       float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      uint32_t pk[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const float2 y = __ffma2_rn(
-              make_float2(__uint_as_float(r[q * 32 + 2 * x]), __uint_as_float(r[q * 32 + 2 * x + 1])), sc, nm);
-          const float2 e = make_float2(fast_exp2(y.x), fast_exp2(y.y));
-          s2[x & 3] = __fadd2_rn(s2[x & 3], e);
-          pk[x] = pack_bf16x2(e.x, e.y);
-        }
-        tmem_st16(tS + lane_off + q * 16, pk);
+      for (int x = 0; x < 32; ++x) {
+        const float2 y =
+            __ffma2_rn(make_float2(__uint_as_float(r[2 * x]), __uint_as_float(r[2 * x + 1])), sc, nm);
+        const float2 e = make_float2(fast_exp2(y.x), fast_exp2(y.y));
+        s2[x & 3] = __fadd2_rn(s2[x & 3], e);
+        pk[x] = pack_bf16x2(e.x, e.y);
       }
-      const float2 s01 = __fadd2_rn(s2[0], s2[1]), s23 = __fadd2_rn(s2[2], s2[3]);
-      const float2 sa = __fadd2_rn(s01, s23);
-      l = fmaf(l, f, sa.x + sa.y);
-      tmem_wait_st();
-      if (any_rescale) {  // rare: O_c is rescaled before P is announced, so the PV sees a consistent O_c
+      // P[buf] is free once PV(g - 2) has completed; at a segment's first tile
+      // the epilogue must also be done with X, which overlays both P buffers
+      if (g >= 2 && !warp_wait(&bars[B_PD + buf], ((g - 2) >> 1) & 1, w)) return;
+      if (i == 0 && k > 0 && !warp_wait(&bars[B_EL], (k - 1) & 1, w)) return;
+      if (any_rescale) {  // rare: O is rescaled (after PV(g - 1)) before P is announced
+        if (!warp_wait(&bars[B_PD + (buf ^ 1)], ((g - 1) >> 1) & 1, w)) return;
+        tc_fence_after();
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           uint32_t o[32];
           tmem_ld32(tO + lane_off + q * 32, o);
           tmem_wait_ld();
@@ -377,42 +412,75 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars
           for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
           tmem_st32(tO + lane_off + q * 32, o);
         }
-        tmem_wait_st();
       }
+      tc_fence_after();
+      tmem_st16(tmem + 256 + buf * 64 + half * 32 + lane_off, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+      tmem_st16(tmem + 256 + buf * 64 + half * 32 + 16 + lane_off, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+      const float2 s01 = __fadd2_rn(s2[0], s2[1]), s23 = __fadd2_rn(s2[2], s2[3]);
+      const float2 sa = __fadd2_rn(s01, s23);
+      l = fmaf(l, f, sa.x + sa.y);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(pf_leader);
+      if (lane == 0) mbar_arrive(&bars[pf_bar + buf]);
     }
     // the epilogue has read the previous segment's statistics
-    if (k > 0 && !warp_wait(&bars[B_SC], (k - 1) & 1, w)) return;
-    stats[(c * 2 + 0) * 128 + row] = m;
-    stats[(c * 2 + 1) * 128 + row] = l;
+    if (k > 0 && !warp_wait(&bars[B_STC], (k - 1) & 1, w)) return;
+    if (half == 0) stats[row] = m;
+    stats[(1 + half) * 128 + row] = l;
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[B_ST]);
     ++k;
   }
 }
 
+// ------------------------------------------------------------------ forwarder
+// One thread of rank 1: relays its softmax warps' per-tile signals (S[i & 1]
+// read, P(i) written) to rank 0's barriers with one cluster-scope arrive each,
+// in the order they occur, so that no softmax warp pays for a remote arrive.
+__device__ __forceinline__ void forwarder(const AttnParams& p, uint64_t* bars, const unsigned u_begin,
+                                          const unsigned u_end, const WaitCtl& w) {
+  const uint32_t sc0 = cluster_map(smem_u32(&bars[B_SC]), 0), pf0 = cluster_map(smem_u32(&bars[B_PF]), 0);
+  uint32_t g = 0;
+  unsigned u = u_begin;
+  Seg s;
+  while (next_seg(p, u, u_end, s)) {
+    for (int i = 0; i < s.j1 - s.j0; ++i, ++g) {
+      const uint32_t buf = g & 1, ph = (g >> 1) & 1;
+      if (!mbar_wait(&bars[B_SCL + buf], ph, w)) return;
+      mbar_arrive_cluster(sc0 + buf * 8);
+      if (!mbar_wait(&bars[B_PFL + buf], ph, w)) return;
+      mbar_arrive_cluster(pf0 + buf * 8);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ epilogue
-// 16-byte chunk i (four floats, columns 4i..4i+3) of row r of an fp32 partial
-// slot lies at float index (i * 128 + r) * 4, so a warp's chunk is one
-// contiguous 512-byte span; (m, l) follow at kPartStats.
+// A contributor's piece: O / l rounded to bf16, rows in four 8 KB quarters
+// (one per epilogue warp); within quarter q, 16-byte chunk c (columns
+// 8c..8c+7) of row 32q + r lies at byte q * 8192 + (c * 32 + r) * 16, so a
+// warp's chunk is one contiguous 512-byte span and a warp's quarter is one
+// 8 KB block that the finishing CTA copies into shared memory whole.  (m, l)
+// follow in fp32 at float kPartStats.
 constexpr int kPartStats = 128 * 128;
+constexpr uint32_t kPartQuarter = 8192;
 
 // One warpgroup, one query row per thread.  At the end of a segment (its MMAs
-// done, both chains' statistics in shared memory):
-//  * own piece: m = max(m_0, m_1), l = l_0 a_0 + l_1 a_1, O = (O_0 a_0 + O_1 a_1) / l
-//    with a_c = 2^(m_c - m);
+// done, the statistics in shared memory):
+//  * own piece: m, l = l_lo + l_hi, O / l;
 //  * a segment that does not start at key tile 0 (a contributor) stores its
-//    piece (O normalised, m, l) in fp32 and raises this warp's ready flag;
-//  * a segment holding a whole block writes O (+ X) through per-warp staging
-//    boxes and TMA tile stores;
+//    piece (O / l in bf16, m, l) and raises this warp's ready flag;
+//  * a segment holding a whole block writes O / l (+ X) through per-warp
+//    staging boxes and TMA tile stores;
 //  * a segment that starts a block continued by the next pairs (always the
-//    pair's last segment) also waits for those pairs' flags and merges their
-//    pieces in key order before adding X.
-// Tensor memory is handed back (B_EO on rank 0) as soon as it has been read.
+//    pair's last segment) merges their pieces in key order before adding X.
+//    Those pieces are ready long before the segment's MMAs end, so while they
+//    run this warp acquires the flags, reads the pieces' (m, l) and copies the
+//    first piece's quarter into the Q slot the segment does not use.
+// Tensor memory is handed back (B_EO on rank 0 for the issuer, B_EL locally
+// for the softmax) as soon as O and X have been read.
 __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bars, const float* stats, uint8_t* stage,
-                                              const CUtensorMap* tm_o, const uint32_t tmem, const int cta,
+                                              uint8_t* sQ, const CUtensorMap* tm_o, const uint32_t tmem, const int cta,
                                               const int rank, const int quarter, const int lane,
                                               const unsigned u_begin, const unsigned u_end, volatile int* abort_flag,
                                               const WaitCtl& w) {
@@ -428,42 +496,26 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
   unsigned u = u_begin;
   Seg s;
   while (next_seg(p, u, u_end, s)) {
-    const int n = s.j1 - s.j0;
     const int b = s.bh / p.heads, h = s.bh % p.heads;
     const bool writer = s.j0 == 0, full = writer && s.j1 == p.nkv;
     const int qt = 2 * s.blk + rank;
     const bool row_ok = qt * 128 + row < p.q_len;
     const bool warp_on = qt * 128 + quarter * 32 < p.q_len;  // warp-uniform
+    const bool with_x = writer && use_inter;
     int n_contrib = 0;
     if (writer && !full && (n_contrib = contributors(p, pair, s)) < 0) {
       record_error(p.err, kDevBadShape);  // the host partition rules this out
       *abort_flag = 1;
       return false;
     }
-    if (!warp_wait(&bars[B_SD], k & 1, w)) return false;
-    if (!warp_wait(&bars[B_ST], k & 1, w)) return false;
-    tc_fence_after();
-    const float m0 = stats[0 * 128 + row], l0 = stats[1 * 128 + row];
-    const float m1 = n > 1 ? stats[2 * 128 + row] : -INFINITY, l1 = n > 1 ? stats[3 * 128 + row] : 0.f;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars[B_SC]);
-    const float M = fmaxf(m0, m1);
-    const float e0 = fast_exp2(m0 - M), e1 = n > 1 ? fast_exp2(m1 - M) : 0.f;
-    const float L = l0 * e0 + l1 * e1;
-    // weights of this pair's own piece and of the contributors' pieces
-    float a0 = 0.f, a1 = 0.f, wk[kMaxContrib];
+    uint8_t* piece = sQ + ((k + 1) & 1) * kQTile + quarter * kPartQuarter;
+    float mk[kMaxContrib], lk[kMaxContrib];
 #pragma unroll
-    for (int q = 0; q < kMaxContrib; ++q) wk[q] = 0.f;
-    if (!writer) {
-      const float inv = 1.f / L;
-      a0 = e0 * inv;
-      a1 = e1 * inv;
-    } else if (n_contrib == 0) {
-      const float inv = row_ok ? 1.f / L : 0.f;
-      a0 = e0 * inv;
-      a1 = e1 * inv;
-    } else {
-      // the contributors' flags (one per warp of their epilogue), then their statistics
+    for (int q = 0; q < kMaxContrib; ++q) {
+      mk[q] = -INFINITY;
+      lk[q] = 0.f;
+    }
+    if (n_contrib > 0) {
       if (lane == 0) {
         for (int q = 0; q < n_contrib && !*abort_flag; ++q) {
           const unsigned* f = p.ready + (size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter;
@@ -476,24 +528,44 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
             }
           }
         }
+        // the other Q slot is free once the previous segment's MMAs are done
+        if (!*abort_flag && (k == 0 || mbar_wait(&bars[B_QE + ((k + 1) & 1)], ((k - 1) >> 1) & 1, w))) {
+          fence_async_global();
+          mbar_expect_tx(&bars[B_PQ + quarter], kPartQuarter);
+          bulk_load(piece, reinterpret_cast<const uint8_t*>(slot_of(p, 2 * (pair + 1) + rank)) + quarter * kPartQuarter,
+                    kPartQuarter, &bars[B_PQ + quarter]);
+        }
       }
       __syncwarp();
       if (*abort_flag) return false;
       for (int q = 0; q < n_contrib; ++q)  // every lane acquires what the contributors released
         (void)ld_acquire(p.ready + (size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter);
-      float mk[kMaxContrib], lk[kMaxContrib];
-      float Mx = M;
 #pragma unroll
       for (int q = 0; q < kMaxContrib; ++q) {
-        mk[q] = -INFINITY;
-        lk[q] = 0.f;
         if (q < n_contrib) {
           const float* st = slot_of(p, 2 * (pair + 1 + q) + rank) + kPartStats;
           mk[q] = st[row];
           lk[q] = st[128 + row];
         }
-        Mx = fmaxf(Mx, mk[q]);
       }
+    }
+    if (!warp_wait(&bars[B_SD], k & 1, w)) return false;
+    if (!warp_wait(&bars[B_ST], k & 1, w)) return false;
+    tc_fence_after();
+    const float M = stats[row], L = stats[128 + row] + stats[256 + row];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[B_STC]);
+    float a0 = 0.f, wk[kMaxContrib];
+#pragma unroll
+    for (int q = 0; q < kMaxContrib; ++q) wk[q] = 0.f;
+    if (!writer) {
+      a0 = 1.f / L;
+    } else if (n_contrib == 0) {
+      a0 = row_ok ? 1.f / L : 0.f;
+    } else {
+      float Mx = M;
+#pragma unroll
+      for (int q = 0; q < kMaxContrib; ++q) Mx = fmaxf(Mx, mk[q]);
       const float es = fast_exp2(M - Mx);
       float Lx = L * es;
 #pragma unroll
@@ -502,33 +574,35 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
         Lx += wk[q];
       }
       const float inv = row_ok ? 1.f / Lx : 0.f;
-      a0 = e0 * es * inv;
-      a1 = e1 * es * inv;
+      a0 = es * inv;
 #pragma unroll
       for (int q = 0; q < kMaxContrib; ++q) wk[q] *= inv;
     }
-    if (!use_intra) a0 = a1 = 0.f;
-    const float2 A0 = make_float2(a0, a0), A1 = make_float2(a1, a1);
+    if (!use_intra) a0 = 0.f;
+    const float2 A0 = make_float2(a0, a0);
     if (!writer) {  // ------------------------------------------------------ contributor
       float* slot = slot_of(p, cta);
-      float4* d4 = reinterpret_cast<float4*>(slot) + row;
+      uint4* d4 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(slot) + quarter * kPartQuarter) + lane;
 #pragma unroll 1
-      for (int q = 0; q < 8; ++q) {  // 16 columns at a time
-        uint32_t o0[16], o1[16];
-        tmem_ld16(tmem + 256 + lane_off + q * 16, o0);
-        if (n > 1) tmem_ld16(tmem + 384 + lane_off + q * 16, o1);
+      for (int q = 0; q < 4; ++q) {  // 32 columns at a time
+        uint32_t o0[32];
+        tmem_ld32(tmem + 384 + lane_off + q * 32, o0);
         tmem_wait_ld();
-        float2* v = reinterpret_cast<float2*>(o0);
-        const float2* v1 = reinterpret_cast<const float2*>(o1);
+        const float2* v = reinterpret_cast<const float2*>(o0);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) v[x] = n > 1 ? __ffma2_rn(v1[x], A1, __fmul2_rn(v[x], A0)) : __fmul2_rn(v[x], A0);
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-          d4[(4 * q + x) * 128] = make_float4(v[2 * x].x, v[2 * x].y, v[2 * x + 1].x, v[2 * x + 1].y);
+        for (int x = 0; x < 4; ++x) {
+          const float2 v0 = __fmul2_rn(v[4 * x], A0), v1 = __fmul2_rn(v[4 * x + 1], A0);
+          const float2 v2 = __fmul2_rn(v[4 * x + 2], A0), v3 = __fmul2_rn(v[4 * x + 3], A0);
+          d4[(4 * q + x) * 32] = make_uint4(pack_bf16x2(v0.x, v0.y), pack_bf16x2(v1.x, v1.y), pack_bf16x2(v2.x, v2.y),
+                                            pack_bf16x2(v3.x, v3.y));
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(eo_leader);
+      if (lane == 0) {
+        mbar_arrive_cluster(eo_leader);
+        mbar_arrive(&bars[B_EL]);
+      }
       slot[kPartStats + row] = M;
       slot[kPartStats + 128 + row] = L;
       __threadfence();
@@ -540,53 +614,65 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
     // ------------------------------------------------------------------ writer
     if (lane == 0 && staged) bulk_wait_read0();  // this warp's previous tile store has read its boxes
     __syncwarp();
+    if (n_contrib > 0 && !warp_wait(&bars[B_PQ + quarter], 0, w)) return false;  // once per launch
 #pragma unroll 1
-    for (int q = 0; q < 8; ++q) {  // 16 columns at a time
-      uint32_t o0[16], o1[16], rx[16];
-      tmem_ld16(tmem + 256 + lane_off + q * 16, o0);
-      if (n > 1) tmem_ld16(tmem + 384 + lane_off + q * 16, o1);
-      if (use_inter) tmem_ld16(tmem + 128 + lane_off + q * 16, rx);
+    for (int q = 0; q < 4; ++q) {  // 32 columns at a time
+      uint32_t o0[32], rx[32];
+      tmem_ld32(tmem + 384 + lane_off + q * 32, o0);
+      if (with_x) tmem_ld32(tmem + 256 + lane_off + q * 32, rx);
       tmem_wait_ld();
+      if (q == 3) {  // O and X are read: hand tensor memory back
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(eo_leader);
+          mbar_arrive(&bars[B_EL]);
+        }
+      }
       float2* v = reinterpret_cast<float2*>(o0);
-      const float2* v1 = reinterpret_cast<const float2*>(o1);
 #pragma unroll
-      for (int x = 0; x < 8; ++x) v[x] = n > 1 ? __ffma2_rn(v1[x], A1, __fmul2_rn(v[x], A0)) : __fmul2_rn(v[x], A0);
+      for (int x = 0; x < 16; ++x) v[x] = __fmul2_rn(v[x], A0);
       if (n_contrib > 0 && use_intra) {
 #pragma unroll 1
         for (int c2 = 0; c2 < n_contrib; ++c2) {
-          const float4* src = reinterpret_cast<const float4*>(slot_of(p, 2 * (pair + 1 + c2) + rank)) + row;
+          // the first piece from shared memory, any others from global memory
+          const uint4* src =
+              c2 == 0 ? reinterpret_cast<const uint4*>(piece) + lane
+                      : reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(slot_of(p, 2 * (pair + 1 + c2) + rank)) +
+                                                       quarter * kPartQuarter) + lane;
           const float2 W = make_float2(wk[c2], wk[c2]);
+          uint4 t4[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) t4[x] = src[(4 * q + x) * 32];
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
-            const float4 t4 = src[(4 * q + x) * 128];
-            v[2 * x] = __ffma2_rn(make_float2(t4.x, t4.y), W, v[2 * x]);
-            v[2 * x + 1] = __ffma2_rn(make_float2(t4.z, t4.w), W, v[2 * x + 1]);
+            const uint32_t w4[4] = {t4[x].x, t4[x].y, t4[x].z, t4[x].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              v[4 * x + e] = __ffma2_rn(make_float2(__uint_as_float(w4[e] << 16), __uint_as_float(w4[e] & 0xFFFF0000u)), W,
+                                        v[4 * x + e]);
           }
         }
       }
-      if (use_inter) {
+      if (with_x) {
         const float2* x2 = reinterpret_cast<const float2*>(rx);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) v[x] = __fadd2_rn(v[x], x2[x]);
+        for (int x = 0; x < 16; ++x) v[x] = __fadd2_rn(v[x], x2[x]);
       }
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const int ch = 2 * q + x;  // 16-byte chunk of the row: box ch / 8, chunk ch % 8 swizzled by row
+      for (int x = 0; x < 4; ++x) {
+        const int ch = 4 * q + x;  // 16-byte chunk of the row: box ch / 8, chunk ch % 8 swizzled by row
         *reinterpret_cast<uint4*>(wst + (ch >> 3) * 4096 + lane * 128 + (((ch & 7) ^ (lane & 7)) << 4)) =
             make_uint4(pack_bf16x2(v[4 * x].x, v[4 * x].y), pack_bf16x2(v[4 * x + 1].x, v[4 * x + 1].y),
                        pack_bf16x2(v[4 * x + 2].x, v[4 * x + 2].y), pack_bf16x2(v[4 * x + 3].x, v[4 * x + 3].y));
       }
     }
-    tc_fence_before();
     fence_async_smem();
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive_cluster(eo_leader);
-      if (warp_on) {
-        tma_store_3d(tm_o, wst, h * 128, qt * 128 + quarter * 32, b);
-        tma_store_3d(tm_o, wst + 4096, h * 128 + 64, qt * 128 + quarter * 32, b);
-        bulk_commit();
-      }
+    if (lane == 0 && warp_on) {
+      tma_store_3d(tm_o, wst, h * 128, qt * 128 + quarter * 32, b);
+      tma_store_3d(tm_o, wst + 4096, h * 128 + 64, qt * 128 + quarter * 32, b);
+      bulk_commit();
     }
     staged = true;
     if (n_contrib > 0 && lane == 0) {  // the pieces are read: their flags go back to zero for the next launch
@@ -611,7 +697,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTilesBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* stats = reinterpret_cast<float*>(smem + kTilesBytes + kBarBytes);  // [2 chains][m, l][128]
+  float* stats = reinterpret_cast<float*>(smem + kTilesBytes + kBarBytes);  // m[128], l_lo[128], l_hi[128]
+  float* xmax = stats + 3 * 128;                                            // [2 halves][2 tiles][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
@@ -625,9 +712,12 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t count = 1;
-      if (i == B_PF || i == B_PF + 1 || i == B_EO) count = 8;  // 4 warps x 2 CTAs (rank 0's copies)
-      if (i == B_ST) count = 8;                                // 4 warps x 2 chains (local)
-      if (i == B_SC) count = 4;                                // the epilogue's 4 warps (local)
+      if (i >= B_SC && i < B_PF + 2) count = 9;   // rank 0's 8 softmax warps + rank 1's forwarder
+      if (i >= B_SCL && i < B_PFL + 2) count = 8;  // rank 1's 8 softmax warps
+      if (i >= B_XQ && i < B_XQ + 8) count = 2;   // the two halves' warps of one quarter
+      if (i == B_ST) count = 8;                    // 8 softmax warps
+      if (i == B_STC || i == B_EL) count = 4;      // the epilogue's 4 warps
+      if (i == B_EO) count = 8;                    // 4 epilogue warps x 2 CTAs (rank 0's copy)
       mbar_init(&bars[i], count);
     }
     *abort_flag = fits ? 0 : 1;
@@ -652,14 +742,16 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         producer(p, bars, sQ, sR, &tm_q, &tm_k, &tm_v, &tm_mq, rank, u_begin, u_end, w);
       } else if (warp == 1 && lane == 0 && rank == 0) {
         mma_issuer(p, bars, tmem, smem_u32(sQ), smem_u32(sR), u_begin, u_end, w);
+      } else if (warp == 3 && lane == 0 && rank == 1) {
+        forwarder(p, bars, u_begin, u_end, w);
       }
       __syncwarp();
     } else if (wg == 3) {
       regs_dec<kEpiRegs>();
-      epilogue_role(p, bars, stats, sStage, &tm_o, tmem, cta, rank, warp & 3, lane, u_begin, u_end, abort_flag, w);
+      epilogue_role(p, bars, stats, sStage, sQ, &tm_o, tmem, cta, rank, warp & 3, lane, u_begin, u_end, abort_flag, w);
     } else {
       regs_inc<kSoftmaxRegs>();
-      softmax_role(p, bars, stats, tmem, wg - 1, warp & 3, lane, u_begin, u_end, w);
+      softmax_role(p, bars, stats, xmax, tmem, rank, wg - 1, warp & 3, lane, u_begin, u_end, w);
     }
   }
 

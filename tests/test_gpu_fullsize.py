@@ -185,3 +185,45 @@ def test_every_query_row_of_a_full_size_pass(index):
         e = max_rel(g_out[key], r)
         assert e <= OUT_TOL, (key, e)
     assert frob_rel(g_S[-1], r_S[-1]) <= STATE_TOL
+
+
+def _split_block_rows(cfg, pairs=74):
+    """Query rows (of every head) whose 256-row block the pair kernel's stream-K
+    partition splits between two or more CTA pairs, for `pairs` resident pairs
+    (74 on a 148-SM B200): every block whose key range does not lie inside one
+    pair's contiguous range of (block, key tile) units."""
+    n_qt = (cfg.tokens + 127) // 128
+    n_blk, nkv = (n_qt + 1) // 2, (cfg.tokens + 127) // 128
+    units = cfg.batch * cfg.heads * n_blk * nkv
+    bounds = [units * c // pairs for c in range(pairs + 1)]
+    split = set()
+    for c in range(1, pairs):
+        u = bounds[c]
+        if u % nkv:  # a pair boundary inside a block
+            bh, blk = divmod(u // nkv, n_blk)
+            split.add((bh, blk))
+    return split, n_blk
+
+
+def test_split_blocks_err_like_whole_blocks():
+    """Pieces of split blocks travel between CTA pairs as O / l rounded to bf16
+    (one extra rounding step that whole blocks do not take).  Their rows must
+    err like the rows of whole blocks: at most twice the largest error of the
+    whole blocks' rows, plus one bf16 step of the output scale."""
+    cfg = W.CONFIGS[1]
+    wl = W.Workload(cfg)
+    keep = lambda n, p: n == 1 and p == 0
+    g_out, _ = run_gpu_stream(cfg, wl, frames=2, keep=keep)
+    r_out, _ = run_oracle_stream(cfg, wl, frames=2, keep=keep)
+    g, r = g_out[(1, 0)], r_out[(1, 0)]          # [B, L, H, d]
+    scale = np.abs(r).max()
+    err = np.abs(g - r).max(axis=3) / scale       # [B, L, H]
+    split, n_blk = _split_block_rows(cfg)
+    assert split, "the 1560-token frame has split blocks at 74 pairs"
+    mask = np.zeros(err.shape, dtype=bool)
+    for bh, blk in split:
+        b, h = divmod(bh, cfg.heads)
+        mask[b, blk * 256:(blk + 1) * 256, h] = True
+    e_split, e_whole = err[mask].max(), err[~mask].max()
+    assert e_split <= OUT_TOL and e_whole <= OUT_TOL
+    assert e_split <= 2 * e_whole + 2.0 ** -8, (e_split, e_whole)
