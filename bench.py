@@ -727,13 +727,13 @@ def cpu_oracle_rate(cfg: W.Config, budget_s: float = 12.0, sample_note=True):
                       f"numpy float64, {dt:.1f} s"}
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_bf16_kernel
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_pair_kernel
 # launch on the single-hybrid-layer-bf16 workload, from one ncu capture of
 # `bench.py --profile-small --no-graphs`; reported only while the kernel sources
-# hash to the value the capture was taken on.
-ATTN_TRAFFIC = {"bytes": 15408128 + 512, "sources_sha256": "1338d0ad68e85518eab263f946646a789e09e516479508343aa1599b31758f38",
-                "capture": "profiles/attn_bf16_kernel_single-hybrid-layer-bf16.md"}
-ATTN_SOURCES = ("hybrid_linear_attention_arl2_b200/csrc/attn_bf16.cu",
+# hash to the value the capture was taken on (None: not captured yet).
+ATTN_TRAFFIC = {"bytes": None, "sources_sha256": None,
+                "capture": "profiles/attn_pair_kernel_single-hybrid-layer-bf16.md"}
+ATTN_SOURCES = ("hybrid_linear_attention_arl2_b200/csrc/attn_pair.cu",
                 "hybrid_linear_attention_arl2_b200/csrc/sm100.cuh",
                 "hybrid_linear_attention_arl2_b200/csrc/params.h")
 
@@ -872,7 +872,7 @@ def main():
                 "pct_bf16_peak": {"value": 100.0 * res["stack_tflops"] / peak_burst,
                                   "basis": f"burst bf16 {src}",
                                   "sustained_basis": 100.0 * res["stack_tflops"] / peak_sus},
-                "roofline": {"bound": "tensor", "kernel": "attn_bf16_kernel (KV-cache softmax layers)",
+                "roofline": {"bound": "tensor", "kernel": "attn_pair_kernel (KV-cache softmax layers)",
                              "achieved": res["kv_tflops"], "peak": peak_burst, "unit": "TFLOP/s",
                              "frac": res["kv_tflops"] / peak_burst, "traffic": None,
                              "peak_basis": f"bf16_tflops (burst) {src}",
@@ -896,7 +896,7 @@ def main():
         "tokens_per_s": res["value"] * cfg.tokens * cfg.batch,
         "pct_bf16_peak": {"value": 100.0 * frame_tflops / peak_burst, "basis": f"burst bf16 {src}",
                           "sustained_basis": 100.0 * frame_tflops / peak_sus},
-        "roofline": {"bound": "tensor", "kernel": "attn_bf16_kernel", "achieved": attn_tflops, "peak": peak_burst,
+        "roofline": {"bound": "tensor", "kernel": "attn_pair_kernel", "achieved": attn_tflops, "peak": peak_burst,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak_burst, "traffic": attn_traffic(),
                      "peak_basis": f"bf16_tflops (burst) {src}",
                      "frac_vs_sustained": attn_tflops / peak_sus},

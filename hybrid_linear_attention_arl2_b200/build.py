@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libarl2.so")
-SOURCES = ["arl2_api.cu", "attn_bf16.cu", "attn_pair.cu", "gemm_bf16.cu", "state_bf16.cu", "f32_path.cu", "util.cu", "block.cu", "token_level.cu"]
+SOURCES = ["arl2_api.cu", "attn_pair.cu", "gemm_bf16.cu", "state_bf16.cu", "f32_path.cu", "util.cu", "block.cu", "token_level.cu"]
 HEADERS = ["params.h", "layer.h", "sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -17,11 +17,11 @@
 // accumulator in its own tensor memory.  S and P are double-buffered in tensor
 // memory and S is issued two key tiles ahead of the PV that consumes the
 // matching P, so the softmax of tile i finds S(i) ready as soon as it is done
-// with tile i - 1: it never waits for a PV, and the tensor core never waits
-// for the softmax of the tile it is about to compute.  The softmax of one tile
-// is split by columns between two warpgroups (keys 0..63 and 64..127 of the
-// same 128 rows), which exchange their partial row maxima through shared
-// memory.  The sequence of (block, key tile) units over all (stream, head)
+// with tile i - 2: it never waits for a PV, and the tensor core never waits
+// for the softmax of the tile it is about to compute.  The two softmax
+// warpgroups take alternate key tiles of the same 128 rows (the running row
+// max is handed from tile to tile through shared memory), so that one's waits
+// hide behind the other's exponentials.  The sequence of (block, key tile) units over all (stream, head)
 // pairs is cut into contiguous equal ranges, one per CTA pair ("stream-K").  A
 // block whose key range is split across pairs is finished by the pair holding
 // its key tile 0 (always that pair's last segment); the pairs continuing it
@@ -35,13 +35,11 @@
 //                halves of K_j, V_j (and of MqT for blocks it finishes)
 //                through a ring of 16 KB slots; the loads of both CTAs count
 //                on rank 0's barriers;
-//   warp 1       (rank 0 only) tcgen05 issuer: S(i) = Q K_i^T, O += P(i) V_i,
-//                X = Q MqT^T;
+//   warp 1       (rank 0 only) tcgen05 issuer of S(i) = Q K_i^T;
 //   warp 2       tensor-memory allocator (both CTAs, cta_group::2);
-//   warp 3       (rank 1 only) forwards its softmax warps' per-tile signals to
-//                rank 0's barriers, one cluster-scope arrive per signal;
-//   warps 4..7   softmax, keys 0..63 of every tile (one query row per thread);
-//   warps 8..11  softmax, keys 64..127;
+//   warp 3       (rank 0 only) tcgen05 issuer of O += P(i) V_i and X = Q MqT^T;
+//   warps 4..7   softmax of the even key tiles (one query row per thread);
+//   warps 8..11  softmax of the odd key tiles;
 //   warps 12..15 epilogue: at the end of a segment reads O (and X) from
 //                tensor memory, hands it back at once, merges the other pairs'
 //                pieces of a split block and writes the output with TMA tile
@@ -69,14 +67,14 @@ constexpr uint32_t kBox = 16384;    // 128 rows x 64 bf16
 constexpr uint32_t kSlot = 16384;   // a half tile: 64 keys x 128 dims, 128 keys x 64 dims, or 64 rows of MqT
 constexpr uint32_t kTilesBytes = 2 * kQTile + kRing * kSlot + kQTile;  // Q x2, ring, output staging
 constexpr uint32_t kBarBytes = 512;
-constexpr uint32_t kStatsBytes = 3 * 128 * 4 + 2 * 2 * 128 * 4;  // (m, l_lo, l_hi); partial maxima [2 halves][2 tiles]
+constexpr uint32_t kStatsBytes = 4 * 128 * 4 + 2 * 128 * 4;  // (m, l) per softmax warpgroup; running max hand-off [2]
 constexpr int kSmem = 232448;
 static_assert(kTilesBytes + kBarBytes + kStatsBytes + 1024 <= uint32_t(kSmem), "shared memory layout too large");
 constexpr int kMaxContrib = 8;
 constexpr int kLaunchRegs = 128;
-constexpr int kCtlRegs = 64;
-constexpr int kSoftmaxRegs = 160;
-constexpr int kEpiRegs = 128;
+constexpr int kCtlRegs = 56;
+constexpr int kSoftmaxRegs = 168;
+constexpr int kEpiRegs = 112;
 static_assert(128 * kCtlRegs + 256 * kSoftmaxRegs + 128 * kEpiRegs <= kThreads * kLaunchRegs,
               "register split too large");
 
@@ -86,19 +84,17 @@ enum {
   B_RF = 4,              // [kRing] ring slot loaded (rank 0: both CTAs' bytes)
   B_RE = 4 + kRing,      // [kRing] ring slot free (commit, both CTAs)
   B_SF = 4 + 2 * kRing,  // [2] S(i) in S[i & 1] (commit, both CTAs)
-  B_SC = B_SF + 2,       // [2] S[i & 1] read by the softmax (rank 0: its 8 warps + 1 forwarded from rank 1)
-  B_PF = B_SC + 2,       // [2] P(i) in P[i & 1] (rank 0: its 8 warps + 1 forwarded from rank 1)
-  B_PD = B_PF + 2,       // [2] PV(i) completed: P[i & 1] free, O current (commit, both CTAs)
-  B_XQ = B_PD + 2,       // [2 tiles][4 quarters] partial row maxima exchanged (local: 2 warps)
-  B_SD = B_XQ + 8,       // every MMA of the segment completed (commit, both CTAs)
+  B_SC = B_SF + 2,       // [2] S[i & 1] read by the softmax (rank 0: the owning warpgroup's 4 warps x 2 CTAs)
+  B_PF = B_SC + 2,       // [2] P(i) in P[i & 1] (rank 0: the owning warpgroup's 4 warps x 2 CTAs)
+  B_PD = B_PF + 2,       // [2] PV(i) done: P[i & 1] free, O current (commit, both CTAs)
+  B_MX = B_PD + 2,       // [2 tile parities][4 quarters] running max after tile i published (local: 1 warp)
+  B_SD = B_MX + 8,       // every MMA of the segment completed (commit, both CTAs)
   B_ST = B_SD + 1,       // the segment's statistics in shared memory (local: 8 warps)
   B_STC = B_ST + 1,      // statistics read by the epilogue (local: 4 warps)
   B_EO = B_STC + 1,      // epilogues done with O and X (rank 0: 4 warps x 2 CTAs)
   B_EL = B_EO + 1,       // this CTA's epilogue done with O and X (local: 4 warps)
   B_PQ = B_EL + 1,       // [4] a contributor's piece of this warp's rows in shared memory (local: bytes)
-  B_SCL = B_PQ + 4,      // [2] rank 1: its 8 softmax warps have read S[i & 1] (local)
-  B_PFL = B_SCL + 2,     // [2] rank 1: its 8 softmax warps have written P(i) (local)
-  B_DRAIN = B_PFL + 2,
+  B_DRAIN = B_PQ + 4,
   B_COUNT
 };
 static_assert(B_COUNT * 8 + 8 <= int(kBarBytes), "barrier area too small");
@@ -119,8 +115,8 @@ __device__ __forceinline__ bool next_seg(const AttnParams& p, unsigned& u, unsig
   return true;
 }
 
-// Ring positions within a segment of n key tiles, in the order the issuer
-// consumes them (S two tiles ahead of PV): K_0, K_1, K_2, V_0, K_3, V_1, ...,
+// Ring positions within a segment of n key tiles, in the order the issuers
+// consume them (S about two tiles ahead of PV): K_0, K_1, K_2, V_0, K_3, V_1, ...,
 // K_{n-1}, V_{n-3}, V_{n-2}, V_{n-1}, then MqT.
 __device__ __forceinline__ int pos_k(int i) { return i < 2 ? i : 2 * i - 2; }
 __device__ __forceinline__ int pos_v(int i, int n) {
@@ -240,26 +236,23 @@ __device__ __forceinline__ void mma_pv_group(const uint32_t d, const uint32_t p_
   }
 }
 
-// One thread of rank 0.  Tiles are counted over the whole launch (g): S(g)
-// goes to S[g & 1] once the softmax of both CTAs has read S(g - 2) out of it
-// (B_SC); PV(g) reads P[g & 1] once both CTAs' softmax has written P(g)
-// (B_PF).  Per segment of n key tiles the order is
-//     S(0), S(1), S(2), PV(0), S(3), PV(1), ..., S(n-1), PV(n-3), PV(n-2), PV(n-1)
-// then, for blocks finished here, X = Q MqT^T over [256, 384) (both P
-// buffers are consumed by then).  A segment's first PV, which overwrites O,
-// waits until the epilogues have read the previous segment's O and X (B_EO).
-__device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, const uint32_t tmem,
-                                           const uint32_t q_addr, const uint32_t r_addr, const unsigned u_begin,
-                                           const unsigned u_end, const WaitCtl& w) {
+// Two threads of rank 0 issue the MMAs, so that a PV whose P is ready never
+// queues behind the issue of an S (a thread issuing tcgen05.mma stalls while
+// the tensor pipe's queue is full, ~the execution time of what it issues).
+// Tiles are counted over the whole launch (g).
+//
+// S issuer: S(g) goes to S[g & 1] once the softmax of both CTAs has read
+// S(g - 2) out of it (B_SC); it runs up to two tiles ahead of the softmax.
+__device__ __forceinline__ void s_issuer(const AttnParams& p, uint64_t* bars, const uint32_t tmem,
+                                         const uint32_t q_addr, const uint32_t r_addr, const unsigned u_begin,
+                                         const unsigned u_end, const WaitCtl& w) {
   constexpr uint32_t kQ16 = kQTile >> 4, kSlot16 = kSlot >> 4;
   const uint32_t id_s = idesc_bf16(256, 128, 0, 0);
-  const uint32_t id_o = idesc_bf16(256, 128, 0, 1);
   const uint64_t dq64 = smem_desc_sw128(q_addr, 16, 1024);
   const uint32_t hi = uint32_t(dq64 >> 32);
   const uint32_t dq0 = uint32_t(dq64);
-  const uint32_t dk0 = uint32_t(smem_desc_sw128(r_addr, 16, 1024));     // K-major ring slot
-  const uint32_t dv0 = uint32_t(smem_desc_sw128(r_addr, kBox, 1024));   // MN-major ring slot
-  uint32_t ring = 0, k = 0, gs = 0, gp = 0;
+  const uint32_t dk0 = uint32_t(smem_desc_sw128(r_addr, 16, 1024));  // K-major ring slot
+  uint32_t ring = 0, k = 0, gs = 0;
   unsigned u = u_begin;
   Seg s;
   while (next_seg(p, u, u_end, s)) {
@@ -267,42 +260,66 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, 
     const uint32_t qs = k & 1;
     const uint32_t dq = dq0 + qs * kQ16;
     if (!mbar_wait(&bars[B_QF + qs], (k >> 1) & 1, w)) return;
-    const uint32_t r0 = ring;
-    for (int i = 0; i < n + 2; ++i) {
-      if (i < n) {  // S(i)
-        const uint32_t rk = r0 + pos_k(i), buf = gs & 1;
-        if (!mbar_wait(&bars[B_RF + rk % kRing], (rk / kRing) & 1, w)) return;
-        if (gs >= 2) {
-          if (!mbar_wait(&bars[B_SC + buf], ((gs - 2) >> 1) & 1, w)) return;
-          tc_fence_after();
-        }
-        mma_s_group(tmem + buf * 128, dq, dk0 + (rk % kRing) * kSlot16, hi, id_s);
-        mma_commit_pair(&bars[B_SF + buf]);
-        mma_commit_pair(&bars[B_RE + rk % kRing]);
-        ++gs;
-      }
-      if (i >= 2 || (n == 1 && i == 1)) {  // PV(j)
-        const int j = n == 1 ? 0 : i - 2;
-        if (j >= n) continue;
-        const uint32_t rv = r0 + pos_v(j, n), buf = gp & 1;
-        if (!mbar_wait(&bars[B_RF + rv % kRing], (rv / kRing) & 1, w)) return;
-        if (!mbar_wait(&bars[B_PF + buf], (gp >> 1) & 1, w)) return;
-        if (j == 0 && k > 0 && !mbar_wait(&bars[B_EO], (k - 1) & 1, w)) return;
+    for (int i = 0; i < n; ++i, ++gs) {
+      const uint32_t rk = ring + pos_k(i), buf = gs & 1;
+      if (!mbar_wait(&bars[B_RF + rk % kRing], (rk / kRing) & 1, w)) return;
+      if (gs >= 2) {
+        if (!mbar_wait(&bars[B_SC + buf], ((gs - 2) >> 1) & 1, w)) return;
         tc_fence_after();
-        const int valid = min(128, p.kv_len - (s.j0 + j) * 128);
-        mma_pv_group(tmem + 384, tmem + 256 + buf * 64, dv0 + (rv % kRing) * kSlot16, hi, id_o, (valid + 15) >> 4,
-                     j > 0);
-        mma_commit_pair(&bars[B_PD + buf]);
-        mma_commit_pair(&bars[B_RE + rv % kRing]);
-        ++gp;
-        if (n == 1) break;
       }
+      mma_s_group(tmem + buf * 128, dq, dk0 + (rk % kRing) * kSlot16, hi, id_s);
+      mma_commit_pair(&bars[B_SF + buf]);
+      mma_commit_pair(&bars[B_RE + rk % kRing]);
     }
-    ring = r0 + 2 * n;
+    ring += 2 * n + ((s.j0 == 0 && p.has_inter) ? 1 : 0);
+    ++k;
+  }
+}
+
+// PV issuer: PV(g) reads P[g & 1] once both CTAs' softmax has written P(g)
+// (B_PF); a segment's first PV, which overwrites O, waits until the
+// epilogues have read the previous segment's O and X (B_EO).  Then, for
+// blocks finished here, X = Q MqT^T over [256, 384) (both P buffers are
+// consumed by then).  Every S of the segment has completed before its last
+// PV is issued (the softmax read S first), so this thread's commits also
+// stand for them: B_SD (the segment's MMAs done) and B_QE (Q slot free).
+__device__ __forceinline__ void pv_issuer(const AttnParams& p, uint64_t* bars, const uint32_t tmem,
+                                          const uint32_t q_addr, const uint32_t r_addr, const unsigned u_begin,
+                                          const unsigned u_end, const WaitCtl& w) {
+  constexpr uint32_t kQ16 = kQTile >> 4, kSlot16 = kSlot >> 4;
+  const uint32_t id_s = idesc_bf16(256, 128, 0, 0);
+  const uint32_t id_o = idesc_bf16(256, 128, 0, 1);
+  const uint64_t dq64 = smem_desc_sw128(q_addr, 16, 1024);
+  const uint32_t hi = uint32_t(dq64 >> 32);
+  const uint32_t dq0 = uint32_t(dq64);
+  const uint32_t dk0 = uint32_t(smem_desc_sw128(r_addr, 16, 1024));    // K-major ring slot (MqT)
+  const uint32_t dv0 = uint32_t(smem_desc_sw128(r_addr, kBox, 1024));  // MN-major ring slot (V)
+  uint32_t ring = 0, k = 0, gp = 0;
+  unsigned u = u_begin;
+  Seg s;
+  while (next_seg(p, u, u_end, s)) {
+    const int n = s.j1 - s.j0;
+    const uint32_t qs = k & 1;
+    for (int j = 0; j < n; ++j, ++gp) {
+      const uint32_t rv = ring + pos_v(j, n), buf = gp & 1;
+      if (!mbar_wait(&bars[B_RF + rv % kRing], (rv / kRing) & 1, w)) return;
+      if (!mbar_wait(&bars[B_PF + buf], (gp >> 1) & 1, w)) return;
+      if (j == 0 && k > 0 && !mbar_wait(&bars[B_EO], (k - 1) & 1, w)) return;
+      tc_fence_after();
+      const int valid = min(128, p.kv_len - (s.j0 + j) * 128);
+      mma_pv_group(tmem + 384, tmem + 256 + buf * 64, dv0 + (rv % kRing) * kSlot16, hi, id_o, (valid + 15) >> 4,
+                   j > 0);
+      mma_commit_pair(&bars[B_PD + buf]);
+      mma_commit_pair(&bars[B_RE + rv % kRing]);
+    }
+    ring += 2 * n;
     if (s.j0 == 0 && p.has_inter) {  // X = Q MqT^T for the rows this pair finishes
       const uint32_t rm = ring;
+      // Q is in (the S issuer saw it); waited on here too so that this
+      // thread's MMA reads it after observing the load's completion
+      if (!mbar_wait(&bars[B_QF + qs], (k >> 1) & 1, w)) return;
       if (!mbar_wait(&bars[B_RF + rm % kRing], (rm / kRing) & 1, w)) return;
-      mma_s_group(tmem + 256, dq, dk0 + (rm % kRing) * kSlot16, hi, id_s);
+      mma_s_group(tmem + 256, dq0 + qs * kQ16, dk0 + (rm % kRing) * kSlot16, hi, id_s);
       mma_commit_pair(&bars[B_RE + rm % kRing]);
       ++ring;
     }
@@ -313,48 +330,104 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint64_t* bars, 
 }
 
 // ------------------------------------------------------------------ softmax
-// Two warpgroups share every tile: half h takes keys 64h .. 64h + 63 of the
-// 128 rows (one row per thread).  Per tile g: its 64 columns of S from S[g & 1]
-// (then S[g & 1] is handed back to the issuer); the half's row maximum,
-// exchanged with the other half through shared memory; lazy rescaling (the
-// running max m moves only when the tile's max exceeds it by more than 8, a
-// factor 256; then O is rescaled in tensor memory, each half its 64 columns,
-// once the previous PV has completed); P = 2^(S * scale * log2(e) - m) packed
-// to bf16 pairs into P[g & 1] (free once PV(g - 2) has completed); the half's
-// running row sum l.  Both halves take the same decisions from the same row
-// maxima.  At the end of a segment (m, l) go to shared memory for the epilogue.
-__device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars, float* stats, float* xmax,
-                                             const uint32_t tmem, const int rank, const int half, const int quarter,
+// The two softmax warpgroups take alternate key tiles of the same 128 rows:
+// warpgroup w owns the tiles g with g & 1 == w, so it always reads S[w] and
+// writes P[w], one query row per thread and all 128 columns of the tile.
+// While one computes the exponentials of tile g the other is on tile g + 1,
+// so each one's waits and tensor-memory round trips hide behind the other's
+// arithmetic.  The running row max m is handed along the tiles in order
+// through shared memory: the owner of tile g takes m after tile g - 1 (which
+// the other warpgroup publishes right after its row max, long before S(g) is
+// in), raises it only when the tile's max exceeds it by more than 8 (a factor
+// 256, so P <= 256), and publishes it before its exponentials.  A raised m
+// rescales O (all 128 columns of the CTA's rows) once PV(g - 1) has completed
+// and before P(g) is announced; rare.  Each warpgroup keeps its own row sum l
+// against the last m it used; at the end of a segment both (m, l) go to
+// shared memory and the epilogue combines them.
+// 2^x for a pair on the FMA pipe: x = n + f with n = round(x) (adding
+// 1.5 * 2^23 leaves n in the low mantissa bits), 2^f from the degree-3
+// polynomial through the four Chebyshev nodes of [-1/2, 1/2] (coefficients of
+// exp2_poly, relative error <= 1.0e-4, below the 2^-9 step of the bf16 P it
+// feeds), 2^n added to the exponent field.  x is clamped below at -125.
+__device__ __forceinline__ float2 exp2_poly_pair(float2 x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  constexpr float c0 = 0.999924541f, c1 = 0.693136752f, c2 = 0.242639482f, c3 = 0.0558382832f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 f = __fadd2_rn(x, __fadd2_rn(make_float2(kRound, kRound), make_float2(-t.x, -t.y)));
+  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = __ffma2_rn(q, f, make_float2(c1, c1));
+  q = __ffma2_rn(q, f, make_float2(c0, c0));
+  return make_float2(__uint_as_float((__float_as_uint(t.x) << 23) + __float_as_uint(q.x)),
+                     __uint_as_float((__float_as_uint(t.y) << 23) + __float_as_uint(q.y)));
+}
+
+// Of the 16 pairs of each 32-column chunk, this many take the FMA-pipe
+// exponential (pairs 1, 4, 7, ...); the rest take the MUFU.
+constexpr int kPolyPerChunk = 5;
+
+// P = 2^(S * scale * log2(e) - m) for 32 columns of a row, packed to bf16
+// pairs; returns their sum.
+template <bool kPoly>
+__device__ __forceinline__ float exp_chunk(const uint32_t* r, const float2 sc, const float2 nm, uint32_t (&pk)[16]) {
+  float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int x = 0; x < 16; ++x) {
+    const float2 y = __ffma2_rn(make_float2(__uint_as_float(r[2 * x]), __uint_as_float(r[2 * x + 1])), sc, nm);
+    const bool poly = kPoly && (x % 3 == 1) && (x / 3) < kPolyPerChunk;
+    const float2 e = poly ? exp2_poly_pair(y) : make_float2(fast_exp2(y.x), fast_exp2(y.y));
+    s2[x & 1] = __fadd2_rn(s2[x & 1], e);
+    pk[x] = pack_bf16x2(e.x, e.y);
+  }
+  const float2 sa = __fadd2_rn(s2[0], s2[1]);
+  return sa.x + sa.y;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars, float* stats, float* mchain,
+                                             const uint32_t tmem, const int rank, const int wgi, const int quarter,
                                              const int lane, const unsigned u_begin, const unsigned u_end,
                                              const WaitCtl& w) {
   const int row = quarter * 32 + lane;
   const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-  // rank 0 arrives on its own barriers; rank 1 on local ones that its
-  // forwarder relays (a cluster-scope arrive costs each warp ~10^3 cycles)
-  const int sc_bar = rank == 0 ? B_SC : B_SCL, pf_bar = rank == 0 ? B_PF : B_PFL;
-  const uint32_t tO = tmem + 384 + half * 64;
-  const float sl2 = p.scale_log2;
+  const uint32_t tS = tmem + wgi * 128 + lane_off;       // S[wgi]
+  const uint32_t tP = tmem + 256 + wgi * 64 + lane_off;  // P[wgi]
+  const uint32_t tO = tmem + 384 + lane_off;
+  // rank 1's warps arrive on rank 0's barriers themselves: a relaxed
+  // cluster-scope arrive after tcgen05.wait and the thread-sync fence (the
+  // release form costs each warp ~10^3 cycles)
+  const uint32_t sc_lead = cluster_map(smem_u32(&bars[B_SC + wgi]), 0);
+  const uint32_t pf_lead = cluster_map(smem_u32(&bars[B_PF + wgi]), 0);
+  const float2 sc = make_float2(p.scale_log2, p.scale_log2);
   uint32_t g = 0, k = 0;
   unsigned u = u_begin;
   Seg s;
   while (next_seg(p, u, u_end, s)) {
     const int n = s.j1 - s.j0;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // the last m this warpgroup used, and its l against it
+    bool first = true;
     for (int i = 0; i < n; ++i, ++g) {
-      const uint32_t buf = g & 1, ph = (g >> 1) & 1;
-      if (!warp_wait(&bars[B_SF + buf], ph, w)) return;
+      if (int(g & 1) != wgi) continue;
+      if (!warp_wait(&bars[B_SF + wgi], (g >> 1) & 1, w)) return;
       tc_fence_after();
-      const int valid = min(128, p.kv_len - (s.j0 + i) * 128) - half * 64;  // valid columns of this half
-      uint32_t r[64];
-      tmem_ld32(tmem + buf * 128 + half * 64 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(tmem + buf * 128 + half * 64 + 32 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      uint32_t r[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[sc_bar + buf]);  // S[buf] may take the next S
-      if (valid < 64) {
+      if (lane == 0) {  // S[wgi] may take S(g + 2)
+        if (rank == 0) mbar_arrive(&bars[B_SC + wgi]);
+        else mbar_arrive_cluster_relaxed(sc_lead);
+      }
+      const int valid = min(128, p.kv_len - (s.j0 + i) * 128);
+      if (valid < 128) {
 #pragma unroll
-        for (int x = 0; x < 64; ++x)
+        for (int x = 0; x < 128; ++x)
           if (x >= valid) r[x] = __float_as_uint(-INFINITY);
       }
       float m4[4];
@@ -362,96 +435,76 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars
       for (int q = 0; q < 4; ++q)
         m4[q] = fmax3(__uint_as_float(r[q]), __uint_as_float(r[4 + q]), __uint_as_float(r[8 + q]));
 #pragma unroll
-      for (int x = 12; x < 60; x += 8)
+      for (int x = 12; x < 124; x += 8)
 #pragma unroll
         for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], __uint_as_float(r[x + q]), __uint_as_float(r[x + 4 + q]));
 #pragma unroll
-      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], __uint_as_float(r[60 + q]));
-      const float pm = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-      xmax[(half * 2 + buf) * 128 + row] = pm;
+      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], __uint_as_float(r[124 + q]));
+      const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sc.x;
+      // m after tile g - 1, from the other warpgroup; waited for at a
+      // segment's first tile too (value unused) so that the two hand-off
+      // slots are never rewritten before they are read
+      float m_in = -INFINITY;
+      if (g > 0) {
+        const uint32_t gq = g - 1;
+        if (!warp_wait(&bars[B_MX + (gq & 1) * 4 + quarter], (gq >> 1) & 1, w)) return;
+        if (i > 0) m_in = mchain[(gq & 1) * 128 + row];
+      }
+      const bool need = i > 0 && mx > m_in + 8.f;
+      const float mg = (i == 0 || need) ? mx : m_in;
+      mchain[(g & 1) * 128 + row] = mg;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_XQ + buf * 4 + quarter]);
-      if (!warp_wait(&bars[B_XQ + buf * 4 + quarter], ph, w)) return;
-      const float mx = fmaxf(pm, xmax[((1 - half) * 2 + buf) * 128 + row]) * sl2;
-      float f = 1.f;
-      bool any_rescale = false;
-      if (i == 0) {
-        m = mx;
-      } else {
-        const bool need = mx > m + 8.f;
-        any_rescale = __any_sync(0xffffffffu, need);
-        if (need) {
-          f = fast_exp2(m - mx);
-          m = mx;
-        }
-      }
-      const float2 sc = make_float2(sl2, sl2), nm = make_float2(-m, -m);
-      float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      uint32_t pk[32];
+      if (lane == 0) mbar_arrive(&bars[B_MX + (g & 1) * 4 + quarter]);
+      const bool any_rescale = __any_sync(0xffffffffu, need);
+      // the exponentials go to registers first: P[wgi] is free only once
+      // PV(g - 2) has completed, and a warpgroup's first tile of a segment
+      // also waits until the epilogue is done with X, which overlays both P
+      // buffers
+      const float2 nm = make_float2(-mg, -mg);
+      float sum = 0.f;
+      uint32_t pk[64];
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const float2 y =
-            __ffma2_rn(make_float2(__uint_as_float(r[2 * x]), __uint_as_float(r[2 * x + 1])), sc, nm);
-        const float2 e = make_float2(fast_exp2(y.x), fast_exp2(y.y));
-        s2[x & 3] = __fadd2_rn(s2[x & 3], e);
-        pk[x] = pack_bf16x2(e.x, e.y);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t(&pc)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk[16 * c]);
+        sum += valid >= 128 ? exp_chunk<true>(&r[32 * c], sc, nm, pc) : exp_chunk<false>(&r[32 * c], sc, nm, pc);
       }
-      // P[buf] is free once PV(g - 2) has completed; at a segment's first tile
-      // the epilogue must also be done with X, which overlays both P buffers
-      if (g >= 2 && !warp_wait(&bars[B_PD + buf], ((g - 2) >> 1) & 1, w)) return;
-      if (i == 0 && k > 0 && !warp_wait(&bars[B_EL], (k - 1) & 1, w)) return;
-      if (any_rescale) {  // rare: O is rescaled (after PV(g - 1)) before P is announced
-        if (!warp_wait(&bars[B_PD + (buf ^ 1)], ((g - 1) >> 1) & 1, w)) return;
+      if (g >= 2 && !warp_wait(&bars[B_PD + wgi], ((g - 2) >> 1) & 1, w)) return;
+      if (first && k > 0 && !warp_wait(&bars[B_EL], (k - 1) & 1, w)) return;
+      first = false;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st16(tP + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * c]));
+      if (any_rescale) {  // O *= 2^(m_in - mg) (1 for rows that keep m) once PV(g - 1) has completed
+        if (!warp_wait(&bars[B_PD + (wgi ^ 1)], ((g - 1) >> 1) & 1, w)) return;
         tc_fence_after();
+        const float f = fast_exp2(m_in - mg);
 #pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
-          tmem_ld32(tO + lane_off + q * 32, o);
+          tmem_ld32(tO + q * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
-          tmem_st32(tO + lane_off + q * 32, o);
+          tmem_st32(tO + q * 32, o);
         }
       }
-      tc_fence_after();
-      tmem_st16(tmem + 256 + buf * 64 + half * 32 + lane_off, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-      tmem_st16(tmem + 256 + buf * 64 + half * 32 + 16 + lane_off, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
-      const float2 s01 = __fadd2_rn(s2[0], s2[1]), s23 = __fadd2_rn(s2[2], s2[3]);
-      const float2 sa = __fadd2_rn(s01, s23);
-      l = fmaf(l, f, sa.x + sa.y);
+      l = fmaf(l, m == mg ? 1.f : fast_exp2(m - mg), sum);
+      m = mg;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[pf_bar + buf]);
+      if (lane == 0) {  // P(g) is in
+        if (rank == 0) mbar_arrive(&bars[B_PF + wgi]);
+        else mbar_arrive_cluster_relaxed(pf_lead);
+      }
     }
     // the epilogue has read the previous segment's statistics
     if (k > 0 && !warp_wait(&bars[B_STC], (k - 1) & 1, w)) return;
-    if (half == 0) stats[row] = m;
-    stats[(1 + half) * 128 + row] = l;
+    stats[wgi * 256 + row] = m;  // -inf, 0 for a warpgroup with no tile in the segment
+    stats[wgi * 256 + 128 + row] = l;
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[B_ST]);
     ++k;
-  }
-}
-
-// ------------------------------------------------------------------ forwarder
-// One thread of rank 1: relays its softmax warps' per-tile signals (S[i & 1]
-// read, P(i) written) to rank 0's barriers with one cluster-scope arrive each,
-// in the order they occur, so that no softmax warp pays for a remote arrive.
-__device__ __forceinline__ void forwarder(const AttnParams& p, uint64_t* bars, const unsigned u_begin,
-                                          const unsigned u_end, const WaitCtl& w) {
-  const uint32_t sc0 = cluster_map(smem_u32(&bars[B_SC]), 0), pf0 = cluster_map(smem_u32(&bars[B_PF]), 0);
-  uint32_t g = 0;
-  unsigned u = u_begin;
-  Seg s;
-  while (next_seg(p, u, u_end, s)) {
-    for (int i = 0; i < s.j1 - s.j0; ++i, ++g) {
-      const uint32_t buf = g & 1, ph = (g >> 1) & 1;
-      if (!mbar_wait(&bars[B_SCL + buf], ph, w)) return;
-      mbar_arrive_cluster(sc0 + buf * 8);
-      if (!mbar_wait(&bars[B_PFL + buf], ph, w)) return;
-      mbar_arrive_cluster(pf0 + buf * 8);
-    }
   }
 }
 
@@ -552,7 +605,8 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
     if (!warp_wait(&bars[B_SD], k & 1, w)) return false;
     if (!warp_wait(&bars[B_ST], k & 1, w)) return false;
     tc_fence_after();
-    const float M = stats[row], L = stats[128 + row] + stats[256 + row];
+    const float m0 = stats[row], m1 = stats[256 + row], M = fmaxf(m0, m1);
+    const float L = stats[128 + row] * fast_exp2(m0 - M) + stats[384 + row] * fast_exp2(m1 - M);
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[B_STC]);
     float a0 = 0.f, wk[kMaxContrib];
@@ -697,8 +751,8 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTilesBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + B_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* stats = reinterpret_cast<float*>(smem + kTilesBytes + kBarBytes);  // m[128], l_lo[128], l_hi[128]
-  float* xmax = stats + 3 * 128;                                            // [2 halves][2 tiles][128]
+  float* stats = reinterpret_cast<float*>(smem + kTilesBytes + kBarBytes);  // per warpgroup m[128], l[128]
+  float* mchain = stats + 4 * 128;                                          // running max hand-off [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
@@ -712,9 +766,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t count = 1;
-      if (i >= B_SC && i < B_PF + 2) count = 9;   // rank 0's 8 softmax warps + rank 1's forwarder
-      if (i >= B_SCL && i < B_PFL + 2) count = 8;  // rank 1's 8 softmax warps
-      if (i >= B_XQ && i < B_XQ + 8) count = 2;   // the two halves' warps of one quarter
+      if (i >= B_SC && i < B_PF + 2) count = 8;   // the owning warpgroup's 4 warps in each CTA
       if (i == B_ST) count = 8;                    // 8 softmax warps
       if (i == B_STC || i == B_EL) count = 4;      // the epilogue's 4 warps
       if (i == B_EO) count = 8;                    // 4 epilogue warps x 2 CTAs (rank 0's copy)
@@ -741,9 +793,9 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tma_prefetch(&tm_v);
         producer(p, bars, sQ, sR, &tm_q, &tm_k, &tm_v, &tm_mq, rank, u_begin, u_end, w);
       } else if (warp == 1 && lane == 0 && rank == 0) {
-        mma_issuer(p, bars, tmem, smem_u32(sQ), smem_u32(sR), u_begin, u_end, w);
-      } else if (warp == 3 && lane == 0 && rank == 1) {
-        forwarder(p, bars, u_begin, u_end, w);
+        s_issuer(p, bars, tmem, smem_u32(sQ), smem_u32(sR), u_begin, u_end, w);
+      } else if (warp == 3 && lane == 0 && rank == 0) {
+        pv_issuer(p, bars, tmem, smem_u32(sQ), smem_u32(sR), u_begin, u_end, w);
       }
       __syncwarp();
     } else if (wg == 3) {
@@ -751,7 +803,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       epilogue_role(p, bars, stats, sStage, sQ, &tm_o, tmem, cta, rank, warp & 3, lane, u_begin, u_end, abort_flag, w);
     } else {
       regs_inc<kSoftmaxRegs>();
-      softmax_role(p, bars, stats, xmax, tmem, rank, wg - 1, warp & 3, lane, u_begin, u_end, w);
+      softmax_role(p, bars, stats, mchain, tmem, rank, wg - 1, warp & 3, lane, u_begin, u_end, w);
     }
   }
 
@@ -836,7 +888,6 @@ int attn_pair_capacity() {
 
 bool attn_pair_partition(AttnParams& p, int batch, int max_pairs) {
   p.n_qt = (p.q_len + 127) / 128;
-  p.n_pair = p.n_qt / 2;
   p.n_blk = (p.n_qt + 1) / 2;
   p.nkv = (p.kv_len + 127) / 128;
   const long long bh = (long long)batch * p.heads;

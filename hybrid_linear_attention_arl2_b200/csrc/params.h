@@ -11,44 +11,37 @@ namespace arl2 {
 
 constexpr int kAttnMaxGrid = 192;  // persistent CTAs at most (>= the SM count of a B200)
 
-// Fused intra-frame softmax + inter-frame read-out (attn_bf16.cu): a
-// persistent grid over (query-tile pair, key tile) units, see the kernel.
+// Fused intra-frame softmax + inter-frame read-out (attn_pair.cu): a
+// persistent grid of CTA pairs over (256-row block, key tile) units, see the
+// kernel.
 struct AttnParams {
   int q_len;            // query tokens per stream
   int kv_len;           // valid key/value tokens per stream
   int heads;
   int n_qt;             // query tiles of 128 per (stream, head)
-  int n_pair;           // n_qt / 2: blocks with two sub-tiles
-  int n_blk;            // blocks per (stream, head): n_pair + n_qt % 2
+  int n_blk;            // blocks of 256 rows per (stream, head): ceil(n_qt / 2)
   int nkv;              // key tiles of 128
   long long total_units;   // B * H * n_blk * nkv
-  int grid;             // persistent CTAs (<= kAttnMaxGrid)
-  unsigned range[kAttnMaxGrid + 1];  // CTA c takes units [range[c], range[c + 1])
+  int grid;             // persistent CTAs, even (<= kAttnMaxGrid)
+  unsigned range[kAttnMaxGrid + 1];  // pair c takes units [range[c], range[c + 1])
   float scale_log2;     // softmax scale * log2(e)
   uint32_t flags;       // 1: intra only, 2: inter only
   int has_inter;        // 1: add Q MqT^T
-  float* scratch;       // [grid][2][kAttnSlotFloats] normalised partial O (bf16, chunk-major) and (m, l)
-  unsigned* ready;      // [grid][2] partial-ready flags, zero between launches
+  float* scratch;       // [grid][kAttnPairSlotFloats] normalised partial O and (m, l) per CTA
+  unsigned* ready;      // [grid][kAttnPairFlags] partial-ready flags, zero between launches
   uint32_t* err;        // device error word
   uint64_t wait_limit_ns;
 };
 
-// floats of one partial slot (one sub-tile of one CTA): 128 x 128 O values
-// normalised by the slot's own l, in bf16, stored chunk-major (16-byte chunk i of row r at byte (i * 128 + r) * 16),
-// then m[128] and l[128] in fp32
-constexpr int kAttnSlotFloats = 128 * 64 + 256;
-
 // floats of one CTA's partial slot of the CTA-pair kernel (attn_pair.cu): its
-// 128 x 128 piece of O in fp32, normalised by its own l, chunk-major (16-byte
-// chunk i of row r at float (i * 128 + r) * 4), then m[128] and l[128]
+// 128 x 128 piece of O normalised by its own l, in bf16 (the first 8192
+// floats' bytes, laid out as the kernel describes), then from float 16384
+// m[128] and l[128] in fp32
 constexpr int kAttnPairSlotFloats = 128 * 128 + 256;
 // ready flags per CTA of the pair kernel (one per epilogue warp)
 constexpr int kAttnPairFlags = 4;
 // device words of the attention scratch and flags a handle allocates for `sms` SMs
-constexpr size_t attn_scratch_floats(int sms) {
-  return size_t(sms) * (2 * size_t(kAttnSlotFloats) > size_t(kAttnPairSlotFloats) ? 2 * size_t(kAttnSlotFloats)
-                                                                                  : size_t(kAttnPairSlotFloats));
-}
+constexpr size_t attn_scratch_floats(int sms) { return size_t(sms) * size_t(kAttnPairSlotFloats); }
 constexpr size_t attn_ready_words(int sms) { return size_t(sms) * kAttnPairFlags; }
 
 // State write and read-out preparation (state_bf16.cu).
@@ -94,22 +87,17 @@ struct F32CommitParams {
   float corr;
 };
 
-// tq, tk, tv: Q, K, V maps; tmq: MqT map (read only when has_inter); tmo: the
-// output O [B, q_len, H, 128] in boxes of 64 columns x 32 rows, written with
-// tile stores.
-cudaError_t launch_attn_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const CUtensorMap& tmq, const CUtensorMap& tmo, const AttnParams& p,
-                             cudaStream_t stream);
-// Fills the partition fields of `p` for B streams on a device with `sms` SMs;
-// false if the problem is too large for 32-bit unit indices.
-bool attn_partition(AttnParams& p, int batch, int sms);
-// The same on CTA pairs (attn_pair.cu): tk holds 64-row boxes (a CTA's half of
-// a key tile), tv 128-row boxes, tmq 64-row boxes of the [B*H, 128, 128] MqT
-// slabs; p.grid is the CTA count (even), p.range is per pair.
+// tq: Q in 128-row boxes; tk: K in 64-row boxes (a CTA's half of a key tile);
+// tv: V in 128-row boxes; tmq: 64-row boxes of the [B*H, 128, 128] MqT slabs
+// (read only when has_inter); tmo: the output O [B, q_len, H, 128] in boxes
+// of 64 columns x 32 rows, written with tile stores.  p.grid is the CTA count
+// (even), p.range is per pair.
 cudaError_t launch_attn_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tmq, const CUtensorMap& tmo, const AttnParams& p,
                              cudaStream_t stream);
-// max_pairs: the clusters of two the device holds at once (attn_pair_capacity).
+// Fills the partition fields of `p` for B streams; max_pairs: the clusters of
+// two the device holds at once (attn_pair_capacity).  False if the problem is
+// too large for 32-bit unit indices.
 bool attn_pair_partition(AttnParams& p, int batch, int max_pairs);
 // Clusters of the pair kernel resident at once on the current device (0 on error).
 int attn_pair_capacity();
