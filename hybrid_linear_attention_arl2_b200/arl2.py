@@ -76,6 +76,7 @@ _SIGS = {
     "arl2_selftest_wait_timeout": (_I32, [_U64, _VP]),
     "arl2_selftest_exp2": (_I32, [_VP, _VP, _I64, _VP]),
     "arl2_gemm_bf16": (_I32, [_VP, _I64, _VP, _I64, _VP, _I64, _I64, _I64, _I64, _VP]),
+    "arl2_attn_partition": (_I32, [_I32, _I32, _I32, _I32, _I32, _VP, _I32, _VP, _VP, _VP]),
     "arl2_status_string": (ctypes.c_char_p, [_I32]),
     "arl2_abi_version": (_I32, []),
 }
@@ -281,6 +282,21 @@ def arl2_gemm_bf16(a, b, c, m, n, k, lda=None, ldb=None, ldc=None, stream=None) 
     dimensions default to k, n and n)."""
     _check(load_library().arl2_gemm_bf16(_ptr(a), lda or k, _ptr(b), ldb or n, _ptr(c), ldc or n, m, n, k,
                                          _stream(stream)), "arl2_gemm_bf16")
+
+
+def arl2_attn_partition(batch, heads, q_len, kv_len, pairs, max_segs=1024):
+    """The attention kernel's work partition (host only): a list per pair of
+    segments (slab, block, j0, j1, n_contrib)."""
+    segs = (ctypes.c_int32 * (5 * max_segs))()
+    first = (ctypes.c_int32 * 97)()
+    n_segs, n_pairs = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load_library().arl2_attn_partition(batch, heads, q_len, kv_len, pairs, ctypes.cast(segs, ctypes.c_void_p).value,
+                                              max_segs, ctypes.cast(first, ctypes.c_void_p).value,
+                                              ctypes.addressof(n_segs), ctypes.addressof(n_pairs)), "arl2_attn_partition")
+    out = []
+    for c in range(n_pairs.value):
+        out.append([tuple(segs[5 * i:5 * i + 5]) for i in range(first[c], first[c + 1])])
+    return out
 
 
 def arl2_selftest_exp2(x, y, stream=None) -> None:

@@ -869,6 +869,32 @@ arl2_status arl2_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   return static_cast<arl2_status>(w);
 }
 
+arl2_status arl2_attn_partition(int batch, int heads, int q_len, int kv_len, int pairs, int32_t* segs, int max_segs,
+                                int32_t* seg_first, int* n_segs, int* n_pairs) {
+  if (!segs || !seg_first || !n_segs || !n_pairs || batch < 1 || heads < 1 || q_len < 1 || kv_len < 1 || pairs < 1 ||
+      pairs > arl2::kAttnMaxGrid / 2 || max_segs < 1)
+    return ARL2_ERR_INVALID_ARGUMENT;
+  arl2::AttnParams p{};
+  p.q_len = q_len;
+  p.kv_len = kv_len;
+  p.heads = heads;
+  if (!arl2::attn_pair_partition(p, batch, pairs) || p.n_segs > max_segs) return ARL2_ERR_UNSUPPORTED;
+  const int np = p.grid / 2;
+  for (int c = 0; c <= np; ++c) seg_first[c] = int32_t(p.seg_first[c]);
+  for (int i = 0; i < p.n_segs; ++i) {
+    const uint2 e = p.seg[i];
+    const int j0 = int((e.y >> 10) & 2047u);
+    segs[5 * i + 0] = int32_t(e.x & 0x0FFFFFFFu);
+    segs[5 * i + 1] = int32_t(e.y & 1023u);
+    segs[5 * i + 2] = j0;
+    segs[5 * i + 3] = j0 + int32_t(e.y >> 21);
+    segs[5 * i + 4] = int32_t(e.x >> 28);
+  }
+  *n_segs = p.n_segs;
+  *n_pairs = np;
+  return ARL2_OK;
+}
+
 arl2_status arl2_gemm_bf16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c, int64_t ldc, int64_t m,
                            int64_t n, int64_t k, void* stream) {
   if (!a || !b || !c || !aligned16(a) || !aligned16(b) || !aligned16(c)) return ARL2_ERR_INVALID_ARGUMENT;

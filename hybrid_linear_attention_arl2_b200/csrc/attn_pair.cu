@@ -21,11 +21,14 @@
 // for the softmax of the tile it is about to compute.  The two softmax
 // warpgroups take alternate key tiles of the same 128 rows (the running row
 // max is handed from tile to tile through shared memory), so that one's waits
-// hide behind the other's exponentials.  The sequence of (block, key tile) units over all (stream, head)
-// pairs is cut into contiguous equal ranges, one per CTA pair ("stream-K").  A
-// block whose key range is split across pairs is finished by the pair holding
-// its key tile 0 (always that pair's last segment); the pairs continuing it
-// store their normalised partial output and (m, l) in fp32 and raise ready
+// hide behind the other's exponentials.  Each pair walks its own list of
+// segments (a run of key tiles of one block), made on the host: whole blocks
+// where the blocks divide evenly over the pairs, the rest cut into pieces
+// (or plain equal ranges of the (block, key tile) sequence, "stream-K", when
+// that costs less).  A block whose key range is split across pairs is
+// finished by the pair holding its key tile 0 (always that pair's last
+// segment); the pairs continuing it (their first segment) store their
+// normalised partial output in bf16 with (m, l) in fp32 and raise ready
 // flags, and the finishing pair combines the pieces in key order
 // (deterministic).
 //
@@ -52,6 +55,9 @@
 // its abort flag and records a timeout; there is no named barrier, so a role
 // that leaves early never strands another.  The same kernel without the
 // read-out serves the softmax layers that keep a growing KV cache.
+
+#include <algorithm>
+#include <vector>
 
 #include "params.h"
 #include "sm100.cuh"
@@ -100,18 +106,17 @@ enum {
 static_assert(B_COUNT * 8 + 8 <= int(kBarBytes), "barrier area too small");
 
 struct Seg {
-  int bh, blk, j0, j1;
+  int bh, blk, j0, j1, n_contrib;
 };
 
 __device__ __forceinline__ bool next_seg(const AttnParams& p, unsigned& u, unsigned u_end, Seg& s) {
   if (u >= u_end) return false;
-  const unsigned per = unsigned(p.n_blk) * unsigned(p.nkv);
-  s.bh = int(u / per);
-  const unsigned r = u - unsigned(s.bh) * per;
-  s.blk = int(r / unsigned(p.nkv));
-  s.j0 = int(r - unsigned(s.blk) * unsigned(p.nkv));
-  s.j1 = int(min(unsigned(p.nkv), unsigned(s.j0) + (u_end - u)));
-  u += unsigned(s.j1 - s.j0);
+  const uint2 e = p.seg[u++];
+  s.bh = int(e.x & 0x0FFFFFFFu);
+  s.n_contrib = int(e.x >> 28);
+  s.blk = int(e.y & 1023u);
+  s.j0 = int((e.y >> 10) & 2047u);
+  s.j1 = s.j0 + int(e.y >> 21);
   return true;
 }
 
@@ -136,17 +141,6 @@ __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   const bool ok = mbar_wait(bar, parity, w);
   return __all_sync(0xffffffffu, ok);
-}
-
-// Pairs after `pair` whose first segment continues block (bh, blk); every
-// pair's range is non-empty, so they are pairs pair + 1 .. pair + n.  -1 if
-// more than kMaxContrib (the host partition rules that out).
-__device__ __forceinline__ int contributors(const AttnParams& p, int pair, const Seg& s) {
-  const unsigned block_end = (unsigned(s.bh) * unsigned(p.n_blk) + unsigned(s.blk) + 1u) * unsigned(p.nkv);
-  const int pairs = p.grid / 2;
-  int n = 0;
-  while (pair + 1 + n < pairs && p.range[pair + 1 + n] < block_end) ++n;
-  return n <= kMaxContrib ? n : -1;
 }
 
 __device__ __forceinline__ float* slot_of(const AttnParams& p, int cta) {
@@ -365,7 +359,7 @@ __device__ __forceinline__ float2 exp2_poly_pair(float2 x) {
 
 // Of the 16 pairs of each 32-column chunk, this many take the FMA-pipe
 // exponential (pairs 1, 4, 7, ...); the rest take the MUFU.
-constexpr int kPolyPerChunk = 5;
+constexpr int kPolyPerChunk = 3;
 
 // P = 2^(S * scale * log2(e) - m) for 32 columns of a row, packed to bf16
 // pairs; returns their sum.
@@ -518,6 +512,29 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars
 constexpr int kPartStats = 128 * 128;
 constexpr uint32_t kPartQuarter = 8192;
 
+// Acquire the ready flags of this warp's quarter of contributors pair + 1 ..
+// pair + n (bounded spin by lane 0, then every lane acquires).
+__device__ __forceinline__ bool acquire_pieces(const AttnParams& p, int pair, int rank, int quarter, int lane, int n,
+                                               volatile int* abort_flag) {
+  if (lane == 0) {
+    for (int q = 0; q < n && !*abort_flag; ++q) {
+      const unsigned* f = p.ready + (size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter;
+      const uint64_t t0 = global_timer_ns();
+      while (ld_acquire(f) == 0u) {
+        if (*abort_flag || global_timer_ns() - t0 > p.wait_limit_ns) {
+          *abort_flag = 1;
+          record_error(p.err, kDevTimeout);
+          break;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  if (*abort_flag) return false;
+  for (int q = 0; q < n; ++q) (void)ld_acquire(p.ready + (size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter);
+  return true;
+}
+
 // One warpgroup, one query row per thread.  At the end of a segment (its MMAs
 // done, the statistics in shared memory):
 //  * own piece: m, l = l_lo + l_hi, O / l;
@@ -555,12 +572,7 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
     const bool row_ok = qt * 128 + row < p.q_len;
     const bool warp_on = qt * 128 + quarter * 32 < p.q_len;  // warp-uniform
     const bool with_x = writer && use_inter;
-    int n_contrib = 0;
-    if (writer && !full && (n_contrib = contributors(p, pair, s)) < 0) {
-      record_error(p.err, kDevBadShape);  // the host partition rules this out
-      *abort_flag = 1;
-      return false;
-    }
+    const int n_contrib = (writer && !full) ? s.n_contrib : 0;  // the host keeps it <= kMaxContrib
     uint8_t* piece = sQ + ((k + 1) & 1) * kQTile + quarter * kPartQuarter;
     float mk[kMaxContrib], lk[kMaxContrib];
 #pragma unroll
@@ -569,30 +581,16 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
       lk[q] = 0.f;
     }
     if (n_contrib > 0) {
-      if (lane == 0) {
-        for (int q = 0; q < n_contrib && !*abort_flag; ++q) {
-          const unsigned* f = p.ready + (size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter;
-          const uint64_t t0 = global_timer_ns();
-          while (ld_acquire(f) == 0u) {
-            if (*abort_flag || global_timer_ns() - t0 > p.wait_limit_ns) {
-              *abort_flag = 1;
-              record_error(p.err, kDevTimeout);
-              break;
-            }
-          }
-        }
-        // the other Q slot is free once the previous segment's MMAs are done
-        if (!*abort_flag && (k == 0 || mbar_wait(&bars[B_QE + ((k + 1) & 1)], ((k - 1) >> 1) & 1, w))) {
-          fence_async_global();
-          mbar_expect_tx(&bars[B_PQ + quarter], kPartQuarter);
-          bulk_load(piece, reinterpret_cast<const uint8_t*>(slot_of(p, 2 * (pair + 1) + rank)) + quarter * kPartQuarter,
-                    kPartQuarter, &bars[B_PQ + quarter]);
-        }
+      if (!acquire_pieces(p, pair, rank, quarter, lane, n_contrib, abort_flag)) return false;
+      // the other Q slot is free once the previous segment's MMAs are done
+      if (lane == 0 && (k == 0 || mbar_wait(&bars[B_QE + ((k + 1) & 1)], ((k - 1) >> 1) & 1, w))) {
+        fence_async_global();
+        mbar_expect_tx(&bars[B_PQ + quarter], kPartQuarter);
+        bulk_load(piece, reinterpret_cast<const uint8_t*>(slot_of(p, 2 * (pair + 1) + rank)) + quarter * kPartQuarter,
+                  kPartQuarter, &bars[B_PQ + quarter]);
       }
       __syncwarp();
       if (*abort_flag) return false;
-      for (int q = 0; q < n_contrib; ++q)  // every lane acquires what the contributors released
-        (void)ld_acquire(p.ready + (size_t(2 * (pair + 1 + q) + rank)) * 4 + quarter);
 #pragma unroll
       for (int q = 0; q < kMaxContrib; ++q) {
         if (q < n_contrib) {
@@ -654,8 +652,8 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_cluster(eo_leader);
         mbar_arrive(&bars[B_EL]);
+        mbar_arrive_cluster_relaxed(eo_leader);
       }
       slot[kPartStats + row] = M;
       slot[kPartStats + 128 + row] = L;
@@ -679,8 +677,8 @@ __device__ __forceinline__ bool epilogue_role(const AttnParams& p, uint64_t* bar
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive_cluster(eo_leader);
           mbar_arrive(&bars[B_EL]);
+          mbar_arrive_cluster_relaxed(eo_leader);
         }
       }
       float2* v = reinterpret_cast<float2*>(o0);
@@ -758,7 +756,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int cta = blockIdx.x;
   const int rank = int(cluster_ctarank());
   const int pair = cta >> 1;
-  const unsigned u_begin = p.range[pair], u_end = p.range[pair + 1];
+  const unsigned u_begin = p.seg_first[pair], u_end = p.seg_first[pair + 1];
   // The same offset in both CTAs (the launch gives both the same dynamic
   // shared memory); a layout that does not fit is refused by both.
   const bool fits = size_t(smem - smem_raw) + kTilesBytes + kBarBytes + kStatsBytes <= size_t(kSmem);
@@ -886,12 +884,127 @@ int attn_pair_capacity() {
   return n;
 }
 
+// Host partition of the (block, key tile) units over the pairs, as explicit
+// per-pair segment lists.  Two schedules are costed (a segment costs its key
+// tiles plus kSegCost for its start-up, drain and epilogue) and the cheaper
+// makespan is taken:
+//  * stream-K: the unit sequence cut into equal contiguous ranges (a range is
+//    the tail of one block, whole blocks, and the head of another);
+//  * whole blocks first: every pair takes floor(NB / pairs) whole blocks; the
+//    NB % pairs remaining blocks are each cut into k near-equal pieces (k
+//    pairs per block, at most one piece per pair).  A contributing piece is
+//    its pair's first segment, so that it is stored early; the piece holding
+//    key tile 0, which merges the others, is its pair's last.
+// In both, a split block is finished by the pair holding its key tile 0 and
+// continued by the pairs right after it; each pair contributes at most one
+// piece (one scratch slot per CTA).
+namespace {
+constexpr int kSegCost = 2;
+// a finishing segment reads its first piece with one bulk copy issued while
+// its MMAs run, and every further piece with latency-bound loads at the end
+constexpr int kMergeCost = 4;
+
+struct HostSeg {
+  long long bh;
+  int blk, j0, j1, n_contrib;
+};
+
+bool pack_segments(AttnParams& p, const std::vector<std::vector<HostSeg>>& per_pair) {
+  int n = 0;
+  for (size_t c = 0; c < per_pair.size(); ++c) {
+    p.seg_first[c] = unsigned(n);
+    for (const HostSeg& h : per_pair[c]) {
+      if (n >= kAttnMaxSegs || h.bh >= (1LL << 28) || h.blk >= 1024 || h.j0 >= 2048 || h.j1 - h.j0 >= 2048 ||
+          h.j1 <= h.j0 || h.n_contrib > kMaxContrib)
+        return false;
+      p.seg[n].x = unsigned(h.bh) | (unsigned(h.n_contrib) << 28);
+      p.seg[n].y = unsigned(h.blk) | (unsigned(h.j0) << 10) | (unsigned(h.j1 - h.j0) << 21);
+      ++n;
+    }
+  }
+  p.seg_first[per_pair.size()] = unsigned(n);
+  p.n_segs = n;
+  return true;
+}
+
+long long makespan(const std::vector<std::vector<HostSeg>>& per_pair) {
+  long long worst = 0;
+  for (const auto& v : per_pair) {
+    long long c = 0;
+    for (const HostSeg& h : v) c += (h.j1 - h.j0) + kSegCost + kMergeCost * std::max(0, h.n_contrib - 1);
+    worst = std::max(worst, c);
+  }
+  return worst;
+}
+
+// stream-K over `units` with `pairs` contiguous ranges
+std::vector<std::vector<HostSeg>> stream_k(const AttnParams& p, long long units, long long pairs) {
+  std::vector<long long> range(static_cast<size_t>(pairs) + 1);
+  for (long long c = 0; c <= pairs; ++c) range[size_t(c)] = units * c / pairs;
+  std::vector<std::vector<HostSeg>> out(static_cast<size_t>(pairs));
+  for (long long c = 0; c < pairs; ++c) {
+    long long u = range[size_t(c)];
+    while (u < range[size_t(c) + 1]) {
+      const long long blk_lin = u / p.nkv;
+      HostSeg h;
+      h.bh = blk_lin / p.n_blk;
+      h.blk = int(blk_lin % p.n_blk);
+      h.j0 = int(u % p.nkv);
+      h.j1 = int(std::min<long long>(p.nkv, h.j0 + (range[size_t(c) + 1] - u)));
+      h.n_contrib = 0;
+      if (h.j0 == 0 && h.j1 < p.nkv) {  // the pairs after this one that continue the block
+        const long long block_end = (blk_lin + 1) * p.nkv;
+        int n = 0;
+        while (c + 1 + n < pairs && range[size_t(c + 1 + n)] < block_end) ++n;
+        h.n_contrib = n;
+      }
+      out[size_t(c)].push_back(h);
+      u += h.j1 - h.j0;
+    }
+  }
+  return out;
+}
+
+std::vector<std::vector<HostSeg>> blocks_first(const AttnParams& p, long long nb, long long pairs) {
+  std::vector<std::vector<HostSeg>> out(static_cast<size_t>(pairs));
+  const long long full = nb / pairs, rem = nb - full * pairs;
+  long long k = rem > 0 ? std::min<long long>({pairs / rem, kMaxContrib + 1, p.nkv}) : 0;
+  if (rem > 0 && k < 1) k = 1;
+  std::vector<HostSeg> first(static_cast<size_t>(pairs), HostSeg{-1, 0, 0, 0, 0});
+  std::vector<HostSeg> last(static_cast<size_t>(pairs), HostSeg{-1, 0, 0, 0, 0});
+  for (long long r = 0; r < rem; ++r) {
+    const long long blk_lin = full * pairs + r;
+    for (long long q = 0; q < k; ++q) {
+      HostSeg h;
+      h.bh = blk_lin / p.n_blk;
+      h.blk = int(blk_lin % p.n_blk);
+      h.j0 = int(p.nkv * q / k);
+      h.j1 = int(p.nkv * (q + 1) / k);
+      h.n_contrib = q == 0 ? int(k - 1) : 0;
+      const long long c = r * k + q;  // block r's pieces on pairs r k .. r k + k - 1
+      (q == 0 ? last : first)[size_t(c)] = h;
+    }
+  }
+  for (long long c = 0; c < pairs; ++c) {
+    if (first[size_t(c)].bh >= 0) out[size_t(c)].push_back(first[size_t(c)]);
+    for (long long f = 0; f < full; ++f) {
+      const long long blk_lin = c * full + f;
+      out[size_t(c)].push_back(HostSeg{blk_lin / p.n_blk, int(blk_lin % p.n_blk), 0, p.nkv, 0});
+    }
+    if (last[size_t(c)].bh >= 0) out[size_t(c)].push_back(last[size_t(c)]);
+  }
+  return out;
+}
+}  // namespace
+
 bool attn_pair_partition(AttnParams& p, int batch, int max_pairs) {
   p.n_qt = (p.q_len + 127) / 128;
   p.n_blk = (p.n_qt + 1) / 2;
   p.nkv = (p.kv_len + 127) / 128;
+  if (p.n_qt < 1 || p.nkv < 1) return false;
   const long long bh = (long long)batch * p.heads;
-  const long long units = bh * p.n_blk * p.nkv;
+  const long long nb = bh * p.n_blk;
+  const long long units = nb * p.nkv;
   if (units >= (1LL << 31)) return false;
   p.total_units = units;
   // Each pair takes at least an eighth of a block, so a block is split across
@@ -901,8 +1014,12 @@ bool attn_pair_partition(AttnParams& p, int batch, int max_pairs) {
   if (pairs > max_pairs) pairs = max_pairs;
   if (pairs > kAttnMaxGrid / 2) pairs = kAttnMaxGrid / 2;
   if (pairs < 1) return false;
-  p.grid = int(2 * pairs);
-  for (int c = 0; c <= int(pairs); ++c) p.range[c] = unsigned(units * c / pairs);
+  std::vector<std::vector<HostSeg>> a = stream_k(p, units, pairs);
+  std::vector<std::vector<HostSeg>> b = blocks_first(p, nb, pairs);
+  std::vector<std::vector<HostSeg>>& best = makespan(b) < makespan(a) ? b : a;
+  while (!best.empty() && best.back().empty()) best.pop_back();  // pairs left without work
+  if (best.empty() || !pack_segments(p, best)) return false;
+  p.grid = int(2 * best.size());
   return true;
 }
 

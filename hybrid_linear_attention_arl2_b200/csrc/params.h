@@ -12,8 +12,9 @@ namespace arl2 {
 constexpr int kAttnMaxGrid = 192;  // persistent CTAs at most (>= the SM count of a B200)
 
 // Fused intra-frame softmax + inter-frame read-out (attn_pair.cu): a
-// persistent grid of CTA pairs over (256-row block, key tile) units, see the
-// kernel.
+// persistent grid of CTA pairs, each walking its own list of segments (a
+// run of key tiles of one 256-row block), see the kernel.
+constexpr int kAttnMaxSegs = 1024;  // segments of one launch at most
 struct AttnParams {
   int q_len;            // query tokens per stream
   int kv_len;           // valid key/value tokens per stream
@@ -23,7 +24,11 @@ struct AttnParams {
   int nkv;              // key tiles of 128
   long long total_units;   // B * H * n_blk * nkv
   int grid;             // persistent CTAs, even (<= kAttnMaxGrid)
-  unsigned range[kAttnMaxGrid + 1];  // pair c takes units [range[c], range[c + 1])
+  int n_segs;           // entries of seg
+  unsigned seg_first[kAttnMaxGrid / 2 + 1];  // pair c walks seg[seg_first[c] .. seg_first[c + 1])
+  // one segment: x = bh | (contributors << 28) (the pairs after this one whose
+  // pieces a finishing segment merges), y = blk | (j0 << 10) | ((j1 - j0) << 21)
+  uint2 seg[kAttnMaxSegs];
   float scale_log2;     // softmax scale * log2(e)
   uint32_t flags;       // 1: intra only, 2: inter only
   int has_inter;        // 1: add Q MqT^T
@@ -34,9 +39,8 @@ struct AttnParams {
 };
 
 // floats of one CTA's partial slot of the CTA-pair kernel (attn_pair.cu): its
-// 128 x 128 piece of O normalised by its own l, in bf16 (the first 8192
-// floats' bytes, laid out as the kernel describes), then from float 16384
-// m[128] and l[128] in fp32
+// 128 x 128 piece of O normalised by its own l, in bf16 (the first 32 KB, laid
+// out as the kernel describes), then from float 16384 m[128] and l[128] in fp32
 constexpr int kAttnPairSlotFloats = 128 * 128 + 256;
 // ready flags per CTA of the pair kernel (one per epilogue warp)
 constexpr int kAttnPairFlags = 4;

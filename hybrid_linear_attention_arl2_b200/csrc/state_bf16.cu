@@ -68,8 +68,8 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
                : "memory");
   return v;
 }
-__device__ __forceinline__ void st_dsmem_b16(uint32_t cluster_addr, uint16_t v) {
-  asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(cluster_addr), "h"(v) : "memory");
+__device__ __forceinline__ void st_dsmem_v2(uint32_t cluster_addr, uint2 v) {
+  asm volatile("st.shared::cluster.v2.b32 [%0], {%1, %2};" ::"r"(cluster_addr), "r"(v.x), "r"(v.y) : "memory");
 }
 
 // Float offset of 16-byte chunk c (columns 4c..4c+3) of row i of a chunk's
@@ -292,7 +292,7 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
       tma_load_3d(sP, &tm_phiq, &bars[P_PQ], 0, 0, h);
       tma_load_3d(sP + kHalfB, &tm_phiq, &bars[P_PQ], 64, 0, h);
     }
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     // This rank's rows of S_N: sum the chunks' partials in chunk order (rank
     // q holds chunk q), then S_N = alpha S_{N-1} + c * sum.
     const int rpc = (128 + nrank - 1) / nrank;
@@ -300,42 +300,77 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     const int nchunks16 = max(0, i1 - i0) * 32;  // 16-byte chunks of this rank's rows
     const uint32_t part_base = smem_u32(sK);
     const float a = p.alpha[slab];
-    for (int q16 = threadIdx.x; ok_all && q16 < nchunks16; q16 += kStateThreads) {
-      {
-        const int i = i0 + q16 / 32, c = q16 % 32;
-        const uint32_t off = part_base + part_off(i, c) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < nrank; ++q) {
-          const float4 v = ld_dsmem_f4(cluster_map(off, uint32_t(q)));
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
+    // Every rank's value of a chunk is loaded before any is added, so the
+    // remote loads overlap, and the sum still runs in chunk order.  A thread's
+    // first kMaxPer chunks (all of them from 9 ranks up) have their S_{N-1}
+    // loaded while the other ranks finish their partials, and keep their bf16
+    // values for the copy to rank 0; further ones are read from global memory.
+    constexpr int kMaxPer = 3;
+    uint2 keep[kMaxPer];
+    float4 prev[kMaxPer];
+#pragma unroll
+    for (int t = 0; t < kMaxPer; ++t) {
+      const int q16 = threadIdx.x + t * kStateThreads;
+      prev[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ok_all && q16 < nchunks16)
+        prev[t] = *reinterpret_cast<const float4*>(p.S_prev + size_t(slab) * 16384 + size_t(i0 + q16 / 32) * 128 +
+                                                   (q16 % 32) * 4);
+    }
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    for (int q16 = threadIdx.x, t = 0; ok_all && q16 < nchunks16; q16 += kStateThreads, ++t) {
+      const int i = i0 + q16 / 32, c = q16 % 32;
+      const uint32_t off = part_base + part_off(i, c) * 4;
+      float4 v[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q < nrank) v[q] = ld_dsmem_f4(cluster_map(off, uint32_t(q)));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        if (q < nrank) {
+          acc.x += v[q].x;
+          acc.y += v[q].y;
+          acc.z += v[q].z;
+          acc.w += v[q].w;
         }
-        const size_t e = size_t(slab) * 16384 + size_t(i) * 128 + c * 4;
-        const float4 sp4 = *reinterpret_cast<const float4*>(p.S_prev + e);
-        float4 r;
-        r.x = fmaf(a, sp4.x, p.corr * acc.x);
-        r.y = fmaf(a, sp4.y, p.corr * acc.y);
-        r.z = fmaf(a, sp4.z, p.corr * acc.z);
-        r.w = fmaf(a, sp4.w, p.corr * acc.w);
-        *reinterpret_cast<float4*>(p.S_next + e) = r;
-        const uint2 bf = make_uint2(pack_bf16x2(r.x, r.y), pack_bf16x2(r.z, r.w));
-        *reinterpret_cast<uint2*>(p.S_next_bf + e) = bf;
       }
+      const size_t e = size_t(slab) * 16384 + size_t(i) * 128 + c * 4;
+      float4 sp4;
+      if (t < kMaxPer) {
+#pragma unroll
+        for (int x = 0; x < kMaxPer; ++x)
+          if (x == t) sp4 = prev[x];
+      } else {
+        sp4 = *reinterpret_cast<const float4*>(p.S_prev + e);
+      }
+      float4 r;
+      r.x = fmaf(a, sp4.x, p.corr * acc.x);
+      r.y = fmaf(a, sp4.y, p.corr * acc.y);
+      r.z = fmaf(a, sp4.z, p.corr * acc.z);
+      r.w = fmaf(a, sp4.w, p.corr * acc.w);
+      *reinterpret_cast<float4*>(p.S_next + e) = r;
+      const uint2 bf = make_uint2(pack_bf16x2(r.x, r.y), pack_bf16x2(r.z, r.w));
+      *reinterpret_cast<uint2*>(p.S_next_bf + e) = bf;
+#pragma unroll
+      for (int x = 0; x < kMaxPer; ++x)
+        if (x == t) keep[x] = bf;
     }
     // every partial is read: rank 0's K/V tiles take the bf16 S_N for the
     // read-out MMA (row k = state row, 64-column boxes, 128-byte swizzle: the
-    // layout the tensor cores read as an MN-major operand)
+    // layout the tensor cores read as an MN-major operand); columns 4c..4c+3
+    // of a row are 8 contiguous bytes of that layout
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    // (each thread re-reads the bf16 values it wrote itself)
-    for (int q16 = threadIdx.x; ok_all && q16 < nchunks16; q16 += kStateThreads) {
+    for (int q16 = threadIdx.x, t = 0; ok_all && q16 < nchunks16; q16 += kStateThreads, ++t) {
       const int i = i0 + q16 / 32, c = q16 % 32;
-      const uint2 bf = *reinterpret_cast<const uint2*>(p.S_next_bf + size_t(slab) * 16384 + size_t(i) * 128 + c * 4);
-      const uint16_t v4[4] = {uint16_t(bf.x & 0xFFFFu), uint16_t(bf.x >> 16), uint16_t(bf.y & 0xFFFFu),
-                              uint16_t(bf.y >> 16)};
+      uint2 bf = make_uint2(0u, 0u);
+      if (t < kMaxPer) {
 #pragma unroll
-      for (int x = 0; x < 4; ++x) st_dsmem_b16(cluster_map(smem_u32(sK) + sw128_offset(i, 4 * c + x), 0u), v4[x]);
+        for (int x = 0; x < kMaxPer; ++x)
+          if (x == t) bf = keep[x];
+      } else {
+        bf = *reinterpret_cast<const uint2*>(p.S_next_bf + size_t(slab) * 16384 + size_t(i) * 128 + c * 4);
+      }
+      st_dsmem_v2(cluster_map(smem_u32(sK) + sw128_offset(i, 4 * c), 0u), bf);
     }
     asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");

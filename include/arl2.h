@@ -245,6 +245,23 @@ arl2_status arl2_block_destroy(arl2_block_t blk);
 arl2_status arl2_gemm_bf16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c, int64_t ldc, int64_t m,
                            int64_t n, int64_t k, void* stream);
 
+/* Diagnostic, host only (no device is touched): the work partition the
+ * attention kernel uses for `batch` streams of `heads` heads with q_len query
+ * rows and kv_len keys on `pairs` CTA pairs.  The (stream, head) slabs are cut
+ * into blocks of 256 query rows, each block into key tiles of 128; every pair
+ * walks its own list of segments (a run [j0, j1) of key tiles of one block).
+ * A block split across pairs is finished by the pair holding key tile 0, which
+ * merges the pieces of the n_contrib pairs right after it.  On return
+ * *n_pairs is the pairs used (<= pairs), *n_segs the segments, seg_first
+ * [*n_pairs + 1] the offsets of each pair's list and segs [*n_segs][5] the
+ * segments as (slab = stream * heads + head, block, j0, j1, n_contrib).
+ * segs must hold max_segs segments, seg_first 97 entries.
+ * Errors: INVALID_ARGUMENT (null pointers, sizes < 1, pairs > 96),
+ * UNSUPPORTED (the problem does not fit the partition's encoding or more than
+ * max_segs segments). */
+arl2_status arl2_attn_partition(int batch, int heads, int q_len, int kv_len, int pairs, int32_t* segs, int max_segs,
+                                int32_t* seg_first, int* n_segs, int* n_pairs);
+
 /* ---- State write without allocation ---------------------------------------
  * The paper has no counterpart to this call; it is a deployment aid.  Some
  * callers cannot call cudaMalloc: code that runs while a CUDA graph is being
