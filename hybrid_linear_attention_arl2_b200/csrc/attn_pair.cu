@@ -378,10 +378,6 @@ __device__ __forceinline__ float exp_chunk(const uint32_t* r, const float2 sc, c
   return sa.x + sa.y;
 }
 
-__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
 __device__ __forceinline__ void softmax_role(const AttnParams& p, uint64_t* bars, float* stats, float* mchain,
                                              const uint32_t tmem, const int rank, const int wgi, const int quarter,
                                              const int lane, const unsigned u_begin, const unsigned u_end,

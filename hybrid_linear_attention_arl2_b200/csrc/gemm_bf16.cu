@@ -3,14 +3,18 @@
 //
 //   C[M][N] = A[M][K] B[K][N]      (all row-major; A = token rows, B = weights)
 //
-// A persistent grid of one CTA per SM walks 128 x 256 output tiles.  Per tile
-// the producer streams K-slices of 64 through a 4-stage TMA ring (A: 128 rows
-// x 64, K-major; B: 64 rows x 256 columns, read as an MN-major operand), one
-// thread issues tcgen05.mma 128 x 256 x 16 (the shape that keeps the tensor
-// core at its full rate) into one of two tensor-memory accumulators, and the
-// epilogue warpgroup drains the other accumulator -- bf16 conversion, 64-column
-// chunks staged in shared memory, TMA tile stores (rows and columns past M and
-// N are clipped by the tensor map) -- while the next tile accumulates.
+// Persistent clusters of two CTAs (one per SM of a pair) walk 256 x 256
+// output tiles with tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16: the
+// shape that keeps the tensor cores at their full rate).  Per tile each CTA
+// streams K-slices of 64 through a 6-stage TMA ring: its own 128 rows of A
+// (K-major) and its own 128 of the 256 columns of B (read as an MN-major
+// operand), so that a CTA reads a third less from L2 per output than a
+// single-SM 128 x 256 tile.  Rank 0's thread issues the MMAs into one of two
+// tensor-memory accumulators (256 columns each; every CTA holds its 128 rows);
+// each CTA's epilogue warpgroup drains the other accumulator -- bf16
+// conversion, 64-column chunks staged in shared memory, TMA tile stores (rows
+// and columns past M and N are clipped by the tensor map) -- while the next
+// tile accumulates.  No load uses cluster multicast.
 
 #include <cudaTypedefs.h>
 
@@ -22,14 +26,15 @@ namespace arl2 {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kStages = 4;
-constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kStages = 6;
+constexpr int kBM = 128, kBN = 128, kBK = 64;  // per CTA: its rows of A, its half of the pair's 256 columns
 constexpr uint32_t kABytes = kBM * kBK * 2;   // 16 KB
-constexpr uint32_t kBBytes = kBK * kBN * 2;   // 32 KB: four 64-column boxes of 64 rows
+constexpr uint32_t kBBytes = kBK * kBN * 2;   // 16 KB: two 64-column boxes of 64 rows
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kStageOut = 2 * 4096;      // per epilogue warp: two 32-row x 64-column boxes
 constexpr uint32_t kTiles = kStages * kStageBytes + 4 * kStageOut;
 constexpr int kSmem = int(kTiles) + 256 + 1024;
+static_assert(kSmem <= 232448, "shared memory layout too large");
 
 enum { G_FULL = 0, G_EMPTY = kStages, G_AF = 2 * kStages, G_AE = G_AF + 2, G_DRAIN = G_AE + 2, G_COUNT };
 
@@ -38,11 +43,14 @@ __device__ __forceinline__ bool warp_wait_g(uint64_t* bar, uint32_t parity, cons
   return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+// 2-D tile load into this CTA's shared memory whose bytes count on the pair
+// leader's mbarrier at the same offset.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  const uint32_t leader_bar = cluster_map(smem_u32(bar), 0);
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
       "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1)
       : "memory");
 }
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
@@ -52,7 +60,7 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                  const __grid_constant__ CUtensorMap tm_c, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -62,53 +70,56 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + G_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = int(cluster_ctarank());
+  const int pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
+  // the same offset in both CTAs (both launch with the same dynamic shared memory)
   const bool fits = size_t(smem - smem_raw) + kTiles + 256 <= size_t(kSmem);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < G_COUNT; ++i) mbar_init(&bars[i], (i == G_AE || i == G_AE + 1) ? 4u : 1u);
+    for (int i = 0; i < G_COUNT; ++i) mbar_init(&bars[i], (i == G_AE || i == G_AE + 1) ? 8u : 1u);
     *abort_flag = fits ? 0 : 1;
     if (!fits) record_error(p.err, kDevBadShape);
     fence_barrier_init();
   }
-  if (warp == 2) tmem_alloc(tmem_holder, 512);
+  if (warp == 2) tmem_alloc_pair(tmem_holder, 512);
   tc_fence_before();
   __syncthreads();
+  cluster_barrier();  // both CTAs' barriers initialised before any remote arrive or load
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const WaitCtl w{abort_flag, p.err, p.wait_limit_ns};
-  const int tiles_m = (p.M + kBM - 1) / kBM, tiles_n = (p.N + kBN - 1) / kBN;
+  const int tiles_m = (p.M + 2 * kBM - 1) / (2 * kBM), tiles_n = (p.N + 2 * kBN - 1) / (2 * kBN);
   const int n_tiles = tiles_m * tiles_n;
   const int nk = (p.K + kBK - 1) / kBK;
 
   if (!*abort_flag) {
-    if (warp == 0 && lane == 0) {  // ---------------------------------------- producer
+    if (warp == 0 && lane == 0) {  // ---------------------------------------- producer (both CTAs)
       tma_prefetch(&tm_a);
       tma_prefetch(&tm_b);
       uint32_t it = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-        const int m0 = (t % tiles_m) * kBM, n0 = (t / tiles_m) * kBN;
+      for (int t = pair; t < n_tiles; t += pairs) {
+        const int m0 = (t % tiles_m) * 2 * kBM + rank * kBM, n0 = (t / tiles_m) * 2 * kBN + rank * kBN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t s = it % kStages;
           if (it >= kStages && !mbar_wait(&bars[G_EMPTY + s], ((it / kStages) - 1) & 1, w)) break;
           uint8_t* dst = smem + s * kStageBytes;
-          mbar_expect_tx(&bars[G_FULL + s], kStageBytes);
-          tma_load_2d(dst, &tm_a, &bars[G_FULL + s], kb * kBK, m0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            tma_load_2d(dst + kABytes + q * (kBBytes / 4), &tm_b, &bars[G_FULL + s], n0 + 64 * q, kb * kBK);
+          if (rank == 0) mbar_expect_tx(&bars[G_FULL + s], 2 * kStageBytes);
+          tma_load_2d_pair(dst, &tm_a, &bars[G_FULL + s], kb * kBK, m0);
+          tma_load_2d_pair(dst + kABytes, &tm_b, &bars[G_FULL + s], n0, kb * kBK);
+          tma_load_2d_pair(dst + kABytes + kBBytes / 2, &tm_b, &bars[G_FULL + s], n0 + 64, kb * kBK);
         }
         if (*abort_flag) break;
       }
-    } else if (warp == 1 && lane == 0) {  // ---------------------------------- MMA issuer
-      const uint32_t id = idesc_bf16(kBM, kBN, 0, 1);
+    } else if (warp == 1 && lane == 0 && rank == 0) {  // -------------------- MMA issuer (rank 0)
+      const uint32_t id = idesc_bf16(2 * kBM, 2 * kBN, 0, 1);
       const uint32_t base = smem_u32(smem);
-      const uint64_t da64 = smem_desc_sw128(base, 16, 1024);            // A: K-major, 128-byte rows
-      const uint64_t db64 = smem_desc_sw128(base + kABytes, kBBytes / 4, 1024);  // B: MN-major, 64-column chunks 8 KB apart
+      const uint64_t da64 = smem_desc_sw128(base, 16, 1024);                     // A: K-major, 128-byte rows
+      const uint64_t db64 = smem_desc_sw128(base + kABytes, kBBytes / 2, 1024);  // B: MN-major, 64-column boxes 8 KB apart
       const uint32_t hi = uint32_t(da64 >> 32);
       const uint32_t da0 = uint32_t(da64), db0 = uint32_t(db64);
       uint32_t it = 0, tc = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
+      for (int t = pair; t < n_tiles; t += pairs, ++tc) {
         const uint32_t acc = tc & 1;
-        // the epilogue has drained this accumulator (two tiles ago)
+        // both CTAs' epilogues have drained this accumulator (two tiles ago)
         if (tc >= 2 && !mbar_wait(&bars[G_AE + acc], ((tc >> 1) - 1) & 1, w)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * 256;
@@ -119,29 +130,24 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
             ok = false;
             break;
           }
+          tc_fence_after();
           const uint32_t so = (s * kStageBytes) >> 4;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-                "setp.ne.b32 p, %5, 0;\n\t"
-                "mov.b64 da, {%1, %3};\n\t"
-                "mov.b64 db, {%2, %3};\n\t"
-                "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d),
-                "r"(da0 + so + kk * 2), "r"(db0 + so + kk * 128), "r"(hi), "r"(id), "r"(uint32_t(kb > 0 || kk > 0)));
-          }
-          mma_commit(&bars[G_EMPTY + s]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_pair_ss(d, da0 + so + kk * 2, db0 + so + kk * 128, hi, id, uint32_t(kb > 0 || kk > 0));
+          mma_commit_pair(&bars[G_EMPTY + s]);
         }
         if (!ok) break;
-        mma_commit(&bars[G_AF + acc]);
+        mma_commit_pair(&bars[G_AF + acc]);
       }
-    } else if (warp >= 4) {  // ------------------------------------------------ epilogue
+    } else if (warp >= 4) {  // ------------------------------------------------ epilogue (both CTAs)
       const int quarter = warp & 3;
       const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+      const uint32_t ae_leader = cluster_map(smem_u32(&bars[G_AE]), 0);
       uint8_t* wst = sOut + quarter * kStageOut;
       uint32_t tc = 0, stores = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
-        const int m0 = (t % tiles_m) * kBM, n0 = (t / tiles_m) * kBN;
+      for (int t = pair; t < n_tiles; t += pairs, ++tc) {
+        const int m0 = (t % tiles_m) * 2 * kBM + rank * kBM, n0 = (t / tiles_m) * 2 * kBN;
         const uint32_t acc = tc & 1;
         if (!warp_wait_g(&bars[G_AF + acc], (tc >> 1) & 1, w)) break;
         tc_fence_after();
@@ -156,7 +162,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
           if (q == 3) {  // the accumulator is read: the MMA may reuse it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[G_AE + acc]);
+            if (lane == 0) mbar_arrive_cluster_relaxed(ae_leader + acc * 8);
           }
           uint8_t* box = wst + (stores & 1) * 4096;
           if (lane == 0 && stores >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
@@ -172,9 +178,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
           }
           fence_async_smem();
           __syncwarp();
-          if (lane == 0 && warp_on && n0 + 64 * q < p.N) {
-            tma_store_2d(&tm_c, box, n0 + 64 * q, m0 + quarter * 32);
-          }
+          if (lane == 0 && warp_on && n0 + 64 * q < p.N) tma_store_2d(&tm_c, box, n0 + 64 * q, m0 + quarter * 32);
           if (lane == 0) bulk_commit();
           ++stores;
         }
@@ -186,8 +190,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   // ------------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 1 && lane == 0) {  // every MMA completed before tensor memory is released
-    mma_commit(&bars[G_DRAIN]);
+  if (warp == 1 && lane == 0 && rank == 0) {  // every MMA completed before tensor memory is released
+    mma_commit_pair(&bars[G_DRAIN]);
+  }
+  if (warp == 1 && lane == 0) {  // both CTAs see the drain commit (multicast)
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(&bars[G_DRAIN], 0) && global_timer_ns() - t0 < 10000000ull) {
     }
@@ -198,9 +204,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     }
   }
   __syncthreads();
+  cluster_barrier();  // neither CTA leaves while the other may still signal it
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -251,9 +258,22 @@ cudaError_t gemm_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, vo
   static unsigned done = 0;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_bf16_kernel), kSmem, &done);
   if (e != cudaSuccess) return e;
-  const int tiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
-  const int grid = tiles < sms ? tiles : sms;
-  gemm_bf16_kernel<<<grid, kThreads, kSmem, stream>>>(ta, tb, tc, p);
+  const int tiles = ((p.M + 2 * kBM - 1) / (2 * kBM)) * ((p.N + 2 * kBN - 1) / (2 * kBN));
+  cudaLaunchConfig_t cfg{};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = size_t(kSmem);
+  cfg.stream = stream;
+  // clusters of two resident at once
+  int cap = 0;
+  cfg.gridDim = dim3(2);
+  e = cudaOccupancyMaxActiveClusters(&cap, gemm_bf16_kernel, &cfg);
+  if (e != cudaSuccess) return e;
+  if (cap < 1) return cudaErrorInvalidConfiguration;
+  (void)sms;
+  const int pairs = tiles < cap ? tiles : cap;
+  cfg.gridDim = dim3(2 * pairs);
+  e = cudaLaunchKernelEx(&cfg, gemm_bf16_kernel, ta, tb, tc, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
