@@ -731,7 +731,7 @@ def cpu_oracle_rate(cfg: W.Config, budget_s: float = 12.0, sample_note=True):
 # launch on the single-hybrid-layer-bf16 workload, from one ncu capture of
 # `bench.py --profile-small --no-graphs`; reported only while the kernel sources
 # hash to the value the capture was taken on (None: not captured yet).
-ATTN_TRAFFIC = {"bytes": None, "sources_sha256": None,
+ATTN_TRAFFIC = {"bytes": 14850560 + 0, "sources_sha256": "edf16c75f7da6b30cb4bd7463f020160af76084df75c92f63af910b150eeb000",
                 "capture": "profiles/attn_pair_kernel_single-hybrid-layer-bf16.md"}
 ATTN_SOURCES = ("hybrid_linear_attention_arl2_b200/csrc/attn_pair.cu",
                 "hybrid_linear_attention_arl2_b200/csrc/sm100.cuh",
