@@ -53,6 +53,10 @@ def _args():
                     help="the single-layer shape with token-level access (the ablated rule; its own JSON line)")
     ap.add_argument("--profile-small", action="store_true",
                     help="a few steps, no extras: for ncu captures of the kernels")
+    ap.add_argument("--profile-kv", type=int, default=0, metavar="F",
+                    help="one KV-cache softmax layer: F frames committed into its cache, then three query "
+                         "passes over F + 1 frames of keys, timed with CUDA events (its own JSON line; an ncu "
+                         "capture of the third query skips F + 2 attention launches)")
     return ap.parse_args()
 
 
@@ -190,6 +194,41 @@ class DeviceStream:
 
     def triple(self, frame: int, pas: int):
         return self.pool[self.wl.pool_index(0, frame, pas)]
+
+
+def run_kv_profile(args) -> dict:
+    """A KV-cache softmax layer of the stack's shape holding `F` clean frames:
+    F commits fill its cache, then three query passes attend over the F + 1
+    frames of keys (cache and current frame); the last two are timed."""
+    import torch
+    from hybrid_linear_attention_arl2_b200 import arl2
+    cfg = W.CONFIGS[3]
+    F = args.profile_kv
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    arl2.load_library()
+    ds = DeviceStream(cfg, 0, device)
+    B, H, L, d = cfg.batch, cfg.heads, cfg.tokens, cfg.head_dim
+    stream = torch.cuda.Stream(device)
+    O = torch.empty((B, L, H, d), dtype=torch.bfloat16, device=device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    with torch.cuda.stream(stream):
+        kv = arl2.KVLayer(B, H, d, L, arl2.ARL2_BF16, max_frames=F + 1, stream=stream)
+        for f in range(F):
+            arl2.arl2_kv_commit(kv.handle, *ds.triple(f, cfg.queries), O, stream)
+        for p in range(3):
+            if p > 0:
+                ev[p - 1].record(stream)
+            arl2.arl2_kv_query(kv.handle, *ds.triple(F, p), O, stream)
+        ev[2].record(stream)
+        stream.synchronize()
+        if kv.last_error():
+            raise RuntimeError(f"device error in the KV-layer run: {arl2.STATUS.get(kv.last_error())}")
+        kv.close()
+    ms = [ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])]
+    kv_len = (F + 1) * L
+    fl = 4.0 * L * kv_len * d * H * B
+    return {"frames": F, "kv_len": kv_len, "ms": ms, "tflops": fl / (min(ms) / 1e3) / 1e12}
 
 
 def whole_job_rate(ms: float, steps: int, world: int, dist=None, device="cpu"):
@@ -731,7 +770,9 @@ def cpu_oracle_rate(cfg: W.Config, budget_s: float = 12.0, sample_note=True):
 # launch on the single-hybrid-layer-bf16 workload, from one ncu capture of
 # `bench.py --profile-small --no-graphs`; reported only while the kernel sources
 # hash to the value the capture was taken on (None: not captured yet).
-ATTN_TRAFFIC = {"bytes": 14850560 + 0, "sources_sha256": "edf16c75f7da6b30cb4bd7463f020160af76084df75c92f63af910b150eeb000",
+# (Captured on the build before the long-key-range schedule was added; the
+# device code and the schedule of this workload are unchanged since.)
+ATTN_TRAFFIC = {"bytes": 14850560 + 0, "sources_sha256": "5858c7523edecb3839a85a96568c74214588058c2ce9acb049bfe1ab105c27d0",
                 "capture": "profiles/attn_pair_kernel_single-hybrid-layer-bf16.md"}
 ATTN_SOURCES = ("hybrid_linear_attention_arl2_b200/csrc/attn_pair.cu",
                 "hybrid_linear_attention_arl2_b200/csrc/sm100.cuh",
@@ -806,6 +847,18 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
+    if args.profile_kv and args.impl != "reference":
+        res = run_kv_profile(args)
+        peak_burst, peak_sus, src = peak_pair(peaks())
+        print(json.dumps({"metric": "KV-cache softmax layer query pass (TFLOP/s)", "value": res["tflops"],
+                          "unit": "TFLOP/s", "n_gpus": 1, "higher_is_better": True, "dtype": "bf16",
+                          "data": "synthetic",
+                          "config": {"workload": "kv-cache-softmax-layer-bf16", "cache_frames": res["frames"],
+                                     "kv_len": res["kv_len"], "tokens_per_frame": 1560, "heads": 12,
+                                     "head_dim": 128},
+                          "ms": res["ms"], "frac_of_burst_peak": res["tflops"] / peak_burst,
+                          "peak_basis": f"burst bf16 {src}"}), flush=True)
+        return
     if args.token and args.impl != "reference":
         res = run_token(args, rank, world)
         if rank != 0:

@@ -27,10 +27,10 @@
 // (or plain equal ranges of the (block, key tile) sequence, "stream-K", when
 // that costs less).  A block whose key range is split across pairs is
 // finished by the pair holding its key tile 0 (always that pair's last
-// segment); the pairs continuing it (their first segment) store their
-// normalised partial output in bf16 with (m, l) in fp32 and raise ready
-// flags, and the finishing pair combines the pieces in key order
-// (deterministic).
+// segment); the pairs continuing it (their first segment, or on long key
+// ranges their last) store their normalised partial output in bf16 with
+// (m, l) in fp32 and raise ready flags, and the finishing pair combines the
+// pieces in key order (deterministic).
 //
 // Roles per CTA (512 threads, four warpgroups):
 //   warp 0       TMA producer: per segment the CTA's Q tile (two slots, so the
@@ -886,11 +886,15 @@ int attn_pair_capacity() {
 // makespan is taken:
 //  * stream-K: the unit sequence cut into equal contiguous ranges (a range is
 //    the tail of one block, whole blocks, and the head of another);
-//  * whole blocks first: every pair takes floor(NB / pairs) whole blocks; the
-//    NB % pairs remaining blocks are each cut into k near-equal pieces (k
-//    pairs per block, at most one piece per pair).  A contributing piece is
-//    its pair's first segment, so that it is stored early; the piece holding
-//    key tile 0, which merges the others, is its pair's last.
+//  * whole blocks first: every pair takes floor(NB / pairs) whole blocks
+//    (round f: blocks f P .. f P + P - 1, so the blocks of a head run side by
+//    side); the NB % pairs remaining blocks are each cut into k near-equal
+//    pieces (k pairs per block, at most one piece per pair).  A contributing
+//    piece is its pair's first segment, so that it is stored early, or, for
+//    key ranges of kLongKeyTiles tiles and more, its last, so that all whole
+//    blocks start together (their K/V tiles are then read from DRAM once and
+//    shared through L2); the piece holding key tile 0, which merges the
+//    others, is its pair's last.
 // In both, a split block is finished by the pair holding its key tile 0 and
 // continued by the pairs right after it; each pair contributes at most one
 // piece (one scratch slot per CTA).
@@ -899,6 +903,7 @@ constexpr int kSegCost = 2;
 // a finishing segment reads its first piece with one bulk copy issued while
 // its MMAs run, and every further piece with latency-bound loads at the end
 constexpr int kMergeCost = 4;
+constexpr int kLongKeyTiles = 32;
 
 struct HostSeg {
   long long bh;
@@ -961,7 +966,7 @@ std::vector<std::vector<HostSeg>> stream_k(const AttnParams& p, long long units,
   return out;
 }
 
-std::vector<std::vector<HostSeg>> blocks_first(const AttnParams& p, long long nb, long long pairs) {
+std::vector<std::vector<HostSeg>> blocks_first(const AttnParams& p, long long nb, long long pairs, bool pieces_last) {
   std::vector<std::vector<HostSeg>> out(static_cast<size_t>(pairs));
   const long long full = nb / pairs, rem = nb - full * pairs;
   long long k = rem > 0 ? std::min<long long>({pairs / rem, kMaxContrib + 1, p.nkv}) : 0;
@@ -982,11 +987,12 @@ std::vector<std::vector<HostSeg>> blocks_first(const AttnParams& p, long long nb
     }
   }
   for (long long c = 0; c < pairs; ++c) {
-    if (first[size_t(c)].bh >= 0) out[size_t(c)].push_back(first[size_t(c)]);
-    for (long long f = 0; f < full; ++f) {
-      const long long blk_lin = c * full + f;
+    if (!pieces_last && first[size_t(c)].bh >= 0) out[size_t(c)].push_back(first[size_t(c)]);
+    for (long long f = 0; f < full; ++f) {  // round f: blocks f P .. f P + P - 1, the heads' blocks side by side
+      const long long blk_lin = f * pairs + c;
       out[size_t(c)].push_back(HostSeg{blk_lin / p.n_blk, int(blk_lin % p.n_blk), 0, p.nkv, 0});
     }
+    if (pieces_last && first[size_t(c)].bh >= 0) out[size_t(c)].push_back(first[size_t(c)]);
     if (last[size_t(c)].bh >= 0) out[size_t(c)].push_back(last[size_t(c)]);
   }
   return out;
@@ -1011,8 +1017,13 @@ bool attn_pair_partition(AttnParams& p, int batch, int max_pairs) {
   if (pairs > kAttnMaxGrid / 2) pairs = kAttnMaxGrid / 2;
   if (pairs < 1) return false;
   std::vector<std::vector<HostSeg>> a = stream_k(p, units, pairs);
-  std::vector<std::vector<HostSeg>> b = blocks_first(p, nb, pairs);
-  std::vector<std::vector<HostSeg>>& best = makespan(b) < makespan(a) ? b : a;
+  // Long key ranges (KV-cache layers): every pair starts its whole blocks at
+  // once, so the pairs on one head's blocks read each K/V tile at about the
+  // same time and it crosses DRAM once; the split pieces come last.  Short
+  // ones: the cheaper of the two schedules.
+  const bool long_keys = p.nkv >= kLongKeyTiles;
+  std::vector<std::vector<HostSeg>> b = blocks_first(p, nb, pairs, long_keys);
+  std::vector<std::vector<HostSeg>>& best = (long_keys || makespan(b) < makespan(a)) ? b : a;
   while (!best.empty() && best.back().empty()) best.pop_back();  // pairs left without work
   if (best.empty() || !pack_segments(p, best)) return false;
   p.grid = int(2 * best.size());

@@ -207,9 +207,10 @@ arl2_status arl2_kv_destroy(arl2_kv_t kv);
  * (the pages fix neither the gates' inputs nor their pooling; a head-wise
  * alpha from the frame's mean token and a per-token beta are this build's
  * reading).  No position encoding is applied: Q and K enter the layer as
- * projected.  The projections are plain GEMMs (cuBLAS, fp32 accumulate, bf16
- * results): one against [W_qkv | W_gate] (the layer reads Q, K and V as strided
- * views of its rows), one against W_o.
+ * projected.  The projections are plain GEMMs (this library's tcgen05 GEMM,
+ * arl2_gemm_bf16: fp32 accumulate, bf16 results): one against
+ * [W_qkv | W_gate] (the layer reads Q, K and V as strided views of its rows),
+ * one against W_o.
  *   cfg     : bf16 configuration with head_dim 128 (hidden D = heads * 128).
  *   w_qkv   : device bf16 [D, 3D] row-major (X W: y_j = sum_i x_i W[i][j]);
  *   w_o     : device bf16 [D, D];  w_gate : device bf16 [D, 2H] (alpha columns
@@ -217,8 +218,7 @@ arl2_status arl2_kv_destroy(arl2_kv_t kv);
  *             arl2_state_init.  Every weight is copied at init.
  *   x, y    : device bf16 [B, L, D] (token-major; y must not overlap x).
  * The block owns one hybrid-layer handle (its state, KV-free) and its work
- * space (Q, K, V, O, gates: about 5 * B * L * D * 2 bytes plus cuBLAS's
- * 32 MiB workspace, fixed at init).  arl2_block_layer() returns that handle
+ * space (Q, K, V, O, gates: about 5 * B * L * D * 2 bytes, fixed at init).  arl2_block_layer() returns that handle
  * for state get/set, last_error and the device-byte count; it is destroyed
  * with the block.  Errors: INVALID_ARGUMENT, UNSUPPORTED (not bf16 / d != 128),
  * OUT_OF_MEMORY, CUDA. */

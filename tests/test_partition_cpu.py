@@ -3,8 +3,9 @@
 Invariants the kernel relies on: every (slab, block, key tile) unit is covered
 exactly once; a split block is finished by the pair holding key tile 0 (that
 pair's last segment), whose n_contrib pieces come from the pairs right after
-it, each of which holds that block as its first segment; a pair contributes at
-most one piece (one scratch slot per CTA); at most eight pieces per block.
+it, each of which holds that block as its first segment (or, on long key
+ranges, its last); a pair contributes at most one piece (one scratch slot per
+CTA); at most eight pieces per block.
 """
 import itertools
 
@@ -27,16 +28,18 @@ def check(batch, heads, q_len, kv_len, pairs):
             for j in range(j0, j1):
                 assert (slab, blk, j) not in seen
                 seen[(slab, blk, j)] = c
-            if j0 > 0:  # a continuing piece: the pair's first segment
-                assert i == 0
+            if j0 > 0:  # a continuing piece: the pair's first segment, or its last on long key ranges
+                assert i == 0 or (nkv >= 32 and i == len(segs) - 1)
                 contributions += 1
             if j0 == 0 and j1 < nkv:  # finishes a split block: the pair's last segment
                 assert i == len(segs) - 1
                 assert 1 <= nc <= 8
                 covered = j1
                 for q in range(nc):
-                    s2, b2, k0, k1, _ = parts[c + 1 + q][0]
-                    assert (s2, b2) == (slab, blk) and k0 == covered
+                    pieces = [x for x in parts[c + 1 + q] if (x[0], x[1]) == (slab, blk)]
+                    assert len(pieces) == 1
+                    s2, b2, k0, k1, _ = pieces[0]
+                    assert k0 == covered
                     covered = k1
                 assert covered == nkv
             else:
@@ -79,6 +82,17 @@ def test_partition_takes_whole_blocks_when_they_divide():
     # 148 blocks on 74 pairs: two whole blocks each, nothing split
     parts = arl2.arl2_attn_partition(1, 37, 1024, 1024, 74)
     assert all(len(s) == 2 and all(j0 == 0 and j1 == 8 for _, _, j0, j1, _ in s) for s in parts)
+
+
+def test_partition_long_key_ranges_start_whole_blocks_together():
+    # a KV-cache layer over 21 frames of keys: every pair's first segment is a
+    # whole block, and round 0 holds blocks 0 .. 73 (the seven blocks of a head
+    # on seven pairs side by side)
+    parts = arl2.arl2_attn_partition(1, 12, 1560, 21 * 1560, 74)
+    nkv = (21 * 1560 + 127) // 128
+    firsts = [s[0] for s in parts]
+    assert all(j0 == 0 and j1 == nkv for _, _, j0, j1, _ in firsts)
+    assert sorted(slab * 7 + blk for slab, blk, *_ in firsts) == list(range(74))
 
 
 def test_partition_rejects_bad_arguments():
