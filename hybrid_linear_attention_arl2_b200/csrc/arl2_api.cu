@@ -579,6 +579,8 @@ arl2_status token_pass(arl2_state* h, const void* q, const void* k, const void* 
   p.s_in = h->S[h->cur];
   p.s_out = commit ? h->S[nxt] : nullptr;
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.err = h->err;
+  p.wait_limit_ns = h->wait_ns;
   ARL2_TRY(launch_token_level(p, !(c.flags & ARL2_INTRA_ONLY), st));
   if (commit) {  // S_N becomes the current state; its bf16 copy and read-out operand follow it
     h->cur = nxt;

@@ -46,6 +46,8 @@ struct TokenParams {
   const float* s_in;
   float* s_out;
   __nv_bfloat16* o;
+  uint32_t* err;          // the handle's device error word (a wait that ran out)
+  uint64_t wait_limit_ns;
 };
 size_t token_scratch_floats(int B, int H, int L);
 void token_bind_scratch(TokenParams& p, float* base);

@@ -33,6 +33,7 @@
 
 #include "layer.h"
 #include "params.h"
+#include "sm100.cuh"
 
 namespace arl2 {
 namespace {
@@ -45,37 +46,124 @@ constexpr size_t kChunkSmem = (3 * size_t(kChunk) * kLd + 3 * kChunk) * sizeof(f
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
 
-// (1) One block per (stream, token, head), one thread per channel j:
-// q'_j = sum_i q_i phi_q[i][j], k' likewise then divided by max(|k'|, 1e-12),
-// v' likewise.  Rows go to [B, H, L, 128] f32.
-__global__ void __launch_bounds__(kD) tok_maps_kernel(TokenParams p) {
-  const int r = blockIdx.x;  // (b * L + t) * H + h
-  const int h = r % p.H, bt = r / p.H, t = bt % p.L, b = bt / p.L;
-  const int j = threadIdx.x;
-  __shared__ float xq[kD], xk[kD], xv[kD], red[kD / 32];
-  const size_t row = (size_t(bt) * p.H + h) * kD;
-  xq[j] = bf(p.q[row + j]);
-  xk[j] = bf(p.k[row + j]);
-  xv[j] = bf(p.v[row + j]);
-  __syncthreads();
-  const __nv_bfloat16* pq = p.phi_q + size_t(h) * kD * kD + j;        // pq[i * kD] = phi_q[h][i][j]
-  const __nv_bfloat16* pk = p.phi_k_t + (size_t(h) * kD + j) * kD;    // pk[i] = phi_k[h][i][j]
-  const __nv_bfloat16* pv = p.phi_v_t + (size_t(h) * kD + j) * kD;    // pv[i] = phi_v[h][i][j]
-  float aq = 0.f, ak = 0.f, av = 0.f;
-  for (int i = 0; i < kD; ++i) {
-    aq = fmaf(xq[i], bf(pq[size_t(i) * kD]), aq);
-    ak = fmaf(xk[i], bf(pk[i]), ak);
-    av = fmaf(xv[i], bf(pv[i]), av);
+// (1) One CTA per (stream, head, 128-token chunk), 128 threads (thread t =
+// token t of the chunk).  The chunk's Q, K and V rows and the head's phi_q,
+// phi_k^T and phi_v^T go to shared memory in the 128-byte-swizzle layout of
+// two 64-column boxes; three tcgen05 MMAs (M = tokens, N = K = 128, fp32
+// accumulation in tensor memory) give Q phi_q, K phi_k and V phi_v; thread t
+// reads its rows and writes q'_t, k'_t / max(|k'_t|, 1e-12) and v'_t in f32 to
+// [B, H, L, 128].
+constexpr uint32_t kMapTile = 32768;   // 128 rows x 128 bf16
+constexpr uint32_t kMapHalf = 16384;   // one 64-column box
+constexpr int kMapsSmem = int(6 * kMapTile) + 64 + 1024;
+
+// Byte offset of bf16 element (row, col) of a 128-row tile stored as two
+// 64-column boxes with the 128-byte swizzle (16-byte chunks of a row XORed
+// with row % 8): the layout the tensor cores read through smem_desc_sw128.
+__device__ __forceinline__ uint32_t tok_sw128(int row, int col) {
+  const int box = col >> 6, cc = col & 63;
+  return uint32_t(box) * kMapHalf + uint32_t(row) * 128 + uint32_t(((cc >> 3) ^ (row & 7)) * 16 + (cc & 7) * 2);
+}
+
+__global__ void __launch_bounds__(kD, 1) tok_maps_kernel(TokenParams p) {
+  extern __shared__ uint8_t tok_smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tok_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sX = sm;                   // Q, K, V rows of the chunk (A operands, K-major)
+  uint8_t* sF = sm + 3 * kMapTile;    // phi_q (B, MN-major: rows i), phi_k^T, phi_v^T (B, K-major: rows j)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 6 * kMapTile);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const int c = blockIdx.x % p.n_chunks, bh = blockIdx.x / p.n_chunks;
+  const int b = bh / p.H, h = bh % p.H;
+  const int t0 = c * kChunk, n = min(kChunk, p.L - t0);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
   }
-  float sq = ak * ak;
-  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-  if ((j & 31) == 0) red[j >> 5] = sq;
+  if (warp == 0) tmem_alloc(tmem_holder, 512);
+  const __nv_bfloat16* xs[3] = {p.q, p.k, p.v};
+  const __nv_bfloat16* fs[3] = {p.phi_q, p.phi_k_t, p.phi_v_t};
+  for (int x = tid; x < 3 * 2048; x += kD) {  // 16-byte chunks: tile x >> 11, row (x >> 4) & 127, chunk x & 15
+    const int m = x >> 11, r = (x >> 4) & 127, cc = x & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < n) v = *reinterpret_cast<const uint4*>(xs[m] + ((size_t(b) * p.L + t0 + r) * p.H + h) * kD + cc * 8);
+    *reinterpret_cast<uint4*>(sX + m * kMapTile + tok_sw128(r, cc * 8)) = v;
+    const uint4 f = *reinterpret_cast<const uint4*>(fs[m] + (size_t(h) * kD + r) * kD + cc * 8);
+    *reinterpret_cast<uint4*>(sF + m * kMapTile + tok_sw128(r, cc * 8)) = f;
+  }
+  fence_async_smem();  // the tiles were written through the generic proxy
+  tc_fence_before();
   __syncthreads();
-  const float inv = 1.f / fmaxf(sqrtf(red[0] + red[1] + red[2] + red[3]), 1e-12f);
-  const size_t out = ((size_t(b) * p.H + h) * p.L + t) * kD + j;
-  p.qp[out] = aq;
-  p.kp[out] = ak * inv;
-  p.vp[out] = av;
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtl w{abort_flag, p.err, p.wait_limit_ns};
+  if (tid == 0) {
+    const uint32_t xa = smem_u32(sX), fa = smem_u32(sF);
+    const uint32_t id_mn = idesc_bf16(128, 128, 0, 1), id_k = idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {  // Q phi_q: phi_q stored [i][j], N = j contiguous (MN-major)
+      const uint32_t aoff = (kk >> 2) * kMapHalf + (kk & 3) * 32;
+      mma_ss(tmem, smem_desc_sw128(xa + aoff, 16, 1024), smem_desc_sw128(fa + kk * 2048, kMapHalf, 1024), id_mn,
+             kk > 0);
+    }
+#pragma unroll
+    for (int m = 1; m < 3; ++m) {  // K phi_k, V phi_v: phi^T stored [j][i], K = i contiguous (K-major)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * kMapHalf + (kk & 3) * 32;
+        mma_ss(tmem + m * 128, smem_desc_sw128(xa + m * kMapTile + off, 16, 1024),
+               smem_desc_sw128(fa + m * kMapTile + off, 16, 1024), id_k, kk > 0);
+      }
+    }
+    mma_commit(bar);
+  }
+  bool ok = mbar_wait(bar, 0, w);
+  ok = __all_sync(0xffffffffu, ok);
+  if (ok) {
+    tc_fence_after();
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const size_t out = ((size_t(b) * p.H + h) * p.L + t0 + tid) * kD;
+    float ss = 0.f;  // |k~_t|^2
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      uint32_t r[32];
+      tmem_ld32(tmem + 128 + lane_off + q * 32, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int x = 0; x < 32; ++x) ss = fmaf(__uint_as_float(r[x]), __uint_as_float(r[x]), ss);
+    }
+    const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
+    float* dsts[3] = {p.qp, p.kp, p.vp};
+#pragma unroll 1
+    for (int m = 0; m < 3; ++m) {
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t r[32];
+        tmem_ld32(tmem + m * 128 + lane_off + q * 32, r);
+        tmem_wait_ld();
+        if (tid < n) {
+          const float sc = m == 1 ? inv : 1.f;
+          float4* d4 = reinterpret_cast<float4*>(dsts[m] + out + q * 32);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(r[4 * x]) * sc, __uint_as_float(r[4 * x + 1]) * sc,
+                                __uint_as_float(r[4 * x + 2]) * sc, __uint_as_float(r[4 * x + 3]) * sc);
+        }
+      }
+    }
+  } else if (tid == 0) {  // the MMAs land before tensor memory is released
+    const uint64_t t_0 = global_timer_ns();
+    while (!mbar_try_wait(bar, 0) && global_timer_ns() - t_0 < 10000000ull) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 // (2) One block per (stream, head, chunk), 128 threads.
@@ -111,21 +199,54 @@ __global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
     }
   }
   __syncthreads();
-  // A (strictly lower part; the unit diagonal is implicit) and P, row t per thread
-  if (tid < n) {
-    const float* kt = Kc + size_t(tid) * kD;
-    const float* qt = Qc + size_t(tid) * kD;
-    float g = 1.f;  // G[t][s], s going down from t - 1
-    for (int s = tid - 1; s >= 0; --s) {
-      const float* ks = Kc + size_t(s) * kD;
-      float dk = 0.f, dq = 0.f;
+  // K K^T and Q K^T of the chunk: K and Q staged in X1 and X2 (rows past n
+  // zero), then register-tiled products, thread (ty, tx) = (tid / 8, tid % 8)
+  // owning rows 8 ty .. 8 ty + 7 and columns tx + 8 c (c < 16)
+  for (int x = tid; x < kChunk * kD; x += kChunk) {
+    const int t = x / kD, i = x % kD;
+    X1[t * kLd + i] = t < n ? Kc[size_t(t) * kD + i] : 0.f;
+    X2[t * kLd + i] = t < n ? Qc[size_t(t) * kD + i] : 0.f;
+  }
+  __syncthreads();
+  {
+    const int ty = tid >> 3, tx = tid & 7;
+    float acc[8][16];
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {  // pass 0: K K^T into X0; pass 1: Q K^T into X2
+      const float* Arows = pass == 0 ? X1 : X2;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) acc[r][c2] = 0.f;
+#pragma unroll 4
       for (int i = 0; i < kD; ++i) {
-        dk = fmaf(kt[i], ks[i], dk);
-        dq = fmaf(qt[i], ks[i], dq);
+        float av[8], bv[16];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) av[r] = Arows[(8 * ty + r) * kLd + i];
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) bv[c2] = X1[(tx + 8 * c2) * kLd + i];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c2 = 0; c2 < 16; ++c2) acc[r][c2] = fmaf(av[r], bv[c2], acc[r][c2]);
       }
-      X0[tid * kLd + s] = w[tid] * g * dk;
-      X2[tid * kLd + s] = g * dq;
-      g *= a[s];
+      float* dst = pass == 0 ? X0 : X2;
+      if (pass == 1) __syncthreads();  // every thread is done reading Q out of X2
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) dst[(8 * ty + r) * kLd + tx + 8 * c2] = acc[r][c2];
+    }
+  }
+  __syncthreads();
+  // A (strictly lower part; the unit diagonal is implicit) and P, row t per
+  // thread: A[t][s] = w_t G[t][s] (K K^T)[t][s], P[t][s] = G[t][s] (Q K^T)[t][s]
+  if (tid < n) {
+    float g = 1.f;  // G[t][s], s going down from t - 1
+    for (int s2 = tid - 1; s2 >= 0; --s2) {
+      X0[tid * kLd + s2] *= w[tid] * g;
+      X2[tid * kLd + s2] *= g;
+      g *= a[s2];
     }
   }
   __syncthreads();
@@ -187,48 +308,57 @@ __global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
 // (3) One block per (stream, head, 16-column slab of S), thread i = row i:
 // S_next = M S + N over the chunks in order; the state entering each chunk is
 // kept for (4), and the final one goes to s_out (a commit) or nowhere (a query).
+// Each chunk's M is first copied into shared memory with coalesced loads.
+constexpr int kStateSmem = (kD * kLd + kD * kSlab) * int(sizeof(float));
 __global__ void __launch_bounds__(kD) tok_state_kernel(TokenParams p) {
-  __shared__ float Ss[kD][kSlab];
+  extern __shared__ float st_sm[];
+  float* Ms = st_sm;                                            // [kD][kLd]
+  float(*Ss)[kSlab] = reinterpret_cast<float(*)[kSlab]>(st_sm + kD * kLd);  // [kD][kSlab]
   const int slab = blockIdx.x % (kD / kSlab), bh = blockIdx.x / (kD / kSlab);
   const int i = threadIdx.x, j0 = slab * kSlab;
   for (int jj = 0; jj < kSlab; ++jj) Ss[i][jj] = p.s_in[(size_t(bh) * kD + i) * kD + j0 + jj];
-  __syncthreads();
   for (int c = 0; c < p.n_chunks; ++c) {
     const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
+    for (int x = i; x < kD * kD; x += kD) Ms[(x / kD) * kLd + x % kD] = p.m[mn0 + x];
+    __syncthreads();  // M in; the previous step's state rows are all written
     float acc[kSlab];
     for (int jj = 0; jj < kSlab; ++jj) {
       p.s_chunk[mn0 + size_t(i) * kD + j0 + jj] = Ss[i][jj];
       acc[jj] = p.n[mn0 + size_t(i) * kD + j0 + jj];
     }
-    const float* mrow = p.m + mn0 + size_t(i) * kD;
+    const float* mrow = Ms + i * kLd;
     for (int k = 0; k < kD; ++k) {
       const float mv = mrow[k];
 #pragma unroll
       for (int jj = 0; jj < kSlab; ++jj) acc[jj] = fmaf(mv, Ss[k][jj], acc[jj]);
     }
-    __syncthreads();
+    __syncthreads();  // every row of the entering state is read
 #pragma unroll
     for (int jj = 0; jj < kSlab; ++jj) Ss[i][jj] = acc[jj];
-    __syncthreads();
   }
+  __syncthreads();
   if (p.s_out)
     for (int jj = 0; jj < kSlab; ++jj) p.s_out[(size_t(bh) * kD + i) * kD + j0 + jj] = Ss[i][jj];
 }
 
 // (4) One block per (stream, head, chunk), thread j = channel j:
-// o_t += Qt_t S_c + Ot_t on top of the intra-frame output already in o.
+// o_t += Qt_t S_c + Ot_t on top of the intra-frame output already in o.  The
+// chunk's entering state and its Qt rows are first copied into shared memory.
+constexpr int kOutSmem = (kD * kD + kChunk * kLd) * int(sizeof(float));
 __global__ void __launch_bounds__(kD) tok_out_kernel(TokenParams p) {
-  extern __shared__ float Sc[];  // [kD][kD], the state entering the chunk
+  extern __shared__ float Sc[];  // [kD][kD], the state entering the chunk; then Qt [kChunk][kLd]
+  float* Qs = Sc + kD * kD;
   const int c = blockIdx.x % p.n_chunks, bh = blockIdx.x / p.n_chunks;
   const int b = bh / p.H, h = bh % p.H;
   const int t0 = c * kChunk, n = min(kChunk, p.L - t0);
   const int j = threadIdx.x;
   const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
-  for (int i = 0; i < kD; ++i) Sc[i * kD + j] = p.s_chunk[mn0 + size_t(i) * kD + j];
-  __syncthreads();
   const size_t tok0 = size_t(bh) * p.L + t0;
+  for (int i = 0; i < kD; ++i) Sc[i * kD + j] = p.s_chunk[mn0 + size_t(i) * kD + j];
+  for (int x = j; x < n * kD; x += kD) Qs[(x / kD) * kLd + x % kD] = p.qt[tok0 * kD + x];
+  __syncthreads();
   for (int t = 0; t < n; ++t) {
-    const float* qrow = p.qt + (tok0 + t) * kD;
+    const float* qrow = Qs + t * kLd;
     float acc = p.ot[(tok0 + t) * kD + j];
     for (int i = 0; i < kD; ++i) acc = fmaf(qrow[i], Sc[i * kD + j], acc);
     const size_t o = ((size_t(b) * p.L + t0 + t) * p.H + h) * kD + j;
@@ -260,16 +390,21 @@ void token_bind_scratch(TokenParams& p, float* base) {
 }
 
 cudaError_t launch_token_level(const TokenParams& p, bool with_out, cudaStream_t st) {
-  static unsigned done_chunk = 0, done_out = 0;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(tok_chunk_kernel), int(kChunkSmem), &done_chunk);
+  static unsigned done_chunk = 0, done_out = 0, done_maps = 0;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(tok_maps_kernel), kMapsSmem, &done_maps);
   if (e != cudaSuccess) return e;
-  e = ensure_smem_attr(reinterpret_cast<const void*>(tok_out_kernel), int(kD * kD * sizeof(float)), &done_out);
+  e = ensure_smem_attr(reinterpret_cast<const void*>(tok_chunk_kernel), int(kChunkSmem), &done_chunk);
+  if (e != cudaSuccess) return e;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(tok_out_kernel), kOutSmem, &done_out);
+  if (e != cudaSuccess) return e;
+  static unsigned done_state = 0;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(tok_state_kernel), kStateSmem, &done_state);
   if (e != cudaSuccess) return e;
   const unsigned bh = unsigned(p.B) * unsigned(p.H);
-  tok_maps_kernel<<<unsigned(p.B) * unsigned(p.L) * unsigned(p.H), kD, 0, st>>>(p);
+  tok_maps_kernel<<<bh * unsigned(p.n_chunks), kD, kMapsSmem, st>>>(p);
   tok_chunk_kernel<<<bh * unsigned(p.n_chunks), kChunk, kChunkSmem, st>>>(p);
-  tok_state_kernel<<<bh * unsigned(kD / kSlab), kD, 0, st>>>(p);
-  if (with_out) tok_out_kernel<<<bh * unsigned(p.n_chunks), kD, kD * kD * sizeof(float), st>>>(p);
+  tok_state_kernel<<<bh * unsigned(kD / kSlab), kD, kStateSmem, st>>>(p);
+  if (with_out) tok_out_kernel<<<bh * unsigned(p.n_chunks), kD, kOutSmem, st>>>(p);
   return cudaGetLastError();
 }
 
