@@ -46,6 +46,57 @@ constexpr size_t kChunkSmem = (3 * size_t(kChunk) * kLd + 3 * kChunk) * sizeof(f
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
 
+// acc[r][c] = sum over s < ns of A(8 ty + r, s) B(s, tx + 8 c) for thread
+// (ty, tx) = (tid / 8, tid % 8) of 128: a 128 x 128 product tiled 8 x 16 per
+// thread (operands read through the accessors, from shared memory).
+template <class FA, class FB>
+__device__ __forceinline__ void tile_product(float (&acc)[8][16], int ns, FA fa, FB fb) {
+  const int ty = threadIdx.x >> 3, tx = threadIdx.x & 7;
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 16; ++c) acc[r][c] = 0.f;
+#pragma unroll 2
+  for (int s = 0; s < ns; ++s) {
+    float av[8], bv[16];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) av[r] = fa(8 * ty + r, s);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) bv[c] = fb(s, tx + 8 * c);
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+  }
+}
+
+// Copy rows [0, n) of a row-major [rows][128] f32 matrix into shared memory
+// with row pitch `ld` floats (rows n .. 127 zero when zero_tail), 128 threads,
+// eight 16-byte loads in flight per thread.
+__device__ __forceinline__ void stage_rows(float* dst, int ld, const float* src, int n, bool zero_tail) {
+  const int tid = threadIdx.x;
+#pragma unroll 1
+  for (int base = 0; base < 4096; base += 8 * 128) {  // 128 rows x 32 float4
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int x = base + u * 128 + tid, r = x >> 5;
+      v[u] = r < n ? reinterpret_cast<const float4*>(src)[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int x = base + u * 128 + tid, r = x >> 5, c4 = x & 31;
+      if (r < n || zero_tail) {
+        float* d = dst + r * ld + c4 * 4;
+        d[0] = v[u].x;
+        d[1] = v[u].y;
+        d[2] = v[u].z;
+        d[3] = v[u].w;
+      }
+    }
+  }
+}
+
 // (1) One CTA per (stream, head, 128-token chunk), 128 threads (thread t =
 // token t of the chunk).  The chunk's Q, K and V rows and the head's phi_q,
 // phi_k^T and phi_v^T go to shared memory in the 128-byte-swizzle layout of
@@ -83,15 +134,24 @@ __global__ void __launch_bounds__(kD, 1) tok_maps_kernel(TokenParams p) {
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(tmem_holder, 512);
-  const __nv_bfloat16* xs[3] = {p.q, p.k, p.v};
-  const __nv_bfloat16* fs[3] = {p.phi_q, p.phi_k_t, p.phi_v_t};
-  for (int x = tid; x < 3 * 2048; x += kD) {  // 16-byte chunks: tile x >> 11, row (x >> 4) & 127, chunk x & 15
-    const int m = x >> 11, r = (x >> 4) & 127, cc = x & 15;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < n) v = *reinterpret_cast<const uint4*>(xs[m] + ((size_t(b) * p.L + t0 + r) * p.H + h) * kD + cc * 8);
-    *reinterpret_cast<uint4*>(sX + m * kMapTile + tok_sw128(r, cc * 8)) = v;
-    const uint4 f = *reinterpret_cast<const uint4*>(fs[m] + (size_t(h) * kD + r) * kD + cc * 8);
-    *reinterpret_cast<uint4*>(sF + m * kMapTile + tok_sw128(r, cc * 8)) = f;
+#pragma unroll 1
+  for (int base = 0; base < 3 * 2048; base += 8 * kD) {  // 16-byte chunks: tile x >> 11, row (x >> 4) & 127, chunk x & 15
+    uint4 v[8], f[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int x = base + u * kD + tid, m = x >> 11, r = (x >> 4) & 127, cc = x & 15;
+      const __nv_bfloat16* xsrc = m == 0 ? p.q : (m == 1 ? p.k : p.v);
+      const __nv_bfloat16* fsrc = m == 0 ? p.phi_q : (m == 1 ? p.phi_k_t : p.phi_v_t);
+      v[u] = r < n ? *reinterpret_cast<const uint4*>(xsrc + ((size_t(b) * p.L + t0 + r) * p.H + h) * kD + cc * 8)
+                   : make_uint4(0u, 0u, 0u, 0u);
+      f[u] = *reinterpret_cast<const uint4*>(fsrc + (size_t(h) * kD + r) * kD + cc * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int x = base + u * kD + tid, m = x >> 11, r = (x >> 4) & 127, cc = x & 15;
+      *reinterpret_cast<uint4*>(sX + m * kMapTile + tok_sw128(r, cc * 8)) = v[u];
+      *reinterpret_cast<uint4*>(sF + m * kMapTile + tok_sw128(r, cc * 8)) = f[u];
+    }
   }
   fence_async_smem();  // the tiles were written through the generic proxy
   tc_fence_before();
@@ -135,9 +195,9 @@ __global__ void __launch_bounds__(kD, 1) tok_maps_kernel(TokenParams p) {
       for (int x = 0; x < 32; ++x) ss = fmaf(__uint_as_float(r[x]), __uint_as_float(r[x]), ss);
     }
     const float inv = 1.f / fmaxf(sqrtf(ss), 1e-12f);
-    float* dsts[3] = {p.qp, p.kp, p.vp};
 #pragma unroll 1
     for (int m = 0; m < 3; ++m) {
+      float* dst_m = m == 0 ? p.qp : (m == 1 ? p.kp : p.vp);
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         uint32_t r[32];
@@ -145,7 +205,7 @@ __global__ void __launch_bounds__(kD, 1) tok_maps_kernel(TokenParams p) {
         tmem_wait_ld();
         if (tid < n) {
           const float sc = m == 1 ? inv : 1.f;
-          float4* d4 = reinterpret_cast<float4*>(dsts[m] + out + q * 32);
+          float4* d4 = reinterpret_cast<float4*>(dst_m + out + q * 32);
 #pragma unroll
           for (int x = 0; x < 8; ++x)
             d4[x] = make_float4(__uint_as_float(r[4 * x]) * sc, __uint_as_float(r[4 * x + 1]) * sc,
@@ -202,11 +262,8 @@ __global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
   // K K^T and Q K^T of the chunk: K and Q staged in X1 and X2 (rows past n
   // zero), then register-tiled products, thread (ty, tx) = (tid / 8, tid % 8)
   // owning rows 8 ty .. 8 ty + 7 and columns tx + 8 c (c < 16)
-  for (int x = tid; x < kChunk * kD; x += kChunk) {
-    const int t = x / kD, i = x % kD;
-    X1[t * kLd + i] = t < n ? Kc[size_t(t) * kD + i] : 0.f;
-    X2[t * kLd + i] = t < n ? Qc[size_t(t) * kD + i] : 0.f;
-  }
+  stage_rows(X1, kLd, Kc, n, true);
+  stage_rows(X2, kLd, Qc, n, true);
   __syncthreads();
   {
     const int ty = tid >> 3, tx = tid & 7;
@@ -262,77 +319,119 @@ __global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
     }
   }
   __syncthreads();
-  // W = T diag(w g_prev) K and U' = T diag(w) V, column j per thread (128 columns)
-  const int j = tid;
-  for (int t = 0; t < n; ++t) {
-    float aw = 0.f, au = 0.f;
-    for (int s = 0; s <= t; ++s) {
-      const float tv = X1[t * kLd + s];
-      aw = fmaf(tv * w[s] * g_prev[s], Kc[size_t(s) * kD + j], aw);
-      au = fmaf(tv * w[s], Vc[size_t(s) * kD + j], au);
+  // The rest as register-tiled products over shared memory (thread (ty, tx)
+  // owns rows 8 ty + r and columns tx + 8 c), rows past n kept at zero:
+  // W = T diag(w g_prev) K and U' = T diag(w) V (K, then V, staged in X0)
+  const int ty = tid >> 3, tx = tid & 7;
+  float acc[8][16];
+  const float* Vc2 = Vc;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    stage_rows(X0, kLd, pass == 0 ? Kc : Vc2, n, true);
+    __syncthreads();
+    tile_product(acc, n, [&](int t, int s2) { return X1[t * kLd + s2] * (pass == 0 ? w[s2] * g_prev[s2] : w[s2]); },
+                 [&](int s2, int jj) { return X0[s2 * kLd + jj]; });
+    float* dst = pass == 0 ? p.w : p.u;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int t = 8 * ty + r;
+      if (t < n)
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) dst[(tok0 + t) * kD + tx + 8 * c2] = acc[r][c2];
     }
-    p.w[(tok0 + t) * kD + j] = aw;
-    p.u[(tok0 + t) * kD + j] = au;
+    __syncthreads();  // X0 is read; the next pass restages it
   }
-  __syncthreads();  // every thread is done with T and A: W into X0, U' into X1
-  for (int t = 0; t < n; ++t) {
-    X0[t * kLd + j] = p.w[(tok0 + t) * kD + j];
-    X1[t * kLd + j] = p.u[(tok0 + t) * kD + j];
-  }
+  // W into X0, U' into X1 (T is done with)
+  stage_rows(X0, kLd, p.w + tok0 * kD, n, true);
+  stage_rows(X1, kLd, p.u + tok0 * kD, n, true);
   __syncthreads();
-  // M = g_C I - Kt^T W and N = Kt^T U', column j per thread, rows i over the state
-  const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
-  for (int i = 0; i < kD; ++i) {
-    float am = i == j ? g_all : 0.f, an = 0.f;
-    for (int s = 0; s < n; ++s) {
-      const float kt = g_tail[s] * Kc[size_t(s) * kD + i];
-      am = fmaf(-kt, X0[s * kLd + j], am);
-      an = fmaf(kt, X1[s * kLd + j], an);
+  // Qt = diag(g_prev) Q - P W and Ot = P U' (P strictly lower)
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const float* Bm = pass == 0 ? X0 : X1;
+    tile_product(acc, n, [&](int t, int s2) { return s2 < t ? X2[t * kLd + s2] : 0.f; },
+                 [&](int s2, int jj) { return Bm[s2 * kLd + jj]; });
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int t = 8 * ty + r;
+      if (t < n) {
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) {
+          const int jj = tx + 8 * c2;
+          if (pass == 0)
+            p.qt[(tok0 + t) * kD + jj] = g_prev[t] * Qc[size_t(t) * kD + jj] - acc[r][c2];
+          else
+            p.ot[(tok0 + t) * kD + jj] = acc[r][c2];
+        }
+      }
     }
-    p.m[mn0 + size_t(i) * kD + j] = am;
-    p.n[mn0 + size_t(i) * kD + j] = an;
   }
-  // Qt = diag(g_prev) Q - P W and Ot = P U', column j per thread
-  for (int t = 0; t < n; ++t) {
-    float aq = g_prev[t] * Qc[size_t(t) * kD + j], ao = 0.f;
-    for (int s = 0; s < t; ++s) {
-      const float pv = X2[t * kLd + s];
-      aq = fmaf(-pv, X0[s * kLd + j], aq);
-      ao = fmaf(pv, X1[s * kLd + j], ao);
+  __syncthreads();  // P is done with: K into X2
+  stage_rows(X2, kLd, Kc, n, true);
+  __syncthreads();
+  // M = g_C I - Kt^T W and N = Kt^T U', Kt = diag(g_tail) K (rows i of the state)
+  const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const float* Bm = pass == 0 ? X0 : X1;
+    tile_product(acc, n, [&](int i, int s2) { return g_tail[s2] * X2[s2 * kLd + i]; },
+                 [&](int s2, int jj) { return Bm[s2 * kLd + jj]; });
+    float* dst = pass == 0 ? p.m : p.n;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int i = 8 * ty + r;
+#pragma unroll
+      for (int c2 = 0; c2 < 16; ++c2) {
+        const int jj = tx + 8 * c2;
+        dst[mn0 + size_t(i) * kD + jj] = pass == 0 ? ((i == jj ? g_all : 0.f) - acc[r][c2]) : acc[r][c2];
+      }
     }
-    p.qt[(tok0 + t) * kD + j] = aq;
-    p.ot[(tok0 + t) * kD + j] = ao;
   }
 }
 
 // (3) One block per (stream, head, 16-column slab of S), thread i = row i:
 // S_next = M S + N over the chunks in order; the state entering each chunk is
 // kept for (4), and the final one goes to s_out (a commit) or nowhere (a query).
-// Each chunk's M is first copied into shared memory with coalesced loads.
-constexpr int kStateSmem = (kD * kLd + kD * kSlab) * int(sizeof(float));
+// Each chunk's M is copied into one of two shared-memory buffers with
+// asynchronous copies issued a chunk ahead, so the copy of chunk c + 1 runs
+// while chunk c computes.
+constexpr int kStateSmem = (2 * kD * kLd + kD * kSlab) * int(sizeof(float));
+
+__device__ __forceinline__ void copy_async_m(float* dst, const float* src) {  // [128][128] f32 into pitch kLd
+  const int tid = threadIdx.x;
+#pragma unroll 8
+  for (int x = tid; x < kD * kD; x += kD) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst + (x >> 7) * kLd + (x & 127)));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src + x) : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(kD) tok_state_kernel(TokenParams p) {
   extern __shared__ float st_sm[];
-  float* Ms = st_sm;                                            // [kD][kLd]
-  float(*Ss)[kSlab] = reinterpret_cast<float(*)[kSlab]>(st_sm + kD * kLd);  // [kD][kSlab]
+  float* Mbuf = st_sm;                                                              // [2][kD][kLd]
+  float(*Ss)[kSlab] = reinterpret_cast<float(*)[kSlab]>(st_sm + 2 * kD * kLd);  // [kD][kSlab]
   const int slab = blockIdx.x % (kD / kSlab), bh = blockIdx.x / (kD / kSlab);
   const int i = threadIdx.x, j0 = slab * kSlab;
   for (int jj = 0; jj < kSlab; ++jj) Ss[i][jj] = p.s_in[(size_t(bh) * kD + i) * kD + j0 + jj];
+  copy_async_m(Mbuf, p.m + size_t(bh) * p.n_chunks * kD * kD);
   for (int c = 0; c < p.n_chunks; ++c) {
     const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
-    for (int x = i; x < kD * kD; x += kD) Ms[(x / kD) * kLd + x % kD] = p.m[mn0 + x];
-    __syncthreads();  // M in; the previous step's state rows are all written
     float acc[kSlab];
-    for (int jj = 0; jj < kSlab; ++jj) {
-      p.s_chunk[mn0 + size_t(i) * kD + j0 + jj] = Ss[i][jj];
-      acc[jj] = p.n[mn0 + size_t(i) * kD + j0 + jj];
-    }
-    const float* mrow = Ms + i * kLd;
+#pragma unroll
+    for (int jj = 0; jj < kSlab; ++jj) acc[jj] = p.n[mn0 + size_t(i) * kD + j0 + jj];
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();  // M(c) in; the previous step's state rows are all written
+    if (c + 1 < p.n_chunks) copy_async_m(Mbuf + ((c + 1) & 1) * kD * kLd, p.m + mn0 + kD * kD);
+#pragma unroll
+    for (int jj = 0; jj < kSlab; ++jj) p.s_chunk[mn0 + size_t(i) * kD + j0 + jj] = Ss[i][jj];
+    const float* mrow = Mbuf + (c & 1) * kD * kLd + i * kLd;
     for (int k = 0; k < kD; ++k) {
       const float mv = mrow[k];
 #pragma unroll
       for (int jj = 0; jj < kSlab; ++jj) acc[jj] = fmaf(mv, Ss[k][jj], acc[jj]);
     }
-    __syncthreads();  // every row of the entering state is read
+    __syncthreads();  // every row of the entering state and of M(c) is read
 #pragma unroll
     for (int jj = 0; jj < kSlab; ++jj) Ss[i][jj] = acc[jj];
   }
@@ -354,15 +453,29 @@ __global__ void __launch_bounds__(kD) tok_out_kernel(TokenParams p) {
   const int j = threadIdx.x;
   const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
   const size_t tok0 = size_t(bh) * p.L + t0;
-  for (int i = 0; i < kD; ++i) Sc[i * kD + j] = p.s_chunk[mn0 + size_t(i) * kD + j];
-  for (int x = j; x < n * kD; x += kD) Qs[(x / kD) * kLd + x % kD] = p.qt[tok0 * kD + x];
+  stage_rows(Sc, kD, p.s_chunk + mn0, kD, true);
+  stage_rows(Qs, kLd, p.qt + tok0 * kD, n, true);
   __syncthreads();
-  for (int t = 0; t < n; ++t) {
-    const float* qrow = Qs + t * kLd;
-    float acc = p.ot[(tok0 + t) * kD + j];
-    for (int i = 0; i < kD; ++i) acc = fmaf(qrow[i], Sc[i * kD + j], acc);
-    const size_t o = ((size_t(b) * p.L + t0 + t) * p.H + h) * kD + j;
-    p.o[o] = __float2bfloat16_rn(bf(p.o[o]) + acc);
+  // Qt S_c as a register-tiled product (thread (ty, tx): tokens 8 ty + r,
+  // channels tx + 8 c), then o += it + Ot with every load of the tile in flight
+  float acc[8][16];
+  tile_product(acc, kD, [&](int t, int i) { return Qs[t * kLd + i]; }, [&](int i, int jj) { return Sc[i * kD + jj]; });
+  const int ty = j >> 3, tx = j & 7;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int t = 8 * ty + r;
+    if (t < n) {
+      float ot[16];
+      __nv_bfloat16 ov[16];
+      const size_t o0 = ((size_t(b) * p.L + t0 + t) * p.H + h) * kD;
+#pragma unroll
+      for (int c2 = 0; c2 < 16; ++c2) {
+        ot[c2] = p.ot[(tok0 + t) * kD + tx + 8 * c2];
+        ov[c2] = p.o[o0 + tx + 8 * c2];
+      }
+#pragma unroll
+      for (int c2 = 0; c2 < 16; ++c2) p.o[o0 + tx + 8 * c2] = __float2bfloat16_rn(bf(ov[c2]) + acc[r][c2] + ot[c2]);
+    }
   }
 }
 
