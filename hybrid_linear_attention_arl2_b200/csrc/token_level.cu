@@ -70,22 +70,46 @@ __device__ __forceinline__ void tile_product(float (&acc)[8][16], int ns, FA fa,
   }
 }
 
+// The same with 256 threads: thread (ty, tx) = (tid / 8, tid % 8) owns rows
+// 4 ty + r (r < 4) and columns tx + 8 c.
+template <class FA, class FB>
+__device__ __forceinline__ void tile_product4(float (&acc)[4][16], int ns, FA fa, FB fb) {
+  const int ty = threadIdx.x >> 3, tx = threadIdx.x & 7;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 16; ++c) acc[r][c] = 0.f;
+#pragma unroll 2
+  for (int s = 0; s < ns; ++s) {
+    float av[4], bv[16];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) av[r] = fa(4 * ty + r, s);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) bv[c] = fb(s, tx + 8 * c);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+  }
+}
+
 // Copy rows [0, n) of a row-major [rows][128] f32 matrix into shared memory
-// with row pitch `ld` floats (rows n .. 127 zero when zero_tail), 128 threads,
-// eight 16-byte loads in flight per thread.
+// with row pitch `ld` floats (rows n .. 127 zero when zero_tail), NT threads
+// (128 or 256), eight 16-byte loads in flight per thread.
+template <int NT = 128>
 __device__ __forceinline__ void stage_rows(float* dst, int ld, const float* src, int n, bool zero_tail) {
   const int tid = threadIdx.x;
 #pragma unroll 1
-  for (int base = 0; base < 4096; base += 8 * 128) {  // 128 rows x 32 float4
+  for (int base = 0; base < 4096; base += 8 * NT) {  // 128 rows x 32 float4
     float4 v[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int x = base + u * 128 + tid, r = x >> 5;
+      const int x = base + u * NT + tid, r = x >> 5;
       v[u] = r < n ? reinterpret_cast<const float4*>(src)[x] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int x = base + u * 128 + tid, r = x >> 5, c4 = x & 31;
+      const int x = base + u * NT + tid, r = x >> 5, c4 = x & 31;
       if (r < n || zero_tail) {
         float* d = dst + r * ld + c4 * 4;
         d[0] = v[u].x;
@@ -226,8 +250,10 @@ __global__ void __launch_bounds__(kD, 1) tok_maps_kernel(TokenParams p) {
   }
 }
 
-// (2) One block per (stream, head, chunk), 128 threads.
-__global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
+// (2) One block per (stream, head, chunk), 256 threads (the row-per-thread
+// steps use the first 128).
+constexpr int kChunkThreads = 256;
+__global__ void __launch_bounds__(kChunkThreads, 1) tok_chunk_kernel(TokenParams p) {
   extern __shared__ float sm[];
   float* X0 = sm;                    // A, then W
   float* X1 = X0 + kChunk * kLd;     // T = A^-1, then U'
@@ -261,38 +287,24 @@ __global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
   __syncthreads();
   // K K^T and Q K^T of the chunk: K and Q staged in X1 and X2 (rows past n
   // zero), then register-tiled products, thread (ty, tx) = (tid / 8, tid % 8)
-  // owning rows 8 ty .. 8 ty + 7 and columns tx + 8 c (c < 16)
-  stage_rows(X1, kLd, Kc, n, true);
-  stage_rows(X2, kLd, Qc, n, true);
+  // owning rows 4 ty .. 4 ty + 3 and columns tx + 8 c (c < 16)
+  stage_rows<kChunkThreads>(X1, kLd, Kc, n, true);
+  stage_rows<kChunkThreads>(X2, kLd, Qc, n, true);
   __syncthreads();
   {
     const int ty = tid >> 3, tx = tid & 7;
-    float acc[8][16];
+    float acc[4][16];
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {  // pass 0: K K^T into X0; pass 1: Q K^T into X2
       const float* Arows = pass == 0 ? X1 : X2;
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) acc[r][c2] = 0.f;
-#pragma unroll 4
-      for (int i = 0; i < kD; ++i) {
-        float av[8], bv[16];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) av[r] = Arows[(8 * ty + r) * kLd + i];
-#pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) bv[c2] = X1[(tx + 8 * c2) * kLd + i];
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int c2 = 0; c2 < 16; ++c2) acc[r][c2] = fmaf(av[r], bv[c2], acc[r][c2]);
-      }
+      tile_product4(acc, kD, [&](int t, int i) { return Arows[t * kLd + i]; },
+                    [&](int i, int s2) { return X1[s2 * kLd + i]; });
       float* dst = pass == 0 ? X0 : X2;
       if (pass == 1) __syncthreads();  // every thread is done reading Q out of X2
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
+      for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) dst[(8 * ty + r) * kLd + tx + 8 * c2] = acc[r][c2];
+        for (int c2 = 0; c2 < 16; ++c2) dst[(4 * ty + r) * kLd + tx + 8 * c2] = acc[r][c2];
     }
   }
   __syncthreads();
@@ -320,21 +332,21 @@ __global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
   }
   __syncthreads();
   // The rest as register-tiled products over shared memory (thread (ty, tx)
-  // owns rows 8 ty + r and columns tx + 8 c), rows past n kept at zero:
+  // owns rows 4 ty + r and columns tx + 8 c), rows past n kept at zero:
   // W = T diag(w g_prev) K and U' = T diag(w) V (K, then V, staged in X0)
   const int ty = tid >> 3, tx = tid & 7;
-  float acc[8][16];
+  float acc[4][16];
   const float* Vc2 = Vc;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
-    stage_rows(X0, kLd, pass == 0 ? Kc : Vc2, n, true);
+    stage_rows<kChunkThreads>(X0, kLd, pass == 0 ? Kc : Vc2, n, true);
     __syncthreads();
-    tile_product(acc, n, [&](int t, int s2) { return X1[t * kLd + s2] * (pass == 0 ? w[s2] * g_prev[s2] : w[s2]); },
+    tile_product4(acc, n, [&](int t, int s2) { return X1[t * kLd + s2] * (pass == 0 ? w[s2] * g_prev[s2] : w[s2]); },
                  [&](int s2, int jj) { return X0[s2 * kLd + jj]; });
     float* dst = pass == 0 ? p.w : p.u;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int t = 8 * ty + r;
+    for (int r = 0; r < 4; ++r) {
+      const int t = 4 * ty + r;
       if (t < n)
 #pragma unroll
         for (int c2 = 0; c2 < 16; ++c2) dst[(tok0 + t) * kD + tx + 8 * c2] = acc[r][c2];
@@ -342,18 +354,18 @@ __global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
     __syncthreads();  // X0 is read; the next pass restages it
   }
   // W into X0, U' into X1 (T is done with)
-  stage_rows(X0, kLd, p.w + tok0 * kD, n, true);
-  stage_rows(X1, kLd, p.u + tok0 * kD, n, true);
+  stage_rows<kChunkThreads>(X0, kLd, p.w + tok0 * kD, n, true);
+  stage_rows<kChunkThreads>(X1, kLd, p.u + tok0 * kD, n, true);
   __syncthreads();
   // Qt = diag(g_prev) Q - P W and Ot = P U' (P strictly lower)
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const float* Bm = pass == 0 ? X0 : X1;
-    tile_product(acc, n, [&](int t, int s2) { return s2 < t ? X2[t * kLd + s2] : 0.f; },
-                 [&](int s2, int jj) { return Bm[s2 * kLd + jj]; });
+    tile_product4(acc, n, [&](int t, int s2) { return s2 < t ? X2[t * kLd + s2] : 0.f; },
+                  [&](int s2, int jj) { return Bm[s2 * kLd + jj]; });
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int t = 8 * ty + r;
+    for (int r = 0; r < 4; ++r) {
+      const int t = 4 * ty + r;
       if (t < n) {
 #pragma unroll
         for (int c2 = 0; c2 < 16; ++c2) {
@@ -367,19 +379,19 @@ __global__ void __launch_bounds__(kChunk) tok_chunk_kernel(TokenParams p) {
     }
   }
   __syncthreads();  // P is done with: K into X2
-  stage_rows(X2, kLd, Kc, n, true);
+  stage_rows<kChunkThreads>(X2, kLd, Kc, n, true);
   __syncthreads();
   // M = g_C I - Kt^T W and N = Kt^T U', Kt = diag(g_tail) K (rows i of the state)
   const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const float* Bm = pass == 0 ? X0 : X1;
-    tile_product(acc, n, [&](int i, int s2) { return g_tail[s2] * X2[s2 * kLd + i]; },
-                 [&](int s2, int jj) { return Bm[s2 * kLd + jj]; });
+    tile_product4(acc, n, [&](int i, int s2) { return g_tail[s2] * X2[s2 * kLd + i]; },
+                  [&](int s2, int jj) { return Bm[s2 * kLd + jj]; });
     float* dst = pass == 0 ? p.m : p.n;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int i = 8 * ty + r;
+    for (int r = 0; r < 4; ++r) {
+      const int i = 4 * ty + r;
 #pragma unroll
       for (int c2 = 0; c2 < 16; ++c2) {
         const int jj = tx + 8 * c2;
@@ -515,7 +527,7 @@ cudaError_t launch_token_level(const TokenParams& p, bool with_out, cudaStream_t
   if (e != cudaSuccess) return e;
   const unsigned bh = unsigned(p.B) * unsigned(p.H);
   tok_maps_kernel<<<bh * unsigned(p.n_chunks), kD, kMapsSmem, st>>>(p);
-  tok_chunk_kernel<<<bh * unsigned(p.n_chunks), kChunk, kChunkSmem, st>>>(p);
+  tok_chunk_kernel<<<bh * unsigned(p.n_chunks), kChunkThreads, kChunkSmem, st>>>(p);
   tok_state_kernel<<<bh * unsigned(kD / kSlab), kD, kStateSmem, st>>>(p);
   if (with_out) tok_out_kernel<<<bh * unsigned(p.n_chunks), kD, kOutSmem, st>>>(p);
   return cudaGetLastError();
