@@ -20,11 +20,12 @@
 //   S_next = M S + N,        M = g_C I - Kt^T W,  N = Kt^T U',  Kt = diag(g_tail) K,
 //   O      = Qt S + Ot,      Qt = diag(g_prev) Q - P W,  Ot = P U',  P = G * (Q K^T),
 //
-// whose operands need no state.  So: (1) the maps per token; (2) one block
-// per (stream, head, chunk) builds M, N, Qt, Ot; (3) one block per (stream,
-// head, 16-column slab of S) runs S_next = M S + N over the chunks in order;
-// (4) one block per (stream, head, chunk) adds Qt S + Ot to the intra-frame
-// output.  This first version computes in fp32 on the CUDA cores.
+// whose operands need no state.  So: (1) the maps per token (tcgen05); (2)
+// one CTA per (stream, head, chunk) builds M, N, Qt, Ot (tcgen05 products,
+// A^-1 in f32 on the CUDA cores); (3) one block per (stream, head, 16-column
+// slab of S) runs S_next = M S + N over the chunks in order (f32); (4) one
+// block per (stream, head, chunk) adds Qt S + Ot to the intra-frame output
+// (f32, register-tiled).
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -42,7 +43,6 @@ constexpr int kD = 128;         // head dim
 constexpr int kChunk = 128;     // tokens per chunk
 constexpr int kLd = kChunk + 1;  // padded row pitch of the chunk matrices in shared memory
 constexpr int kSlab = 16;       // state columns per block of the sequential kernel
-constexpr size_t kChunkSmem = (3 * size_t(kChunk) * kLd + 3 * kChunk) * sizeof(float);
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -65,29 +65,6 @@ __device__ __forceinline__ void tile_product(float (&acc)[8][16], int ns, FA fa,
     for (int c = 0; c < 16; ++c) bv[c] = fb(s, tx + 8 * c);
 #pragma unroll
     for (int r = 0; r < 8; ++r)
-#pragma unroll
-      for (int c = 0; c < 16; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-  }
-}
-
-// The same with 256 threads: thread (ty, tx) = (tid / 8, tid % 8) owns rows
-// 4 ty + r (r < 4) and columns tx + 8 c.
-template <class FA, class FB>
-__device__ __forceinline__ void tile_product4(float (&acc)[4][16], int ns, FA fa, FB fb) {
-  const int ty = threadIdx.x >> 3, tx = threadIdx.x & 7;
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 16; ++c) acc[r][c] = 0.f;
-#pragma unroll 2
-  for (int s = 0; s < ns; ++s) {
-    float av[4], bv[16];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) av[r] = fa(4 * ty + r, s);
-#pragma unroll
-    for (int c = 0; c < 16; ++c) bv[c] = fb(s, tx + 8 * c);
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
 #pragma unroll
       for (int c = 0; c < 16; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
   }
@@ -250,25 +227,85 @@ __global__ void __launch_bounds__(kD, 1) tok_maps_kernel(TokenParams p) {
   }
 }
 
-// (2) One block per (stream, head, chunk), 256 threads (the row-per-thread
-// steps use the first 128).
-constexpr int kChunkThreads = 256;
-__global__ void __launch_bounds__(kChunkThreads, 1) tok_chunk_kernel(TokenParams p) {
-  extern __shared__ float sm[];
-  float* X0 = sm;                    // A, then W
-  float* X1 = X0 + kChunk * kLd;     // T = A^-1, then U'
-  float* X2 = X1 + kChunk * kLd;     // P
-  float* w = X2 + kChunk * kLd;      // c beta
+// (2) The chunk's maps on tcgen05: one CTA per (stream, head, chunk), 128 threads
+// (thread t = token t, or state row t).  bf16 operands in shared memory (the
+// 128-byte-swizzle tiles the tensor cores read), f32 accumulation in tensor
+// memory; A^-1 by forward substitution in f32 on the CUDA cores.  Products:
+//   K K^T, Q K^T                  -> A (f32), P = G * (Q K^T) (bf16)
+//   W = T1 K,  U' = T2 V          T1 = T diag(w g_prev), T2 = T diag(w)
+//   M' = K^T Wt, N = K^T Ut       Wt = diag(g_tail) W, Ut = diag(g_tail) U'
+//   Qt' = P W, Ot = P U'          M = g_C I - M', Qt = diag(g_prev) Q - Qt'
+// (bf16 operands keep the outputs within 6e-3 and the state within 4e-3 of
+// the f64 recurrence on the 1560-token frame, CPU emulation.)
+constexpr uint32_t kTcTile = 32768, kTcHalf = 16384;
+constexpr uint32_t kTcF32 = 66560;  // one f32 128 x 129 matrix, rounded up to 1 KB
+constexpr int kTcSmem = int(2 * kTcTile + 2 * kTcF32) + 3 * kChunk * 4 + 64 + 1024;
+
+// Row `row` of a bf16 tile from 128 f32 values (16-byte chunks, swizzled).
+__device__ __forceinline__ void tile_row_bf16(uint8_t* tile, int row, const float (&v)[128]) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    *reinterpret_cast<uint4*>(tile + tok_sw128(row, 8 * c)) =
+        make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                   pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+}
+
+// Rows [0, n) of a row-major [rows][128] f32 matrix into a bf16 tile (rows
+// past n zero), 128 threads.
+__device__ __forceinline__ void tile_from_f32(uint8_t* tile, const float* src, int n) {
+#pragma unroll 4
+  for (int x = threadIdx.x; x < 2048; x += kD) {
+    const int r = x >> 4, cc = x & 15;
+    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a4;
+    if (r < n) {
+      a4 = reinterpret_cast<const float4*>(src + r * kD + cc * 8)[0];
+      b4 = reinterpret_cast<const float4*>(src + r * kD + cc * 8)[1];
+    }
+    *reinterpret_cast<uint4*>(tile + tok_sw128(r, cc * 8)) =
+        make_uint4(pack_bf16x2(a4.x, a4.y), pack_bf16x2(a4.z, a4.w), pack_bf16x2(b4.x, b4.y), pack_bf16x2(b4.z, b4.w));
+  }
+}
+
+// 128 x 128 x 128 product into tensor memory: A and B by their descriptors'
+// layouts (K-major: 64-column boxes, K steps of 32 bytes; MN-major: K steps of
+// 2048 bytes, boxes kTcHalf apart).
+__device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, bool a_mn, uint32_t b, bool b_mn) {
+  const uint32_t id = idesc_bf16(128, 128, a_mn ? 1 : 0, b_mn ? 1 : 0);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t koff = (kk >> 2) * kTcHalf + (kk & 3) * 32, moff = kk * 2048;
+    mma_ss(d, a_mn ? smem_desc_sw128(a + moff, kTcHalf, 1024) : smem_desc_sw128(a + koff, 16, 1024),
+           b_mn ? smem_desc_sw128(b + moff, kTcHalf, 1024) : smem_desc_sw128(b + koff, 16, 1024), id, kk > 0);
+  }
+}
+
+__device__ __forceinline__ void tmem_row128(uint32_t taddr, float (&v)[128]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_ld32(taddr + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * q]));
+  tmem_wait_ld();
+}
+
+__global__ void __launch_bounds__(kD, 1) tok_chunk_tc_kernel(TokenParams p) {
+  extern __shared__ uint8_t tc_smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tK = sm;                       // K' [t][d] (bf16)
+  uint8_t* tP = sm + kTcTile;             // Q' [t][d], then P [t][s]
+  uint8_t* R0 = sm + 2 * kTcTile;         // A (f32), then T1, T2; then Wt, W (bf16 tiles)
+  uint8_t* R1 = R0 + kTcF32;              // G, then T (f32); then V'; then Ut, U' (bf16 tiles)
+  float* F0 = reinterpret_cast<float*>(R0);
+  float* F1 = reinterpret_cast<float*>(R1);
+  float* w = reinterpret_cast<float*>(R1 + kTcF32);  // c beta
   float* g_prev = w + kChunk;
   float* g_tail = g_prev + kChunk;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(g_tail + kChunk);  // [3] MMA phases
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   __shared__ float g_all;
   const int c = blockIdx.x % p.n_chunks, bh = blockIdx.x / p.n_chunks;
   const int t0 = c * kChunk, n = min(kChunk, p.L - t0);
-  const int tid = threadIdx.x;
-  const size_t tok0 = size_t(bh) * p.L + t0;  // row of the chunk's first token in the [B, H, L] arrays
-  const float* Kc = p.kp + tok0 * kD;
-  const float* Qc = p.qp + tok0 * kD;
-  const float* Vc = p.vp + tok0 * kD;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t lane_off = uint32_t(warp * 32) << 16;
+  const size_t tok0 = size_t(bh) * p.L + t0;
   const float* a = p.alpha_tok + tok0;
   if (tid < n) w[tid] = p.corr * p.beta[tok0 + tid];
   if (tid == 0) {
@@ -279,125 +316,169 @@ __global__ void __launch_bounds__(kChunkThreads, 1) tok_chunk_kernel(TokenParams
     }
     g_all = g;
     g = 1.f;
-    for (int s = n - 1; s >= 0; --s) {
-      g_tail[s] = g;
-      g *= a[s];
-    }
-  }
-  __syncthreads();
-  // K K^T and Q K^T of the chunk: K and Q staged in X1 and X2 (rows past n
-  // zero), then register-tiled products, thread (ty, tx) = (tid / 8, tid % 8)
-  // owning rows 4 ty .. 4 ty + 3 and columns tx + 8 c (c < 16)
-  stage_rows<kChunkThreads>(X1, kLd, Kc, n, true);
-  stage_rows<kChunkThreads>(X2, kLd, Qc, n, true);
-  __syncthreads();
-  {
-    const int ty = tid >> 3, tx = tid & 7;
-    float acc[4][16];
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {  // pass 0: K K^T into X0; pass 1: Q K^T into X2
-      const float* Arows = pass == 0 ? X1 : X2;
-      tile_product4(acc, kD, [&](int t, int i) { return Arows[t * kLd + i]; },
-                    [&](int i, int s2) { return X1[s2 * kLd + i]; });
-      float* dst = pass == 0 ? X0 : X2;
-      if (pass == 1) __syncthreads();  // every thread is done reading Q out of X2
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) dst[(4 * ty + r) * kLd + tx + 8 * c2] = acc[r][c2];
-    }
-  }
-  __syncthreads();
-  // A (strictly lower part; the unit diagonal is implicit) and P, row t per
-  // thread: A[t][s] = w_t G[t][s] (K K^T)[t][s], P[t][s] = G[t][s] (Q K^T)[t][s]
-  if (tid < n) {
-    float g = 1.f;  // G[t][s], s going down from t - 1
-    for (int s2 = tid - 1; s2 >= 0; --s2) {
-      X0[tid * kLd + s2] *= w[tid] * g;
-      X2[tid * kLd + s2] *= g;
+    for (int s2 = n - 1; s2 >= 0; --s2) {
+      g_tail[s2] = g;
       g *= a[s2];
     }
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_holder, 512);
+  tile_from_f32(tK, p.kp + tok0 * kD, n);
+  tile_from_f32(tP, p.qp + tok0 * kD, n);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtl wc{abort_flag, p.err, p.wait_limit_ns};
+  const uint32_t aK = smem_u32(tK), aP = smem_u32(tP), a0 = smem_u32(R0), a1 = smem_u32(R1);
+  if (tid == 0) {  // K K^T and Q K^T
+    mma_tile(tmem, aK, false, aK, false);
+    mma_tile(tmem + 128, aP, false, aK, false);
+    mma_commit(&bars[0]);
+  }
+  bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[0], 0, wc));
+  const int t = tid;
+  if (ok) {
+    tc_fence_after();
+    // A[t][s] = w_t G[t][s] (K K^T)[t][s] (s < t) into F0, G[t][s] into F1
+    float v[128];
+    tmem_row128(tmem + lane_off, v);
+    float g = 1.f;
+    const float wt = t < n ? w[t] : 0.f;
+#pragma unroll
+    for (int s2 = kChunk - 1; s2 >= 0; --s2) {
+      if (s2 < t && t < n) {
+        F0[t * kLd + s2] = wt * g * v[s2];
+        F1[t * kLd + s2] = g;
+        g *= a[s2];
+      }
+    }
+    // P[t][s] = G[t][s] (Q K^T)[t][s] (s < t), bf16 over Q' (read by the MMA)
+    tmem_row128(tmem + 128 + lane_off, v);
+#pragma unroll
+    for (int s2 = 0; s2 < kChunk; ++s2) v[s2] = (s2 < t && t < n) ? v[s2] * F1[t * kLd + s2] : 0.f;
+    tile_row_bf16(tP, t, v);
   }
   __syncthreads();
-  // T = A^-1 by forward substitution, column j per thread (each thread reads
-  // and writes only its own column of T)
-  if (tid < n) {
+  // T = A^-1 (unit lower triangular) by forward substitution, column j per
+  // thread, into F1; each dot product runs as four interleaved partial sums
+  if (ok && tid < n) {
     const int j = tid;
     for (int i = 0; i < n; ++i) {
-      float x = i == j ? 1.f : 0.f;
-      if (i > j)
-        for (int k = j; k < i; ++k) x = fmaf(-X0[i * kLd + k], X1[k * kLd + j], x);
-      X1[i * kLd + j] = x;
+      float x0 = i == j ? 1.f : 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+      if (i > j) {
+        const float* ai = F0 + i * kLd;
+        int k = j;
+        for (; k + 3 < i; k += 4) {
+          x0 = fmaf(-ai[k], F1[k * kLd + j], x0);
+          x1 = fmaf(-ai[k + 1], F1[(k + 1) * kLd + j], x1);
+          x2 = fmaf(-ai[k + 2], F1[(k + 2) * kLd + j], x2);
+          x3 = fmaf(-ai[k + 3], F1[(k + 3) * kLd + j], x3);
+        }
+        for (; k < i; ++k) x0 = fmaf(-ai[k], F1[k * kLd + j], x0);
+      }
+      F1[i * kLd + j] = (x0 + x1) + (x2 + x3);
     }
   }
   __syncthreads();
-  // The rest as register-tiled products over shared memory (thread (ty, tx)
-  // owns rows 4 ty + r and columns tx + 8 c), rows past n kept at zero:
-  // W = T diag(w g_prev) K and U' = T diag(w) V (K, then V, staged in X0)
-  const int ty = tid >> 3, tx = tid & 7;
-  float acc[4][16];
-  const float* Vc2 = Vc;
-#pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    stage_rows<kChunkThreads>(X0, kLd, pass == 0 ? Kc : Vc2, n, true);
-    __syncthreads();
-    tile_product4(acc, n, [&](int t, int s2) { return X1[t * kLd + s2] * (pass == 0 ? w[s2] * g_prev[s2] : w[s2]); },
-                 [&](int s2, int jj) { return X0[s2 * kLd + jj]; });
-    float* dst = pass == 0 ? p.w : p.u;
+  // T1 = T diag(w g_prev), T2 = T diag(w) (rows t, columns s <= t < n) as bf16 tiles over A
+  if (ok) {
+    float v[128];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int t = 4 * ty + r;
-      if (t < n)
+    for (int s2 = 0; s2 < kChunk; ++s2) v[s2] = (s2 <= t && t < n) ? F1[t * kLd + s2] * w[s2] * g_prev[s2] : 0.f;
+    tile_row_bf16(R0, t, v);
 #pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) dst[(tok0 + t) * kD + tx + 8 * c2] = acc[r][c2];
-    }
-    __syncthreads();  // X0 is read; the next pass restages it
+    for (int s2 = 0; s2 < kChunk; ++s2) v[s2] = (s2 <= t && t < n) ? F1[t * kLd + s2] * w[s2] : 0.f;
+    tile_row_bf16(R0 + kTcTile, t, v);
   }
-  // W into X0, U' into X1 (T is done with)
-  stage_rows<kChunkThreads>(X0, kLd, p.w + tok0 * kD, n, true);
-  stage_rows<kChunkThreads>(X1, kLd, p.u + tok0 * kD, n, true);
+  __syncthreads();  // T is read: V' into its place
+  tile_from_f32(R1, p.vp + tok0 * kD, n);
+  fence_async_smem();
+  tc_fence_before();
   __syncthreads();
-  // Qt = diag(g_prev) Q - P W and Ot = P U' (P strictly lower)
+  if (ok && tid == 0) {  // W = T1 K', U' = T2 V' (K' and V' as MN-major B: rows s, columns d)
+    tc_fence_after();
+    mma_tile(tmem + 256, a0, false, aK, true);
+    mma_tile(tmem + 384, a0 + kTcTile, false, a1, true);
+    mma_commit(&bars[1]);
+  }
+  ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars[1], 0, wc));
+  if (ok) {  // row s of W and U': Wt, W over T1, T2; Ut, U' over V'
+    tc_fence_after();
+    const int s2 = tid;
+    const float gt = s2 < n ? g_tail[s2] : 0.f;
+    float v[128];
+    tmem_row128(tmem + 256 + lane_off, v);
+    tile_row_bf16(R0 + kTcTile, s2, v);
+#pragma unroll
+    for (int j = 0; j < kD; ++j) v[j] *= gt;
+    tile_row_bf16(R0, s2, v);
+    tmem_row128(tmem + 384 + lane_off, v);
+    tile_row_bf16(R1 + kTcTile, s2, v);
+#pragma unroll
+    for (int j = 0; j < kD; ++j) v[j] *= gt;
+    tile_row_bf16(R1, s2, v);
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (ok && tid == 0) {  // M' = K'^T Wt, N = K'^T Ut (K' as MN-major A), Qt' = P W, Ot = P U'
+    tc_fence_after();
+    mma_tile(tmem, aK, true, a0, true);
+    mma_tile(tmem + 128, aK, true, a1, true);
+    mma_tile(tmem + 256, aP, false, a0 + kTcTile, true);
+    mma_tile(tmem + 384, aP, false, a1 + kTcTile, true);
+    mma_commit(&bars[2]);
+  }
+  ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars[2], 0, wc));
+  if (ok) {
+    tc_fence_after();
+    const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
+    const int i = tid;
 #pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    const float* Bm = pass == 0 ? X0 : X1;
-    tile_product4(acc, n, [&](int t, int s2) { return s2 < t ? X2[t * kLd + s2] : 0.f; },
-                  [&](int s2, int jj) { return Bm[s2 * kLd + jj]; });
+    for (int part = 0; part < 4; ++part) {
+      float v[128];
+      tmem_row128(tmem + part * 128 + lane_off, v);
+      if (part < 2) {  // M (row i), N (row i)
+        float* dst = (part == 0 ? p.m : p.n) + mn0 + size_t(i) * kD;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int t = 4 * ty + r;
-      if (t < n) {
+        for (int j4 = 0; j4 < 32; ++j4) {
+          float4 o;
+          o.x = part == 0 ? ((i == 4 * j4 ? g_all : 0.f) - v[4 * j4]) : v[4 * j4];
+          o.y = part == 0 ? ((i == 4 * j4 + 1 ? g_all : 0.f) - v[4 * j4 + 1]) : v[4 * j4 + 1];
+          o.z = part == 0 ? ((i == 4 * j4 + 2 ? g_all : 0.f) - v[4 * j4 + 2]) : v[4 * j4 + 2];
+          o.w = part == 0 ? ((i == 4 * j4 + 3 ? g_all : 0.f) - v[4 * j4 + 3]) : v[4 * j4 + 3];
+          reinterpret_cast<float4*>(dst)[j4] = o;
+        }
+      } else if (t < n) {  // Qt (row t), Ot (row t)
+        float* dst = (part == 2 ? p.qt : p.ot) + (tok0 + t) * kD;
+        const float* q = p.qp + (tok0 + t) * kD;
+        const float gp = g_prev[t];
 #pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) {
-          const int jj = tx + 8 * c2;
-          if (pass == 0)
-            p.qt[(tok0 + t) * kD + jj] = g_prev[t] * Qc[size_t(t) * kD + jj] - acc[r][c2];
-          else
-            p.ot[(tok0 + t) * kD + jj] = acc[r][c2];
+        for (int j4 = 0; j4 < 32; ++j4) {
+          float4 o = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+          if (part == 2) {
+            const float4 q4 = reinterpret_cast<const float4*>(q)[j4];
+            o = make_float4(gp * q4.x - o.x, gp * q4.y - o.y, gp * q4.z - o.z, gp * q4.w - o.w);
+          }
+          reinterpret_cast<float4*>(dst)[j4] = o;
         }
       }
     }
-  }
-  __syncthreads();  // P is done with: K into X2
-  stage_rows<kChunkThreads>(X2, kLd, Kc, n, true);
-  __syncthreads();
-  // M = g_C I - Kt^T W and N = Kt^T U', Kt = diag(g_tail) K (rows i of the state)
-  const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
-#pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    const float* Bm = pass == 0 ? X0 : X1;
-    tile_product4(acc, n, [&](int i, int s2) { return g_tail[s2] * X2[s2 * kLd + i]; },
-                  [&](int s2, int jj) { return Bm[s2 * kLd + jj]; });
-    float* dst = pass == 0 ? p.m : p.n;
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int i = 4 * ty + r;
-#pragma unroll
-      for (int c2 = 0; c2 < 16; ++c2) {
-        const int jj = tx + 8 * c2;
-        dst[mn0 + size_t(i) * kD + jj] = pass == 0 ? ((i == jj ? g_all : 0.f) - acc[r][c2]) : acc[r][c2];
-      }
+  } else if (tid == 0) {  // MMAs in flight land before tensor memory is released
+    mma_commit(&bars[2]);
+    const uint64_t t_0 = global_timer_ns();
+    while (!mbar_try_wait(&bars[2], 0) && !mbar_try_wait(&bars[2], 1) && global_timer_ns() - t_0 < 10000000ull) {
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -438,10 +519,18 @@ __global__ void __launch_bounds__(kD) tok_state_kernel(TokenParams p) {
 #pragma unroll
     for (int jj = 0; jj < kSlab; ++jj) p.s_chunk[mn0 + size_t(i) * kD + j0 + jj] = Ss[i][jj];
     const float* mrow = Mbuf + (c & 1) * kD * kLd + i * kLd;
+#pragma unroll 4
     for (int k = 0; k < kD; ++k) {
       const float mv = mrow[k];
+      const float4* sk = reinterpret_cast<const float4*>(Ss[k]);  // row k of the slab: 4 broadcast loads
 #pragma unroll
-      for (int jj = 0; jj < kSlab; ++jj) acc[jj] = fmaf(mv, Ss[k][jj], acc[jj]);
+      for (int q = 0; q < kSlab / 4; ++q) {
+        const float4 s4 = sk[q];
+        acc[4 * q] = fmaf(mv, s4.x, acc[4 * q]);
+        acc[4 * q + 1] = fmaf(mv, s4.y, acc[4 * q + 1]);
+        acc[4 * q + 2] = fmaf(mv, s4.z, acc[4 * q + 2]);
+        acc[4 * q + 3] = fmaf(mv, s4.w, acc[4 * q + 3]);
+      }
     }
     __syncthreads();  // every row of the entering state and of M(c) is read
 #pragma unroll
@@ -518,7 +607,7 @@ cudaError_t launch_token_level(const TokenParams& p, bool with_out, cudaStream_t
   static unsigned done_chunk = 0, done_out = 0, done_maps = 0;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(tok_maps_kernel), kMapsSmem, &done_maps);
   if (e != cudaSuccess) return e;
-  e = ensure_smem_attr(reinterpret_cast<const void*>(tok_chunk_kernel), int(kChunkSmem), &done_chunk);
+  e = ensure_smem_attr(reinterpret_cast<const void*>(tok_chunk_tc_kernel), kTcSmem, &done_chunk);
   if (e != cudaSuccess) return e;
   e = ensure_smem_attr(reinterpret_cast<const void*>(tok_out_kernel), kOutSmem, &done_out);
   if (e != cudaSuccess) return e;
@@ -527,7 +616,7 @@ cudaError_t launch_token_level(const TokenParams& p, bool with_out, cudaStream_t
   if (e != cudaSuccess) return e;
   const unsigned bh = unsigned(p.B) * unsigned(p.H);
   tok_maps_kernel<<<bh * unsigned(p.n_chunks), kD, kMapsSmem, st>>>(p);
-  tok_chunk_kernel<<<bh * unsigned(p.n_chunks), kChunkThreads, kChunkSmem, st>>>(p);
+  tok_chunk_tc_kernel<<<bh * unsigned(p.n_chunks), kD, kTcSmem, st>>>(p);
   tok_state_kernel<<<bh * unsigned(kD / kSlab), kD, kStateSmem, st>>>(p);
   if (with_out) tok_out_kernel<<<bh * unsigned(p.n_chunks), kD, kOutSmem, st>>>(p);
   return cudaGetLastError();
