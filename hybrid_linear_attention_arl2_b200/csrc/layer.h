@@ -42,7 +42,7 @@ struct TokenParams {
   float corr;
   int B, L, H, n_chunks;
   float *qp, *kp, *vp, *w, *u, *qt, *ot;  // [B, H, L, 128]
-  float *m, *n, *s_chunk;                 // [B, H, n_chunks, 128, 128]
+  float *m, *n, *s_chunk;                 // [B, H, n_chunks, 128, 128] (m holds each chunk's M transposed)
   const float* s_in;
   float* s_out;
   __nv_bfloat16* o;

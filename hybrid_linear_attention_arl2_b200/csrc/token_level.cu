@@ -442,17 +442,15 @@ __global__ void __launch_bounds__(kD, 1) tok_chunk_tc_kernel(TokenParams p) {
     for (int part = 0; part < 4; ++part) {
       float v[128];
       tmem_row128(tmem + part * 128 + lane_off, v);
-      if (part < 2) {  // M (row i), N (row i)
-        float* dst = (part == 0 ? p.m : p.n) + mn0 + size_t(i) * kD;
+      if (part == 0) {  // M, stored transposed (column i of M^T per thread: coalesced)
+        float* dst = p.m + mn0 + i;
 #pragma unroll
-        for (int j4 = 0; j4 < 32; ++j4) {
-          float4 o;
-          o.x = part == 0 ? ((i == 4 * j4 ? g_all : 0.f) - v[4 * j4]) : v[4 * j4];
-          o.y = part == 0 ? ((i == 4 * j4 + 1 ? g_all : 0.f) - v[4 * j4 + 1]) : v[4 * j4 + 1];
-          o.z = part == 0 ? ((i == 4 * j4 + 2 ? g_all : 0.f) - v[4 * j4 + 2]) : v[4 * j4 + 2];
-          o.w = part == 0 ? ((i == 4 * j4 + 3 ? g_all : 0.f) - v[4 * j4 + 3]) : v[4 * j4 + 3];
-          reinterpret_cast<float4*>(dst)[j4] = o;
-        }
+        for (int k = 0; k < kD; ++k) dst[size_t(k) * kD] = (i == k ? g_all : 0.f) - v[k];
+      } else if (part == 1) {  // N (row i)
+        float* dst = p.n + mn0 + size_t(i) * kD;
+#pragma unroll
+        for (int j4 = 0; j4 < 32; ++j4)
+          reinterpret_cast<float4*>(dst)[j4] = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
       } else if (t < n) {  // Qt (row t), Ot (row t)
         float* dst = (part == 2 ? p.qt : p.ot) + (tok0 + t) * kD;
         const float* q = p.qp + (tok0 + t) * kD;
@@ -488,22 +486,24 @@ __global__ void __launch_bounds__(kD, 1) tok_chunk_tc_kernel(TokenParams p) {
 // Each chunk's M is copied into one of two shared-memory buffers with
 // asynchronous copies issued a chunk ahead, so the copy of chunk c + 1 runs
 // while chunk c computes.
-constexpr int kStateSmem = (2 * kD * kLd + kD * kSlab) * int(sizeof(float));
+constexpr int kStateSmem = (2 * kD * kD + kD * kSlab) * int(sizeof(float));
 
-__device__ __forceinline__ void copy_async_m(float* dst, const float* src) {  // [128][128] f32 into pitch kLd
+// M^T of a chunk ([128][128] f32, row k = column k of M) into shared memory
+// with 16-byte asynchronous copies.
+__device__ __forceinline__ void copy_async_m(float* dst, const float* src) {
   const int tid = threadIdx.x;
 #pragma unroll 8
-  for (int x = tid; x < kD * kD; x += kD) {
-    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst + (x >> 7) * kLd + (x & 127)));
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src + x) : "memory");
+  for (int x = tid; x < kD * kD / 4; x += kD) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst + 4 * x));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + 4 * x) : "memory");
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(kD) tok_state_kernel(TokenParams p) {
   extern __shared__ float st_sm[];
-  float* Mbuf = st_sm;                                                              // [2][kD][kLd]
-  float(*Ss)[kSlab] = reinterpret_cast<float(*)[kSlab]>(st_sm + 2 * kD * kLd);  // [kD][kSlab]
+  float* Mbuf = st_sm;                                                             // [2][kD][kD]: M^T
+  float(*Ss)[kSlab] = reinterpret_cast<float(*)[kSlab]>(st_sm + 2 * kD * kD);  // [kD][kSlab]
   const int slab = blockIdx.x % (kD / kSlab), bh = blockIdx.x / (kD / kSlab);
   const int i = threadIdx.x, j0 = slab * kSlab;
   for (int jj = 0; jj < kSlab; ++jj) Ss[i][jj] = p.s_in[(size_t(bh) * kD + i) * kD + j0 + jj];
@@ -515,13 +515,13 @@ __global__ void __launch_bounds__(kD) tok_state_kernel(TokenParams p) {
     for (int jj = 0; jj < kSlab; ++jj) acc[jj] = p.n[mn0 + size_t(i) * kD + j0 + jj];
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();  // M(c) in; the previous step's state rows are all written
-    if (c + 1 < p.n_chunks) copy_async_m(Mbuf + ((c + 1) & 1) * kD * kLd, p.m + mn0 + kD * kD);
+    if (c + 1 < p.n_chunks) copy_async_m(Mbuf + ((c + 1) & 1) * kD * kD, p.m + mn0 + kD * kD);
 #pragma unroll
     for (int jj = 0; jj < kSlab; ++jj) p.s_chunk[mn0 + size_t(i) * kD + j0 + jj] = Ss[i][jj];
-    const float* mrow = Mbuf + (c & 1) * kD * kLd + i * kLd;
+    const float* mcol = Mbuf + (c & 1) * kD * kD + i;  // M[i][k] = M^T[k][i]: conflict-free across threads
 #pragma unroll 4
     for (int k = 0; k < kD; ++k) {
-      const float mv = mrow[k];
+      const float mv = mcol[k * kD];
       const float4* sk = reinterpret_cast<const float4*>(Ss[k]);  // row k of the slab: 4 broadcast loads
 #pragma unroll
       for (int q = 0; q < kSlab / 4; ++q) {
