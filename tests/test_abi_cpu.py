@@ -137,3 +137,21 @@ def test_token_level_calls_host_validation(lib):
     assert lib.arl2_token_query(None, 16, 16, 16, 16, 16, 32, None) == 1
     assert lib.arl2_token_commit(None, 16, 16, 16, 16, 16, 32, None) == 1
     assert lib.arl2_token_commit(12345, 16, 16, 16, 16, 16, 32, None) == 1
+
+
+def test_gemm_host_validation(lib):
+    """The projection GEMM rejects bad pointers, sizes and leading dimensions
+    before any CUDA call; an empty product returns at once."""
+    a, b, c = 1 << 20, 2 << 20, 3 << 20   # 16-byte-aligned, disjoint fake addresses, never dereferenced
+    g = lib.arl2_gemm_bf16
+    assert g(None, 64, b, 64, c, 64, 32, 64, 64, None) == 1
+    assert g(a, 64, b, 64, None, 64, 32, 64, 64, None) == 1
+    assert g(a + 8, 64, b, 64, c, 64, 32, 64, 64, None) == 1          # misaligned A
+    assert g(a, 64, b, 64, c, 64, -1, 64, 64, None) == 1              # negative size
+    assert g(a, 32, b, 64, c, 64, 32, 64, 64, None) == 1              # lda < k
+    assert g(a, 64, b, 32, c, 64, 32, 64, 64, None) == 1              # ldb < n
+    assert g(a, 64, b, 64, c, 60, 32, 64, 64, None) == 1              # ldc < n
+    assert g(a, 68, b, 64, c, 64, 32, 64, 64, None) == 1              # lda not a multiple of 8
+    assert g(a, 64, b, 64, a + 64, 64, 32, 64, 64, None) == 1         # C overlaps A
+    assert g(a, 64, b, 64, c, 64, 0, 64, 64, None) == 0               # empty: nothing to do
+    assert g(a, 64, b, 64, c, 64, 32, 0, 64, None) == 0
