@@ -60,6 +60,12 @@ def _args():
     return ap.parse_args()
 
 
+def state_launches(cfg: W.Config) -> int:
+    """Kernels of one commit's state write: one cluster launch when the frame's
+    chunks fit one cluster (at most 16 chunks of 128 tokens), else three."""
+    return 1 if -(-cfg.tokens // 128) <= 16 else 3
+
+
 # ------------------------------------------------------------------ flop / byte accounting
 def frame_flops(cfg: W.Config) -> dict:
     """Algorithmic flops of one frame of one hybrid layer (all streams)."""
@@ -266,25 +272,29 @@ def run_arl2(args, rank: int, world: int):
     with torch.cuda.stream(stream):
         layer = arl2.HybridLayer(B, H, d, L, arl2.ARL2_BF16, *ds.phi, corr_scale=cfg.corr_scale, stream=stream)
         O = torch.empty((B, L, H, d), dtype=torch.bfloat16, device=device)
-        period = 4  # frames per graph: pool phase (20 passes) and state ping-pong both repeat
-        gate_a = [torch.empty((B, H), dtype=torch.float32, device=device) for _ in range(period)]
-        gate_b = [torch.empty((B, H, L), dtype=torch.float32, device=device) for _ in range(period)]
-        # every frame's gates staged on the device before any timing: the timed
-        # loop only copies them into the per-slot buffers the graph reads
+        # frames per graph: the pool phase (20 passes = 4 frames) and the
+        # state ping-pong (2 frames) both return to their start after it
+        period = 20
+        # every frame's gates staged on the device before any timing: before
+        # each graph replay two copies move the next `period` frames' gates
+        # into the slots the graph reads (rows padded to 16 bytes)
+        na, nb = -(-B * H // 4) * 4, B * H * L
         n_frames = args.warmup + args.steps + 2 * period
-        ga_all = torch.empty((n_frames, B, H), dtype=torch.float32, device=device)
-        gb_all = torch.empty((n_frames, B, H, L), dtype=torch.float32, device=device)
+        ga_all = torch.zeros((n_frames, na), dtype=torch.float32, device=device)
+        gb_all = torch.empty((n_frames, nb), dtype=torch.float32, device=device)
         for f in range(n_frames):
             a, b = ds.gates(f)
-            ga_all[f].copy_(torch.from_numpy(a))
-            gb_all[f].copy_(torch.from_numpy(b))
+            ga_all[f, :B * H].copy_(torch.from_numpy(a).reshape(-1))
+            gb_all[f].copy_(torch.from_numpy(b).reshape(-1))
+        gate_a = torch.empty((period, na), dtype=torch.float32, device=device)
+        gate_b = torch.empty((period, nb), dtype=torch.float32, device=device)
 
-        def load_gates(frame):
-            slot = frame % period
-            gate_a[slot].copy_(ga_all[frame], non_blocking=True)
-            gate_b[slot].copy_(gb_all[frame], non_blocking=True)
+        def load_gates(frame, n):
+            """Gates of frames frame .. frame + n - 1 into slots 0 .. n - 1."""
+            gate_a[:n].copy_(ga_all[frame:frame + n], non_blocking=True)
+            gate_b[:n].copy_(gb_all[frame:frame + n], non_blocking=True)
 
-        def frame_calls(frame, ev=None):
+        def frame_calls(frame, slot, ev=None):
             for p in range(cfg.passes):
                 q, k, v = ds.triple(frame, p)
                 if p < cfg.queries:
@@ -294,38 +304,44 @@ def run_arl2(args, rank: int, world: int):
                     if ev is not None:
                         ev[p][1].record(stream)
                 else:
-                    slot = frame % period
-                    arl2.arl2_frame_commit(layer.handle, q, k, v, gate_a[slot], gate_b[slot], O, stream)
+                    arl2.arl2_frame_commit(layer.handle, q, k, v, gate_a[slot, :B * H], gate_b[slot], O, stream)
 
         # warm-up (eager): also exercises every kernel once before any capture
         for f in range(args.warmup):
-            load_gates(f)
-            frame_calls(f)
+            load_gates(f, 1)
+            frame_calls(f, 0)
         stream.synchronize()
         err = layer.last_error()
         if err:
             raise RuntimeError(f"device error during warm-up: {arl2.STATUS.get(err)}")
 
         use_graphs = not args.no_graphs
-        graphs = None
-        if use_graphs:
-            # One graph = `period` frames; the handle's ping-pong parity and the
-            # pool phase both return to their start after it.
-            start = args.warmup
-            graph = torch.cuda.CUDAGraph()
-            for f in range(start, start + period):
-                load_gates(f)
+        base = args.warmup
+        n_rep, n_tail = divmod(args.steps, period) if use_graphs else (0, args.steps)
+        if n_rep:
+            # Two graphs of the same `period` frames: `graph` carries no event
+            # nodes (an event node between two attention launches orders them
+            # fully, so they could not overlap set-up and tail); `graph_ev`
+            # adds external events (event-record nodes) around the first
+            # frame's query launches and runs as the last replay of the timed
+            # region, where it times them on the launching stream.
+            graph, graph_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            ev_q = [(torch.cuda.Event(enable_timing=True, external=True),
+                     torch.cuda.Event(enable_timing=True, external=True))
+                    for _ in range(cfg.queries)]
             stream.synchronize()
-            # external events become event-record nodes of the graph: they time
-            # every query launch of each replay on the launching stream
-            graph_ev = [(torch.cuda.Event(enable_timing=True, external=True),
-                         torch.cuda.Event(enable_timing=True, external=True))
-                        for _ in range(period * cfg.queries)]
-            with torch.cuda.graph(graph, stream=stream):
-                for i, f in enumerate(range(start, start + period)):
-                    frame_calls(f, graph_ev[i * cfg.queries:(i + 1) * cfg.queries])
-            graphs = graph
+            for g, evs in ((graph, None), (graph_ev, ev_q)):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(period):
+                        frame_calls(base + i, i, evs if i == 0 else None)
+            # one untimed replay of each (its upload and first run)
+            for g in (graph, graph_ev):
+                load_gates(base, period)
+                g.replay()
             stream.synchronize()
+            err = layer.last_error()
+            if err:
+                raise RuntimeError(f"device error in the graph warm-up: {arl2.STATUS.get(err)}")
 
         clocks = ClockSampler(local)
         if dist is not None:
@@ -335,30 +351,20 @@ def run_arl2(args, rank: int, world: int):
         clocks.start()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
-        attn_ev = []
-        f = args.warmup
-        if use_graphs:
-            # kernel timing: attention-only events around one captured query per graph replay
-            t0.record(stream)
-            steps_done = 0
-            while steps_done < args.steps:
-                for j in range(period):
-                    load_gates(f + j)
-                graphs.replay()
-                f += period
-                steps_done += period
-            t1.record(stream)
-        else:
-            t0.record(stream)
-            for s in range(args.steps):
-                load_gates(f)
-                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                      for _ in range(cfg.queries)]
-                frame_calls(f, ev)
-                attn_ev.extend(ev)
-                f += 1
-            t1.record(stream)
-            steps_done = args.steps
+        f = base
+        tail_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(cfg.queries * max(n_tail, 1))]
+        t0.record(stream)
+        for r in range(n_rep):
+            load_gates(f, period)
+            (graph_ev if r == n_rep - 1 else graph).replay()
+            f += period
+        for j in range(n_tail):  # eager frames: exactly `steps` frames in all
+            load_gates(f, 1)
+            frame_calls(f, 0, tail_ev[j * cfg.queries:(j + 1) * cfg.queries])
+            f += 1
+        t1.record(stream)
+        steps_done = n_rep * period + n_tail
         t1.synchronize()
         clk = clocks.stop()
         ms = t0.elapsed_time(t1)
@@ -366,9 +372,9 @@ def run_arl2(args, rank: int, world: int):
         if err:
             raise RuntimeError(f"device error in the timed region: {arl2.STATUS.get(err)}")
 
-        # dominant-kernel duration: the query launches of the last graph replay
-        if use_graphs:
-            attn_ev = graph_ev
+        # dominant-kernel duration: the query launches timed in the timed
+        # region (the evented replay's first frame, else the eager frames)
+        attn_ev = ev_q if n_rep else tail_ev[:cfg.queries * n_tail]
         attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
         attn_avg_ms = float(np.mean(attn_ms))
 
@@ -377,7 +383,7 @@ def run_arl2(args, rank: int, world: int):
 
     result = {
         "value": value, "ms_per_step": ms_per_step, "steps": steps_done, "clocks": clk,
-        "attn_avg_ms": attn_avg_ms, "flops": flops, "launches_per_step": cfg.queries + 1 + 3,
+        "attn_avg_ms": attn_avg_ms, "flops": flops, "launches_per_step": cfg.queries + 1 + state_launches(cfg),
     }
     if args.config == 2 and not args.profile_small:
         result["flatness"] = long_stream_flatness(cfg, ds, device, rank)
@@ -526,7 +532,8 @@ def run_block(args, rank: int, world: int) -> dict:
     """The hybrid attention block on the single-layer shape (B=1, H=12, d=128,
     L=1560, hidden 1536): per pass X -> Q, K, V (tcgen05 GEMM) -> hybrid layer -> O W_o;
     the commit also forms its gates from X.  Inputs cycle through 40 seeded
-    token matrices (192 MB > L2); CUDA graphs of four frames, as the layer's run."""
+    token matrices (192 MB > L2); each CUDA graph holds eight frames, the pool's
+    whole cycle, so that every replay reads all 40."""
     import dataclasses
     import torch
     from hybrid_linear_attention_arl2_b200 import arl2
@@ -543,7 +550,7 @@ def run_block(args, rank: int, world: int) -> dict:
     # pool entry i is the tokens of pass i % 5 of frame i // 5
     xs = [to(wl.block_input(0, i // cfg.passes, i % cfg.passes)) for i in range(cfg.pool)]
     stream = torch.cuda.Stream(device)
-    period = 4
+    period = cfg.pool // cfg.passes  # frames per graph: one pass over the pool
     with torch.cuda.stream(stream):
         blk = arl2.HybridBlock(B, H, L, *weights, *phi, corr_scale=cfg.corr_scale, stream=stream)
         Y = torch.empty_like(xs[0])
@@ -563,16 +570,19 @@ def run_block(args, rank: int, world: int) -> dict:
         with torch.cuda.graph(graph, stream=stream):
             for f in range(period):
                 frame(f)
+        graph.replay()  # untimed: the graph's upload and first run
         stream.synchronize()
+        n_rep, n_tail = divmod(args.steps, period)
         clocks = ClockSampler(local)
         torch.cuda.synchronize()
         clocks.start()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        steps = 0
-        while steps < args.steps:
+        for _ in range(n_rep):
             graph.replay()
-            steps += period
+        for f in range(n_tail):  # eager frames: exactly `steps` frames in all
+            frame(f)
+        steps = n_rep * period + n_tail
         t1.record(stream)
         t1.synchronize()
         clk = clocks.stop()
@@ -736,7 +746,7 @@ def run_stack(args, rank: int, world: int) -> dict:
     return {"frames": F, "ms_total": total, "ms_hybrid": t_h, "ms_kv": t_k, "clocks": clk,
             "hybrid_tflops": hyb_flops / (t_h / 1e3) / 1e12, "kv_tflops": kv_flops / (t_k / 1e3) / 1e12,
             "stack_tflops": (hyb_flops + kv_flops) / (total / 1e3) / 1e12, "flops": hyb_flops + kv_flops,
-            "launches": F * cfg.passes * (nh + (nl - nh)) + F * nh * 3}
+            "launches": F * cfg.passes * (nh + (nl - nh)) + F * nh * state_launches(cfg)}
 
 
 # ------------------------------------------------------------------ CPU oracle baseline

@@ -767,7 +767,6 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(&bars[i], count);
     }
     *abort_flag = fits ? 0 : 1;
-    if (!fits) record_error(p.err, kDevBadShape);
     fence_barrier_init();
   }
   if (warp == 2) tmem_alloc_pair(tmem_holder, 512);
@@ -775,6 +774,13 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   __syncthreads();
   cluster_barrier();  // both CTAs' barriers initialised before any remote arrive or load
   tc_fence_after();
+  // The set-up above touches only this pair's shared and tensor memory, so it
+  // may overlap the kernel before this one on the stream; every global access
+  // below follows that kernel's completion.  The next launch of this kernel may
+  // then be scheduled on the SMs this grid frees as its CTAs finish.
+  grid_dependency_wait();
+  allow_dependent_launch();
+  if (threadIdx.x == 0 && !fits) record_error(p.err, kDevBadShape);
   const uint32_t tmem = *tmem_holder;
   const WaitCtl w{abort_flag, p.err, p.wait_limit_ns};
   const int wg = warp >> 2;
@@ -865,6 +871,14 @@ cudaError_t launch_attn_pair(const CUtensorMap& tq, const CUtensorMap& tk, const
     capacity = n;
   }
   if (p.grid / 2 > capacity) return cudaErrorCooperativeLaunchTooLarge;
+  // Programmatic stream serialisation: the grid may be scheduled before the
+  // kernel ahead of it on the stream has finished (the kernel waits for it
+  // before any global access), which hides this launch's set-up.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, attn_pair_kernel, tq, tk, tv, tmq, tmo, p);
 }
 

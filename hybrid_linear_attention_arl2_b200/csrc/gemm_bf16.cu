@@ -77,7 +77,6 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   if (threadIdx.x == 0) {
     for (int i = 0; i < G_COUNT; ++i) mbar_init(&bars[i], (i == G_AE || i == G_AE + 1) ? 8u : 1u);
     *abort_flag = fits ? 0 : 1;
-    if (!fits) record_error(p.err, kDevBadShape);
     fence_barrier_init();
   }
   if (warp == 2) tmem_alloc_pair(tmem_holder, 512);
@@ -85,6 +84,11 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   __syncthreads();
   cluster_barrier();  // both CTAs' barriers initialised before any remote arrive or load
   tc_fence_after();
+  // The set-up above may overlap the kernel before this one on the stream;
+  // every global access below follows its completion.
+  grid_dependency_wait();
+  allow_dependent_launch();
+  if (threadIdx.x == 0 && !fits) record_error(p.err, kDevBadShape);
   const uint32_t tmem = *tmem_holder;
   const WaitCtl w{abort_flag, p.err, p.wait_limit_ns};
   const int tiles_m = (p.M + 2 * kBM - 1) / (2 * kBM), tiles_n = (p.N + 2 * kBN - 1) / (2 * kBN);
@@ -272,6 +276,13 @@ cudaError_t gemm_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, vo
   (void)sms;
   const int pairs = tiles < cap ? tiles : cap;
   cfg.gridDim = dim3(2 * pairs);
+  // programmatic stream serialisation: the grid's set-up may overlap the
+  // previous kernel's tail (the kernel waits for it before any global access)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, gemm_bf16_kernel, ta, tb, tc, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

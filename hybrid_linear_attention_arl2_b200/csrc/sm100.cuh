@@ -43,6 +43,16 @@ __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may be scheduled while the kernel before it on the stream is
+// still running: grid_dependency_wait() returns once that kernel has completed
+// and its memory is visible (at once when nothing precedes it), so every global
+// read or write of such a kernel comes after it.  allow_dependent_launch() lets
+// the next such kernel be scheduled before this one ends; that kernel still
+// waits for this grid's completion before it touches global memory.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
