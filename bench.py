@@ -295,14 +295,15 @@ def run_arl2(args, rank: int, world: int):
             gate_b[:n].copy_(gb_all[frame:frame + n], non_blocking=True)
 
         def frame_calls(frame, slot, ev=None):
+            """One frame; `ev` = (start, end) events around its query launches."""
             for p in range(cfg.passes):
                 q, k, v = ds.triple(frame, p)
                 if p < cfg.queries:
-                    if ev is not None:
-                        ev[p][0].record(stream)
+                    if ev is not None and p == 0:
+                        ev[0].record(stream)
                     arl2.arl2_frame_query(layer.handle, q, k, v, O, stream)
-                    if ev is not None:
-                        ev[p][1].record(stream)
+                    if ev is not None and p == cfg.queries - 1:
+                        ev[1].record(stream)
                 else:
                     arl2.arl2_frame_commit(layer.handle, q, k, v, gate_a[slot, :B * H], gate_b[slot], O, stream)
 
@@ -322,18 +323,19 @@ def run_arl2(args, rank: int, world: int):
             # Two graphs of the same `period` frames: `graph` carries no event
             # nodes (an event node between two attention launches orders them
             # fully, so they could not overlap set-up and tail); `graph_ev`
-            # adds external events (event-record nodes) around the first
-            # frame's query launches and runs as the last replay of the timed
-            # region, where it times them on the launching stream.
+            # adds external events (event-record nodes) before the first frame's
+            # first query launch and after its last, and runs as the last
+            # replay of the timed region: the span of its back-to-back query
+            # launches on the launching stream, divided by their number, is the
+            # attention kernel's average launch duration.
             graph, graph_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
             ev_q = [(torch.cuda.Event(enable_timing=True, external=True),
-                     torch.cuda.Event(enable_timing=True, external=True))
-                    for _ in range(cfg.queries)]
+                     torch.cuda.Event(enable_timing=True, external=True))]
             stream.synchronize()
             for g, evs in ((graph, None), (graph_ev, ev_q)):
                 with torch.cuda.graph(g, stream=stream):
                     for i in range(period):
-                        frame_calls(base + i, i, evs if i == 0 else None)
+                        frame_calls(base + i, i, evs[0] if evs and i == 0 else None)
             # one untimed replay of each (its upload and first run)
             for g in (graph, graph_ev):
                 load_gates(base, period)
@@ -353,7 +355,7 @@ def run_arl2(args, rank: int, world: int):
         t1 = torch.cuda.Event(enable_timing=True)
         f = base
         tail_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(cfg.queries * max(n_tail, 1))]
+                   for _ in range(max(n_tail, 1))]
         t0.record(stream)
         for r in range(n_rep):
             load_gates(f, period)
@@ -361,7 +363,7 @@ def run_arl2(args, rank: int, world: int):
             f += period
         for j in range(n_tail):  # eager frames: exactly `steps` frames in all
             load_gates(f, 1)
-            frame_calls(f, 0, tail_ev[j * cfg.queries:(j + 1) * cfg.queries])
+            frame_calls(f, 0, tail_ev[j])
             f += 1
         t1.record(stream)
         steps_done = n_rep * period + n_tail
@@ -374,9 +376,8 @@ def run_arl2(args, rank: int, world: int):
 
         # dominant-kernel duration: the query launches timed in the timed
         # region (the evented replay's first frame, else the eager frames)
-        attn_ev = ev_q if n_rep else tail_ev[:cfg.queries * n_tail]
-        attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
-        attn_avg_ms = float(np.mean(attn_ms))
+        attn_ev = ev_q if n_rep else tail_ev[:n_tail]
+        attn_avg_ms = float(np.mean([a.elapsed_time(b) for a, b in attn_ev])) / cfg.queries
 
     value, ms_max = whole_job_rate(ms, steps_done, world, dist, device)
     ms_per_step = ms_max / steps_done
@@ -780,9 +781,8 @@ def cpu_oracle_rate(cfg: W.Config, budget_s: float = 12.0, sample_note=True):
 # launch on the single-hybrid-layer-bf16 workload, from one ncu capture of
 # `bench.py --profile-small --no-graphs`; reported only while the kernel sources
 # hash to the value the capture was taken on (None: not captured yet).
-# (Captured on the build before the long-key-range schedule was added; the
-# device code and the schedule of this workload are unchanged since.)
-ATTN_TRAFFIC = {"bytes": 14850560 + 0, "sources_sha256": "5858c7523edecb3839a85a96568c74214588058c2ce9acb049bfe1ab105c27d0",
+ATTN_TRAFFIC = {"bytes": 14858496 + 0, "sources_sha256": "073e8cc8da1853c5d02213298f39ac670ad1622e57c8c0903217f535b09e51fc",
+                "workload": "single-hybrid-layer-bf16",
                 "capture": "profiles/attn_pair_kernel_single-hybrid-layer-bf16.md"}
 ATTN_SOURCES = ("hybrid_linear_attention_arl2_b200/csrc/attn_pair.cu",
                 "hybrid_linear_attention_arl2_b200/csrc/sm100.cuh",
@@ -798,10 +798,11 @@ def attn_sources_sha256() -> str:
     return h.hexdigest()
 
 
-def attn_traffic():
+def attn_traffic(workload: str):
+    """DRAM bytes of one attention launch, for the captured workload only."""
     if ATTN_TRAFFIC["bytes"] is None or ATTN_TRAFFIC["sources_sha256"] != attn_sources_sha256():
         return None
-    return ATTN_TRAFFIC["bytes"]
+    return ATTN_TRAFFIC["bytes"] if workload == ATTN_TRAFFIC["workload"] else None
 
 
 def peaks():
@@ -960,7 +961,7 @@ def main():
         "pct_bf16_peak": {"value": 100.0 * frame_tflops / peak_burst, "basis": f"burst bf16 {src}",
                           "sustained_basis": 100.0 * frame_tflops / peak_sus},
         "roofline": {"bound": "tensor", "kernel": "attn_pair_kernel", "achieved": attn_tflops, "peak": peak_burst,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak_burst, "traffic": attn_traffic(),
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak_burst, "traffic": attn_traffic(cfg.name),
                      "peak_basis": f"bf16_tflops (burst) {src}",
                      "frac_vs_sustained": attn_tflops / peak_sus},
         "clocks": res["clocks"],
