@@ -24,6 +24,7 @@ STATUS = {
     0: "ARL2_OK", 1: "ARL2_ERR_INVALID_ARGUMENT", 2: "ARL2_ERR_UNSUPPORTED",
     3: "ARL2_ERR_OUT_OF_MEMORY", 4: "ARL2_ERR_CUDA", 5: "ARL2_ERR_TIMEOUT", 6: "ARL2_ERR_NO_DEVICE",
     7: "ARL2_ERR_SCRATCH_LIMIT",
+    8: "ARL2_ERR_BOUNDS",
 }
 ARL2_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -79,6 +80,7 @@ _SIGS = {
     "arl2_attn_partition": (_I32, [_I32, _I32, _I32, _I32, _I32, _VP, _I32, _VP, _VP, _VP]),
     "arl2_status_string": (ctypes.c_char_p, [_I32]),
     "arl2_abi_version": (_I32, []),
+    "arl2_debug_bounds_enabled": (_I32, []),
 }
 
 _lib = None
@@ -309,6 +311,11 @@ def arl2_status_string(status: int) -> str:
 
 def arl2_abi_version() -> int:
     return load_library().arl2_abi_version()
+
+
+def arl2_debug_bounds_enabled() -> bool:
+    """Whether the loaded library is the debug build (index checks in its kernels)."""
+    return bool(load_library().arl2_debug_bounds_enabled())
 
 
 # ---------------------------------------------------------------- convenience wrappers

@@ -229,6 +229,7 @@ arl2_status prepare_readout(arl2_state* h, cudaStream_t st) {
   StateParams sp{};
   sp.mqt = mqt_slot(h, h->cur);
   sp.heads = h->cfg.heads;
+  sp.batch = h->cfg.batch;
   sp.err = h->err;
   sp.wait_limit_ns = h->wait_ns;
   ARL2_TRY(launch_readout_prep(h->tm_s_bf, h->tm_phiq, sp, h->cfg.batch, st));
@@ -314,11 +315,20 @@ const char* arl2_status_string(arl2_status s) {
     case ARL2_ERR_TIMEOUT: return "device-side wait timed out";
     case ARL2_ERR_NO_DEVICE: return "no CUDA device";
     case ARL2_ERR_SCRATCH_LIMIT: return "sizes exceed the fixed scratch of the allocation-free state write";
+    case ARL2_ERR_BOUNDS: return "a kernel index check failed (debug build)";
   }
   return "unknown status";
 }
 
 int32_t arl2_abi_version(void) { return 1; }
+
+int32_t arl2_debug_bounds_enabled(void) {
+#ifdef ARL2_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 arl2_status arl2_state_init(const arl2_config* cfg, const void* phi_q, const void* phi_k, const void* phi_v,
                             void* stream, arl2_state_t* out) {
@@ -514,6 +524,7 @@ arl2_status layer_commit_ld(arl2_state* h, const void* q, const void* k, const v
     sp.mqt = mqt_slot(h, nxt);
     sp.L = c.tokens_per_frame;
     sp.heads = c.heads;
+    sp.batch = c.batch;
     sp.n_chunks = h->n_chunks;
     sp.corr = h->corr;
     sp.err = h->err;
@@ -1036,6 +1047,7 @@ extern "C" arl2_status arl2_state_write_noalloc(const arl2_config* cfg, const vo
   sp.mqt = nullptr;
   sp.L = L;
   sp.heads = H;
+  sp.batch = B;
   sp.n_chunks = n_chunks;
   sp.corr = cfg->corr_scale < 0.f ? 1.f / float(L) : cfg->corr_scale;
   sp.err = dev_error;

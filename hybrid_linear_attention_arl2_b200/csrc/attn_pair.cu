@@ -117,6 +117,13 @@ __device__ __forceinline__ bool next_seg(const AttnParams& p, unsigned& u, unsig
   s.blk = int(e.y & 1023u);
   s.j0 = int((e.y >> 10) & 2047u);
   s.j1 = s.j0 + int(e.y >> 21);
+  // (debug build) the segment lies inside the problem and the pairs whose
+  // pieces it merges are pairs of this launch; every role decodes the same
+  // list, so all of them stop at the same segment
+  if (!ARL2_IN_BOUNDS(p.err, s.blk < p.n_blk && s.j0 < s.j1 && s.j1 <= p.nkv && s.n_contrib <= kMaxContrib &&
+                                 2 * (int(blockIdx.x >> 1) + s.n_contrib) + 1 < p.grid &&
+                                 (long long)(s.bh + 1) * p.n_blk * p.nkv <= p.total_units))
+    return false;
   return true;
 }
 
@@ -752,7 +759,11 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int cta = blockIdx.x;
   const int rank = int(cluster_ctarank());
   const int pair = cta >> 1;
-  const unsigned u_begin = p.seg_first[pair], u_end = p.seg_first[pair + 1];
+  // (debug build) the pair's segment list lies inside the launch's list
+  const bool pair_ok = ARL2_CHECKED(int(gridDim.x) == p.grid && p.grid <= kAttnMaxGrid);
+  const unsigned u_begin = pair_ok ? p.seg_first[pair] : 0u, u_end = pair_ok ? p.seg_first[pair + 1] : 0u;
+  const bool segs_ok =
+      pair_ok && ARL2_CHECKED(u_begin <= u_end && u_end <= unsigned(p.n_segs) && p.n_segs <= kAttnMaxSegs);
   // The same offset in both CTAs (the launch gives both the same dynamic
   // shared memory); a layout that does not fit is refused by both.
   const bool fits = size_t(smem - smem_raw) + kTilesBytes + kBarBytes + kStatsBytes <= size_t(kSmem);
@@ -766,7 +777,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (i == B_EO) count = 8;                    // 4 epilogue warps x 2 CTAs (rank 0's copy)
       mbar_init(&bars[i], count);
     }
-    *abort_flag = fits ? 0 : 1;
+    *abort_flag = (fits && segs_ok) ? 0 : 1;
     fence_barrier_init();
   }
   if (warp == 2) tmem_alloc_pair(tmem_holder, 512);
@@ -781,6 +792,7 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   grid_dependency_wait();
   allow_dependent_launch();
   if (threadIdx.x == 0 && !fits) record_error(p.err, kDevBadShape);
+  if (threadIdx.x == 0 && !segs_ok) record_error(p.err, kDevBounds);
   const uint32_t tmem = *tmem_holder;
   const WaitCtl w{abort_flag, p.err, p.wait_limit_ns};
   const int wg = warp >> 2;

@@ -63,6 +63,7 @@ struct StateParams {
   float corr;
   uint32_t* err;
   uint64_t wait_limit_ns;
+  int batch;                // B (the debug build checks the launch shape against it)
 };
 
 // float32 path (f32_path.cu).

@@ -17,7 +17,7 @@
 namespace arl2 {
 
 // Device error codes (the values of arl2_status they map to).
-enum : uint32_t { kDevOk = 0, kDevTimeout = 5, kDevBadShape = 2 };
+enum : uint32_t { kDevOk = 0, kDevTimeout = 5, kDevBadShape = 2, kDevBounds = 8 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -32,6 +32,22 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 __device__ __forceinline__ void record_error(uint32_t* err, uint32_t code) {
   if (err) atomicCAS(err, 0u, code);
 }
+
+// Index checks of the debug build (compiled with -DARL2_DEBUG_BOUNDS): the
+// indices a kernel takes from its parameters or its launch shape are checked
+// against the extents of the arrays they address before the access; a failed
+// check records kDevBounds in the kernel's error word and the caller skips the
+// access (and, where the access feeds other threads, stops its work in step
+// with them, so that no wait is left without its arrival for long).  In the
+// release build the checks vanish and `cond` is not evaluated.
+// ARL2_CHECKED(cond): the condition alone (true in the release build);
+// ARL2_IN_BOUNDS(err, cond): the same, recording kDevBounds when it fails.
+#ifdef ARL2_DEBUG_BOUNDS
+#define ARL2_CHECKED(cond) (cond)
+#else
+#define ARL2_CHECKED(cond) true
+#endif
+#define ARL2_IN_BOUNDS(err, cond) (ARL2_CHECKED(cond) || (::arl2::record_error((err), ::arl2::kDevBounds), false))
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -104,6 +104,9 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
   const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int slab = b * p.heads + h;
   const int rank = kFused ? int(cluster_rank_s()) : 0;
+  // (debug build) the launch is n_chunks x H x B; the test is the same for
+  // every CTA of a cluster, so a whole cluster leaves before any barrier
+  if (!ARL2_IN_BOUNDS(p.err, int(gridDim.x) == p.n_chunks && h < p.heads && b < p.batch)) return;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < P_COUNT; ++i) mbar_init(&bars[i], (i == P_KP || i == P_R) ? 4u : 1u);
@@ -442,6 +445,7 @@ state_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
 __global__ void __launch_bounds__(256) state_finalize_kernel(const StateParams p) {
   const int slab = blockIdx.x;
   const int e = (blockIdx.y * 256 + threadIdx.x) * 4;  // element index within the 128x128 state
+  if (!ARL2_IN_BOUNDS(p.err, slab < p.batch * p.heads && e + 4 <= 16384)) return;  // (debug build)
   const size_t base = size_t(slab) * 16384 + e;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   const float* part = p.partial + size_t(slab) * p.n_chunks * 16384 + e;
@@ -481,6 +485,7 @@ readout_prep_kernel(const __grid_constant__ CUtensorMap tm_s_bf, const __grid_co
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slab = blockIdx.x;
   const int h = slab % p.heads;
+  if (!ARL2_IN_BOUNDS(p.err, slab < p.batch * p.heads)) return;  // (debug build) before any barrier
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < R_COUNT; ++i) mbar_init(&bars[i], 1u);

@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(kD, 1) tok_maps_kernel(TokenParams p) {
   const int b = bh / p.H, h = bh % p.H;
   const int t0 = c * kChunk, n = min(kChunk, p.L - t0);
   const int tid = threadIdx.x, warp = tid >> 5;
+  if (!ARL2_IN_BOUNDS(p.err, bh < p.B * p.H && t0 < p.L)) return;  // (debug build) before any barrier
   if (tid == 0) {
     mbar_init(bar, 1);
     *abort_flag = 0;
@@ -303,6 +304,7 @@ __global__ void __launch_bounds__(kD, 1) tok_chunk_tc_kernel(TokenParams p) {
   __shared__ float g_all;
   const int c = blockIdx.x % p.n_chunks, bh = blockIdx.x / p.n_chunks;
   const int t0 = c * kChunk, n = min(kChunk, p.L - t0);
+  if (!ARL2_IN_BOUNDS(p.err, bh < p.B * p.H && t0 < p.L)) return;  // (debug build) before any barrier
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t lane_off = uint32_t(warp * 32) << 16;
   const size_t tok0 = size_t(bh) * p.L + t0;
@@ -506,6 +508,7 @@ __global__ void __launch_bounds__(kD) tok_state_kernel(TokenParams p) {
   float(*Ss)[kSlab] = reinterpret_cast<float(*)[kSlab]>(st_sm + 2 * kD * kD);  // [kD][kSlab]
   const int slab = blockIdx.x % (kD / kSlab), bh = blockIdx.x / (kD / kSlab);
   const int i = threadIdx.x, j0 = slab * kSlab;
+  if (!ARL2_IN_BOUNDS(p.err, bh < p.B * p.H)) return;  // (debug build)
   for (int jj = 0; jj < kSlab; ++jj) Ss[i][jj] = p.s_in[(size_t(bh) * kD + i) * kD + j0 + jj];
   copy_async_m(Mbuf, p.m + size_t(bh) * p.n_chunks * kD * kD);
   for (int c = 0; c < p.n_chunks; ++c) {
@@ -552,6 +555,7 @@ __global__ void __launch_bounds__(kD) tok_out_kernel(TokenParams p) {
   const int b = bh / p.H, h = bh % p.H;
   const int t0 = c * kChunk, n = min(kChunk, p.L - t0);
   const int j = threadIdx.x;
+  if (!ARL2_IN_BOUNDS(p.err, bh < p.B * p.H && t0 < p.L)) return;  // (debug build)
   const size_t mn0 = (size_t(bh) * p.n_chunks + c) * kD * kD;
   const size_t tok0 = size_t(bh) * p.L + t0;
   stage_rows(Sc, kD, p.s_chunk + mn0, kD, true);

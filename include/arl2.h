@@ -59,8 +59,11 @@ typedef enum {
   ARL2_ERR_CUDA = 4,             /* a CUDA runtime call or kernel launch failed */
   ARL2_ERR_TIMEOUT = 5,          /* a bounded device-side wait ran out */
   ARL2_ERR_NO_DEVICE = 6,        /* no usable CUDA device / driver */
-  ARL2_ERR_SCRATCH_LIMIT = 7     /* sizes need more than the fixed scratch of
+  ARL2_ERR_SCRATCH_LIMIT = 7,    /* sizes need more than the fixed scratch of
                                     arl2_state_write_noalloc */
+  ARL2_ERR_BOUNDS = 8            /* debug builds (libarl2_debug.so) only: a
+                                    kernel's index check failed and the access
+                                    was skipped; surfaced by arl2_last_error */
 } arl2_status;
 
 typedef enum { ARL2_F32 = 0, ARL2_BF16 = 1 } arl2_dtype;
@@ -312,14 +315,22 @@ arl2_status arl2_state_write_noalloc(const arl2_config* cfg, const void* k, cons
 arl2_status arl2_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /* y[i] = 2^x[i] (device float32 arrays of n values) through the FMA-pipe
- * exponential the attention kernel can use for part of its softmax (a degree-3
+ * exponential the attention kernel uses for part of its softmax (a degree-3
  * polynomial after rounding x to an integer; inputs clamped to [-125, 125];
- * relative error <= 1.0e-4; off in the shipped configuration, where the MUFU
- * alone measured faster).  For accuracy tests of that routine. */
+ * relative error <= 1.0e-4).  The attention kernel takes it for 3 of the 16
+ * column pairs of every 32-column chunk, in a paired form with the same
+ * operations, and the MUFU for the rest.  For accuracy tests of that routine. */
 arl2_status arl2_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
 
 const char* arl2_status_string(arl2_status s);
 int32_t arl2_abi_version(void);
+
+/* 1 in the debug build (libarl2_debug.so, kernels compiled with
+ * -DARL2_DEBUG_BOUNDS: each checks the indices it takes from its parameters and
+ * launch shape before it uses them, skips the access when a check fails and
+ * records ARL2_ERR_BOUNDS, which arl2_last_error returns), 0 in the release
+ * build (libarl2.so), whose kernels carry no such checks.  Needs no device. */
+int32_t arl2_debug_bounds_enabled(void);
 
 #ifdef __cplusplus
 }

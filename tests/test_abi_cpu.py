@@ -155,3 +155,16 @@ def test_gemm_host_validation(lib):
     assert g(a, 64, b, 64, a + 64, 64, 32, 64, 64, None) == 1         # C overlaps A
     assert g(a, 64, b, 64, c, 64, 0, 64, 64, None) == 0               # empty: nothing to do
     assert g(a, 64, b, 64, c, 64, 32, 0, 64, None) == 0
+
+
+def test_debug_build_is_flagged_and_complete(lib):
+    """libarl2_debug.so (kernels compiled with -DARL2_DEBUG_BOUNDS) reports
+    itself as the debug build, exports every declared entry point, and the
+    release library reports that it is not."""
+    from hybrid_linear_attention_arl2_b200 import build as _b
+    dbg = ctypes.CDLL(_b.build(debug_bounds=True))
+    assert dbg.arl2_debug_bounds_enabled() == 1
+    assert lib.arl2_debug_bounds_enabled() == 0
+    missing = [n for n in arl2.declared_symbols() if not hasattr(dbg, n)]
+    assert not missing, missing
+    assert arl2.arl2_status_string(8) == "a kernel index check failed (debug build)"
