@@ -23,3 +23,19 @@ def test_reference_arm_json_line():
     cb = j["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == j["value"] and cb["sample"]
     assert j["e2e"] == {"value": j["value"], "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_bench_accounting_helpers():
+    """The launch count and the traffic figure the bench line carries: one
+    state-write launch while a frame's chunks fit one cluster, three beyond;
+    traffic only for the workload the capture was taken on."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from hybrid_linear_attention_arl2_b200 import workloads as W
+    cfg1 = W.CONFIGS[1]
+    assert bench.state_launches(cfg1) == 1  # 1560 tokens: 13 chunks of 128
+    long = W.Config(99, "long", 1, 12, 128, 16 * 128 + 1, 1, 1, "bf16")
+    assert bench.state_launches(long) == 3
+    t = bench.attn_traffic(cfg1.name)
+    assert t is None or t == bench.ATTN_TRAFFIC["bytes"]
+    assert bench.attn_traffic(W.CONFIGS[4].name) is None
