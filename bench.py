@@ -385,6 +385,11 @@ def run_arl2(args, rank: int, world: int):
     result = {
         "value": value, "ms_per_step": ms_per_step, "steps": steps_done, "clocks": clk,
         "attn_avg_ms": attn_avg_ms, "flops": flops, "launches_per_step": cfg.queries + 1 + state_launches(cfg),
+        "timing": ((f"CUDA graphs of {period} frames, {n_rep} replays" + (" + " if n_tail else "") if n_rep else "")
+                   + (f"{n_tail} eager frame" + ("s" if n_tail != 1 else "") if n_tail else "")),
+        "attn_basis": (f"CUDA events before the first and after the last of one frame's {cfg.queries} back-to-back "
+                       "query launches" + (" (last graph replay)" if n_rep else " (every eager frame)")
+                       + f", span / {cfg.queries}"),
     }
     if args.config == 2 and not args.profile_small:
         result["flatness"] = long_stream_flatness(cfg, ds, device, rank)
@@ -959,14 +964,15 @@ def main():
     line = {
         "metric": metric, "value": res["value"], "unit": "frames/s", "n_gpus": world, "steps": res["steps"],
         "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config, timing=res["timing"]),
         "tokens_per_s": res["value"] * cfg.tokens * cfg.batch,
         "pct_bf16_peak": {"value": 100.0 * frame_tflops / peak_burst, "basis": f"burst bf16 {src}",
                           "sustained_basis": 100.0 * frame_tflops / peak_sus},
         "roofline": {"bound": "tensor", "kernel": "attn_pair_kernel", "achieved": attn_tflops, "peak": peak_burst,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak_burst, "traffic": attn_traffic(cfg.name),
                      "peak_basis": f"bf16_tflops (burst) {src}",
-                     "frac_vs_sustained": attn_tflops / peak_sus},
+                     "frac_vs_sustained": attn_tflops / peak_sus, "duration_basis": res["attn_basis"]},
         "clocks": res["clocks"],
         "gpu_launches": res["launches_per_step"] * res["steps"],
     }
