@@ -786,10 +786,11 @@ def cpu_oracle_rate(cfg: W.Config, budget_s: float = 12.0, sample_note=True):
 # launch on the single-hybrid-layer-bf16 workload, from one ncu capture of
 # `bench.py --profile-small --no-graphs`; reported only while the kernel sources
 # hash to the value below (None: not captured yet).  The hash is that of the
-# sources after the debug build's index checks were added: they compile away in
-# the release build, whose attention kernel compiles to the same bytes as the
-# captured sources' (cubins compared from the same path, without line tables).
-ATTN_TRAFFIC = {"bytes": 14858496 + 0, "sources_sha256": "64a10e805169f2745c15405edda715cc4a998c9877791d2c51e297d2b82a1523",
+# sources after the debug build's index checks were added and unused helpers
+# left the header: the checks compile away in the release build, whose
+# attention kernel compiles to the same bytes as the captured sources' (cubins
+# compared from the same path, without line tables).
+ATTN_TRAFFIC = {"bytes": 14858496 + 0, "sources_sha256": "e9affde710f04be4c5a6055f7795bd22b26f637b7bca31df702cc3b70b4c7cf8",
                 "workload": "single-hybrid-layer-bf16",
                 "capture": "profiles/attn_pair_kernel_single-hybrid-layer-bf16.md"}
 ATTN_SOURCES = ("hybrid_linear_attention_arl2_b200/csrc/attn_pair.cu",
