@@ -128,8 +128,9 @@ def main(argv):
     torch.device = _device_or_cpu
     from hybrid_linear_attention_arl2_b200 import arl2
     arl2.load_library = lambda *a, **k: None
-    arl2.HybridLayer = arl2.HybridBlock = Layer
-    for name in ("arl2_frame_query", "arl2_frame_commit", "arl2_block_query", "arl2_block_commit"):
+    arl2.HybridLayer = arl2.HybridBlock = arl2.KVLayer = Layer
+    for name in ("arl2_frame_query", "arl2_frame_commit", "arl2_block_query", "arl2_block_commit",
+                 "arl2_kv_query", "arl2_kv_commit", "arl2_token_query", "arl2_token_commit"):
         setattr(arl2, name, _layer_call)
     import bench
     bench.ClockSampler = _NoClocks

@@ -50,3 +50,16 @@ def test_block_bench_covers_the_pool_and_times_exactly_k_frames():
     # graphs of 8 frames (the 40-matrix pool): warm-up 3, one untimed replay,
     # 2 timed replays and 3 eager frames, 5 calls per frame
     assert calls == 5 * (3 + 8 + 2 * 8 + 3)
+
+
+@pytest.mark.parametrize("args,calls_expected", [
+    (("--config", "3", "--steps", "2", "--warmup", "1"), 3 * 5 * 30),   # warm-up frame + 2 frames, 30 layers
+    (("--token", "--steps", "3", "--warmup", "1"), None),
+    (("--profile-kv", "2", "--steps", "1", "--warmup", "1"), None),
+])
+def test_other_bench_lines_run(args, calls_expected):
+    j, calls = run(*args)
+    for k in ("metric", "value", "unit", "n_gpus", "higher_is_better", "dtype", "data", "config"):
+        assert k in j, k
+    if calls_expected is not None:
+        assert calls == calls_expected
