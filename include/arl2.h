@@ -37,7 +37,11 @@
  *     and launch errors only.  Errors raised inside kernels (a bounded wait that
  *     ran out) are recorded in the handle and returned by arl2_last_error().
  *   - A handle must not be used from two streams at once; calls on one handle
- *     execute in stream order.
+ *     execute in stream order.  The attention and projection-GEMM kernels are
+ *     launched with programmatic stream serialisation: their CTAs may start
+ *     (barrier and tensor-memory set-up only) while the kernel ahead of them
+ *     on the stream finishes, and wait for its completion before any global
+ *     memory access, so the stream's ordering of memory effects is unchanged.
  *   - No C++ exception crosses this interface.
  *   - Supported shapes: bf16 needs head_dim = 128; float32 needs head_dim <= 128
  *     and tokens_per_frame <= 4096.  Anything else returns ARL2_ERR_UNSUPPORTED.
