@@ -69,15 +69,15 @@ def _rank_main(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_gathered_shards_equal_the_whole_layer():
-    world = 2
+@pytest.mark.parametrize("world,ranges", [(2, [(0, 3), (3, 5)]), (3, [(0, 2), (2, 4), (4, 5)])])
+def test_gathered_shards_equal_the_whole_layer(world, ranges):
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, start_method="spawn", join=True)
     from oracle import arl2_oracle as o
     Q, K, V, phi, S, alpha, beta = _case()
     O, S_new = o.frame_commit(S, Q, K, V, phi, alpha, beta, 0.5)
-    assert [out[r][2] for r in range(world)] == [(0, 3), (3, 5)]  # uneven: the gather pads the smaller shard
+    assert [out[r][2] for r in range(world)] == ranges  # uneven: the gather pads the smaller shards
     for r in range(world):
         full, S_r, (h0, h1) = out[r]
         np.testing.assert_allclose(full, O, rtol=0, atol=1e-12)
