@@ -12,6 +12,7 @@ report a failed check through arl2_last_error (ARL2_ERR_BOUNDS).
 from __future__ import annotations
 
 import os
+import re
 import subprocess
 import sys
 
@@ -41,6 +42,27 @@ def _stale(lib: str = LIB) -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
+def _check_launch_registers(cmd: list, echo: bool = False) -> None:
+    """Compile the attention kernel and check that it was allocated exactly
+    the registers per thread its warp-role split (setmaxnreg) is sized for:
+    with any other count the launch is refused at run time (a larger split
+    than the launch holds would never be granted)."""
+    if "-v" not in cmd:
+        cmd = cmd + ["-Xptxas", "-v"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if echo or r.returncode != 0:
+        sys.stderr.write(r.stderr)
+    if r.returncode != 0:
+        raise subprocess.CalledProcessError(r.returncode, cmd)
+    src = open(os.path.join(CSRC, "attn_pair.cu")).read()
+    want = int(re.search(r"constexpr int kLaunchRegs = (\d+);", src).group(1))
+    m = re.search(r"Compiling entry function '[^']*attn_pair_kernel[^']*'.*?Used (\d+) registers", r.stderr, re.S)
+    if not m or int(m.group(1)) != want:
+        got = m.group(1) if m else "an unknown number of"
+        raise RuntimeError(f"attn_pair_kernel compiled to {got} registers per thread; its register split "
+                           f"needs {want}")
+
+
 def build(force: bool = False, verbose_ptxas: bool = False, debug_bounds: bool = False) -> str:
     """Build libarl2.so (or, with debug_bounds, libarl2_debug.so) when a
     source is newer than it; returns its path."""
@@ -59,7 +81,10 @@ def build(force: bool = False, verbose_ptxas: bool = False, debug_bounds: bool =
     for src in SOURCES:
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
         cmd = [nvcc()] + flags + ["-c", os.path.join(CSRC, src), "-o", obj]
-        subprocess.run(cmd, check=True)
+        if src == "attn_pair.cu":
+            _check_launch_registers(cmd, echo=verbose_ptxas)
+        else:
+            subprocess.run(cmd, check=True)
         objs.append(obj)
     tmp = lib + ".tmp"
     subprocess.run([nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"],
